@@ -1,0 +1,156 @@
+"""Seeded synthetic inputs for the MSA forward pass.
+
+This module only draws inputs; it holds none of the method's arithmetic and
+imports neither the CUDA binding nor the oracle, so both sides (and the bench)
+can take their inputs from it.
+
+Recipe (the same for every workload):
+  * one ``torch.Generator`` seeded with ``seed`` draws, in this order, Q, K, V,
+    q_idx and k_idx as standard normals in fp32, row chunk by row chunk;
+  * each tensor is multiplied by 1 (``fp32`` workloads) or by 1/sqrt(d)
+    (``bf16`` workloads, d = head_dim for Q/K/V and index_dim for the index
+    tensors) and rounded once to the workload's dtype (round to nearest even);
+  * needles: for every sequence b and group g, ``needles`` distinct "past"
+    blocks are drawn uniformly (``torch.randperm`` from the same generator, in
+    (b, g) order) from blocks ``0 .. upper-1`` where ``upper`` is the block of
+    the first query when that is > 0, else the block of the last query.  Every
+    token of a drawn block gets ``0.5 * mean_i q_idx[b, i, g, :]`` added to its
+    index key, in fp32, before k_idx is rounded to bf16 (the mean is taken over
+    the sequence's stored, already rounded q_idx rows).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    q_len: int
+    kv_len: int
+    q_pos0: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    index_dim: int
+    block_size: int
+    top_k: int
+    dtype: str          # "f32" or "bf16"
+    needles: int        # planted needle blocks per (sequence, group)
+
+    @property
+    def rows(self) -> int:
+        return self.batch * self.q_len
+
+    @property
+    def nblk(self) -> int:
+        return -(-self.kv_len // self.block_size)
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "tiny": Workload("tiny", 1, 1024, 1024, 0, 8, 2, 64, 32, 128, 4, "f32", 0),
+    "prefill_32k": Workload("prefill_32k", 1, 32768, 32768, 0, 64, 4, 128, 128, 128, 16,
+                            "bf16", 8),
+    "prefill_128k": Workload("prefill_128k", 1, 131072, 131072, 0, 64, 4, 128, 128, 128,
+                             16, "bf16", 32),
+    "decode_128k": Workload("decode_128k", 32, 1, 131072, 131071, 64, 4, 128, 128, 128,
+                            16, "bf16", 32),
+    "chunk_1m": Workload("chunk_1m", 1, 8192, 1048576, 1040384, 64, 4, 128, 128, 128, 16,
+                         "bf16", 64),
+}
+
+_CHUNK_ELEMS = 1 << 24
+
+
+def _draw(gen: torch.Generator, shape, scale: float, dtype: torch.dtype) -> torch.Tensor:
+    """Standard normals drawn in fp32 row chunk by row chunk, scaled, rounded."""
+    out = torch.empty(shape, dtype=dtype)
+    flat = out.view(shape[0], -1)
+    per_row = flat.shape[1]
+    step = max(1, _CHUNK_ELEMS // max(per_row, 1))
+    for r0 in range(0, flat.shape[0], step):
+        r1 = min(flat.shape[0], r0 + step)
+        x = torch.randn((r1 - r0, per_row), generator=gen, dtype=torch.float32)
+        if scale != 1.0:
+            x.mul_(scale)
+        flat[r0:r1] = x.to(dtype)
+    return out
+
+
+def needle_upper(w: Workload) -> int:
+    first = w.q_pos0 // w.block_size
+    return first if first > 0 else (w.q_pos0 + w.q_len - 1) // w.block_size
+
+
+def make_inputs(w: Workload, seed: int = 0) -> Dict[str, torch.Tensor]:
+    """Inputs of workload ``w`` on the CPU: q, k, v, q_idx, k_idx (+ needle ids)."""
+    gen = torch.Generator().manual_seed(seed)
+    dt = w.torch_dtype
+    s_main = 1.0 if w.dtype == "f32" else 1.0 / math.sqrt(w.head_dim)
+    s_idx = 1.0 if w.dtype == "f32" else 1.0 / math.sqrt(w.index_dim)
+    B, Sq, Skv = w.batch, w.q_len, w.kv_len
+    q = _draw(gen, (B * Sq, w.num_q_heads, w.head_dim), s_main, dt)
+    k = _draw(gen, (B * Skv, w.num_kv_heads, w.head_dim), s_main, dt)
+    v = _draw(gen, (B * Skv, w.num_kv_heads, w.head_dim), s_main, dt)
+    q_idx = _draw(gen, (B * Sq, w.num_kv_heads, w.index_dim), s_idx, dt)
+    # k_idx stays fp32 until the needles are in, then is rounded once.
+    k_idx32 = _draw(gen, (B * Skv, w.index_dim), s_idx, torch.float32)
+    needle_ids = torch.full((B, w.num_kv_heads, max(w.needles, 0)), -1, dtype=torch.int64)
+    if w.needles > 0:
+        upper = needle_upper(w)
+        if upper < w.needles:
+            raise ValueError(f"{w.name}: only {upper} past blocks for {w.needles} needles")
+        qi = q_idx.view(B, Sq, w.num_kv_heads, w.index_dim)
+        kv = k_idx32.view(B, Skv, w.index_dim)
+        for b in range(B):
+            for g in range(w.num_kv_heads):
+                blocks = torch.randperm(upper, generator=gen)[: w.needles]
+                needle_ids[b, g] = blocks
+                shift = 0.5 * qi[b, :, g, :].float().mean(dim=0)
+                for c in blocks.tolist():
+                    lo = c * w.block_size
+                    hi = min(lo + w.block_size, Skv)
+                    kv[b, lo:hi] += shift
+    k_idx = k_idx32.to(dt)
+    return {
+        "q": q.view(B, Sq, w.num_q_heads, w.head_dim),
+        "k": k.view(B, Skv, w.num_kv_heads, w.head_dim),
+        "v": v.view(B, Skv, w.num_kv_heads, w.head_dim),
+        "q_idx": q_idx.view(B, Sq, w.num_kv_heads, w.index_dim),
+        "k_idx": k_idx.view(B, Skv, w.index_dim),
+        "needles": needle_ids,
+    }
+
+
+def sample_rows(w: Workload, n: int, seed: int = 0) -> list:
+    """``n`` query rows spread evenly over positions, with a seeded jitter.
+
+    Always includes the first and the last row of the batch.
+    """
+    R = w.rows
+    if n >= R:
+        return list(range(R))
+    gen = torch.Generator().manual_seed(seed + 1)
+    base = torch.linspace(0, R - 1, n).long()
+    jitter = torch.randint(-3, 4, (n,), generator=gen)
+    rows = (base + jitter).clamp(0, R - 1)
+    rows[0] = 0
+    rows[-1] = R - 1
+    return sorted(set(rows.tolist()))
+
+
+def scaled(w: Workload, name: Optional[str] = None, **kw) -> Workload:
+    """A smaller test case with the same structure as ``w``."""
+    return w.with_(name=name or (w.name + "_scaled"), **kw)

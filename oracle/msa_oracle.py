@@ -1,0 +1,304 @@
+"""Plain, slow fp64 CPU oracle of the MiniMax Sparse Attention (MSA) forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import or call
+this module.  The product path (the CUDA library and its Python binding) never
+does, and this module imports nothing from the product package: the two share
+no code.  Inputs are NumPy arrays (or anything ``np.asarray`` accepts) holding
+the exact stored values (fp32, or bf16 values widened to fp32); every
+computation below runs in float64.
+
+Sources (page title, then section):
+  [HF]  "Substantial numerical differences with Minimax MSA attention vs
+        Minimax's Reference" (digest of huggingface/transformers issue 46762),
+        sections "原因分析" (cause analysis), "解决步骤" (fix steps),
+        "验证方法" (verification).
+  [ABS] "MiniMax 稀疏注意力" (hyper.ai page of paper 2606.13392), sections
+        "摘要" (abstract), "核心贡献" (contributions), "引言" (introduction).
+  [DK]  "MiniMax lancerer MSA: blok-sparse attention ..." (snilld.dk), sections
+        "Hvad er MSA i praksis", "Teknisk forklaring hvorfor kompleksiteten
+        skifter".
+  [HU]  "MiniMax új eljárása 28-szorosára csökkenti az AI-figyelem számítási
+        igényét" (aiforradalom.online), section "Hogyan működik az indexelő és
+        a fő ág?".
+
+Layouts (token-major, as in [HF] "原因分析": the per-head selection is
+``[total_qo_len, heads, topk]`` and the kernel list is
+``q2k[num_kv_heads, bsz*q_len, topk]``):
+  q      [B, Sq, Hq, D]        k, v   [B, Skv, Hkv, D]
+  q_idx  [B, Sq, Hkv, di]      k_idx  [B, Skv, di]   (one shared index-key head)
+  q2k    [Hkv, B*Sq, top_k]    int, ascending block ids, -1 padded
+Query row ``r = b*Sq + i`` sits at absolute position ``t = q_pos0 + i`` and may
+see keys ``0..t`` of its own sequence.  Query head ``h`` belongs to GQA group
+``g = h // (Hq // Hkv)`` ([HF] "解决步骤": the mask is expanded per index head
+with ``repeat_interleave(num_q_heads // H_idx)``, so the heads of one group are
+adjacent).
+
+Readings taken where the pages leave a step open (each is also listed in the
+design notes of the repository):
+  R1  the index score is the raw dot product q_idx . k_idx: no scale, no
+      activation ([DK] "Teknisk forklaring": raw scores are ranked).
+  R2  a block's score is the max over its causally visible tokens only.
+  R3  the forced local block counts inside top_k.
+  R4  ties between equal block scores go to the lower block index.
+  R5  a row that sees fewer than top_k blocks selects all of them.
+  R6  the selected ids are returned in ascending order, -1 padded.
+  R7  main-branch scale is 1/sqrt(head_dim) ([DK] "scaled dot-product").
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional, Sequence
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+def _f64(x) -> np.ndarray:
+    """Widen an input to float64 without changing its value."""
+    if hasattr(x, "detach"):  # a torch tensor given by a test
+        x = x.detach().float().cpu().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _rows(batch: int, q_len: int, rows: Optional[Iterable[int]]) -> list:
+    return list(range(batch * q_len)) if rows is None else [int(r) for r in rows]
+
+
+# ---------------------------------------------------------------------------
+# Index branch
+# ---------------------------------------------------------------------------
+
+def index_scores_row(q_vec, k_idx_seq, t: int) -> np.ndarray:
+    """Token scores s_j = q_vec . k_idx_seq[j] for every visible key j = 0..t.
+
+    [DK] "Hvad er MSA i praksis" and [HU] "Hogyan működik...": one index-query
+    head per GQA group is scored against the single shared index-key head over
+    the causally visible key tokens.  Reading R1: the raw dot product.
+    """
+    return _f64(k_idx_seq)[: t + 1] @ _f64(q_vec)
+
+
+def block_maxima_row(scores: np.ndarray, block_size: int) -> np.ndarray:
+    """Max-pool visible token scores into blocks of ``block_size`` tokens.
+
+    [HF] "原因分析": ``scores.amax(dim=-1)`` pools inside each 128-token block.
+    Reading R2: only the visible tokens of the last (local) block take part, so
+    ``scores`` (length t+1) is cut at t.  Returns the maxima of blocks
+    0..floor(t/block_size).
+    """
+    n = scores.shape[0]
+    nvis = (n - 1) // block_size + 1
+    out = np.empty(nvis, dtype=np.float64)
+    for c in range(nvis):
+        out[c] = scores[c * block_size: min((c + 1) * block_size, n)].max()
+    return out
+
+
+def select_row(block_max: np.ndarray, t: int, block_size: int, top_k: int) -> np.ndarray:
+    """Exp-free top-k block selection of one (query, GQA group) row.
+
+    [DK] "Hvad er MSA i praksis": each query keeps k blocks per GQA group and the
+    query's own block is always among them.  [DK] "Teknisk forklaring": softmax
+    keeps the ranking, so raw block scores are ranked (no exponential).
+    [HF] "解决步骤": the local-block boost and top-k are applied per index head.
+    Readings R3-R6: the local block counts inside k; the other k-1 slots go to
+    the highest-scoring earlier blocks, ties to the lower index; a row with fewer
+    than k visible blocks takes all of them; ids ascending, -1 padded.
+    """
+    c_t = t // block_size
+    nvis = c_t + 1
+    ksel = min(top_k, nvis)
+    earlier = sorted(range(c_t), key=lambda c: (-block_max[c], c))
+    chosen = sorted([c_t] + earlier[: ksel - 1])
+    return np.array(chosen + [-1] * (top_k - ksel), dtype=np.int64)
+
+
+def block_scores(q_idx, k_idx, q_pos0: int, block_size: int,
+                 rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """Block maxima ``bmax[g, r, c]`` for every row r (or the given rows).
+
+    Blocks c > floor(t/block_size) are not visible to row r and hold -inf.
+    Shape ``[Hkv, B*Sq, nblk]`` with ``nblk = ceil(Skv / block_size)``; rows
+    not requested stay NaN.
+    """
+    qi = _f64(q_idx)
+    ki = _f64(k_idx)
+    B, Sq, Hkv, _ = qi.shape
+    nblk = -(-ki.shape[1] // block_size)
+    out = np.full((Hkv, B * Sq, nblk), np.nan)
+    for r in _rows(B, Sq, rows):
+        b, i = divmod(r, Sq)
+        t = q_pos0 + i
+        # all groups at once: [t+1, di] @ [di, Hkv]
+        s = ki[b, : t + 1] @ qi[b, i].T
+        out[:, r, :] = NEG_INF
+        for g in range(Hkv):
+            m = block_maxima_row(s[:, g], block_size)
+            out[g, r, : m.shape[0]] = m
+    return out
+
+
+def select(q_idx, k_idx, q_pos0: int, block_size: int, top_k: int,
+           rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """Per-(query, GQA group) selection ``q2k[Hkv, B*Sq, top_k]`` (int64).
+
+    Rows not requested are filled with -2 (never a valid output value).
+    """
+    qi = _f64(q_idx)
+    B, Sq, Hkv, _ = qi.shape
+    bm = block_scores(q_idx, k_idx, q_pos0, block_size, rows)
+    q2k = np.full((Hkv, B * Sq, top_k), -2, dtype=np.int64)
+    for r in _rows(B, Sq, rows):
+        t = q_pos0 + r % Sq
+        for g in range(Hkv):
+            q2k[g, r] = select_row(bm[g, r], t, block_size, top_k)
+    return q2k
+
+
+# ---------------------------------------------------------------------------
+# Main branch
+# ---------------------------------------------------------------------------
+
+def attend_row(q_heads, k_seq_g, v_seq_g, blocks, t: int, block_size: int,
+               scale: float):
+    """Exact softmax attention of one query row's heads of one GQA group.
+
+    [DK] "Hvad er MSA i praksis": the main branch gathers the causally visible
+    tokens of the selected blocks and runs scaled dot-product softmax over
+    exactly those tokens; all query heads of the group share the block set.
+    Returns (o [G, D], lse [G]) with lse the natural log of the softmax
+    normaliser of the scaled logits.
+    """
+    keys = []
+    for c in blocks:
+        if c < 0:
+            continue
+        lo = c * block_size
+        hi = min((c + 1) * block_size, t + 1)
+        keys.extend(range(lo, hi))
+    J = np.array(sorted(keys), dtype=np.int64)
+    K = _f64(k_seq_g)[J]          # [n, D]
+    V = _f64(v_seq_g)[J]
+    z = scale * (_f64(q_heads) @ K.T)  # [G, n]
+    m = z.max(axis=1, keepdims=True)
+    w = np.exp(z - m)
+    l = w.sum(axis=1, keepdims=True)
+    o = (w / l) @ V
+    lse = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+def attend(q, k, v, q2k, q_pos0: int, block_size: int,
+           scale: Optional[float] = None, rows: Optional[Sequence[int]] = None):
+    """Main branch over a given selection: returns (out [B,Sq,Hq,D], lse [B,Sq,Hq]).
+
+    Unrequested rows stay NaN.  ``scale`` defaults to 1/sqrt(D) (reading R7).
+    """
+    qf = _f64(q)
+    B, Sq, Hq, D = qf.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    sel = np.asarray(q2k)
+    out = np.full((B, Sq, Hq, D), np.nan)
+    lse = np.full((B, Sq, Hq), np.nan)
+    kf = _f64(k)
+    vf = _f64(v)
+    for r in _rows(B, Sq, rows):
+        b, i = divmod(r, Sq)
+        t = q_pos0 + i
+        for g in range(Hkv):
+            hs = slice(g * G, (g + 1) * G)
+            o, ls = attend_row(qf[b, i, hs], kf[b, :, g], vf[b, :, g], sel[g, r],
+                               t, block_size, scale)
+            out[b, i, hs] = o
+            lse[b, i, hs] = ls
+    return out, lse
+
+
+def forward(q, k, v, q_idx, k_idx, q_pos0: int, block_size: int, top_k: int,
+            scale: Optional[float] = None, rows: Optional[Sequence[int]] = None):
+    """Index branch then main branch ([ABS] "摘要"; [DK] "Hvad er MSA i praksis").
+
+    Returns (out, lse, q2k).
+    """
+    q2k = select(q_idx, k_idx, q_pos0, block_size, top_k, rows)
+    out, lse = attend(q, k, v, q2k, q_pos0, block_size, scale, rows)
+    return out, lse, q2k
+
+
+# ---------------------------------------------------------------------------
+# Independent references used by the pins
+# ---------------------------------------------------------------------------
+
+def dense_causal_gqa(q, k, v, q_pos0: int, scale: Optional[float] = None,
+                     rows: Optional[Sequence[int]] = None):
+    """Dense causal GQA attention written directly from its definition.
+
+    Query head h reads KV head h // (Hq // Hkv) over keys 0..t.  This is what MSA
+    must equal when top_k * block_size covers every visible key.
+    """
+    qf, kf, vf = _f64(q), _f64(k), _f64(v)
+    B, Sq, Hq, D = qf.shape
+    Hkv = kf.shape[2]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = np.full((B, Sq, Hq, D), np.nan)
+    lse = np.full((B, Sq, Hq), np.nan)
+    for r in _rows(B, Sq, rows):
+        b, i = divmod(r, Sq)
+        t = q_pos0 + i
+        for h in range(Hq):
+            kv = h // G
+            z = scale * (kf[b, : t + 1, kv] @ qf[b, i, h])
+            m = z.max()
+            w = np.exp(z - m)
+            out[b, i, h] = (w @ vf[b, : t + 1, kv]) / w.sum()
+            lse[b, i, h] = m + math.log(w.sum())
+    return out, lse
+
+
+def pooled_select(q_idx, k_idx, q_pos0: int, block_size: int, top_k: int) -> np.ndarray:
+    """The pooled selection that [HF] "原因分析" reports as the bug.
+
+    Block scores are maxed over the index-head axis (``.amax(dim=1)``) so every
+    group shares one selection.  Kept only as a negative control for the tests;
+    returns ``[B*Sq, top_k]``.
+    """
+    bm = block_scores(q_idx, k_idx, q_pos0, block_size)
+    pooled = bm.max(axis=0)
+    Sq = _f64(q_idx).shape[1]
+    return np.stack([select_row(pooled[r], q_pos0 + r % Sq, block_size, top_k)
+                     for r in range(pooled.shape[0])])
+
+
+def selection_metrics(sel_a: np.ndarray, sel_b: np.ndarray) -> dict:
+    """The three selection metrics of [HF] "验证方法".
+
+    ``sel_a`` and ``sel_b`` are ``[Hkv, R, k]`` (-1 padded).  Returns the number
+    of (row, group) selections that differ, the mean per-(row, group) overlap
+    and, for each side, the mean number of distinct blocks one (token, group)
+    reaches.
+    """
+    a = np.asarray(sel_a)
+    b = np.asarray(sel_b)
+    Hkv, R, _ = a.shape
+    differ = 0
+    overlap = 0
+    dist_a = 0
+    dist_b = 0
+    for g in range(Hkv):
+        for r in range(R):
+            sa = set(int(x) for x in a[g, r] if x >= 0)
+            sb = set(int(x) for x in b[g, r] if x >= 0)
+            differ += int(sa != sb)
+            overlap += len(sa & sb)
+            dist_a += len(sa)
+            dist_b += len(sb)
+    n = Hkv * R
+    return {"divergent": differ, "total": n, "mean_overlap": overlap / n,
+            "distinct_a": dist_a / n, "distinct_b": dist_b / n}
