@@ -1,0 +1,521 @@
+"""Throughput of the MSA forward hot path on B200: 128K prefill query-tokens/s
+(plus 128K decode tokens/s), with the roofline fraction of the dominant kernel
+and of the whole path, an end-to-end number through the public API with host
+buffers, and the fp64 CPU oracle timed on the host cores as a baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
+
+Under torchrun each rank runs its own independent problem (weak scaling, no
+collective on the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import multiprocessing as mp
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_gqa_04_b200.workload import WORKLOADS, Workload, make_inputs, sample_rows  # noqa: E402
+
+METRIC = "128K prefill query-tokens/s & decode tok/s on 1 B200; % tensor/HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+# ---------------------------------------------------------------------------
+# algorithmic counts
+# ---------------------------------------------------------------------------
+
+def positions(w: Workload) -> np.ndarray:
+    return (w.q_pos0 + np.arange(w.q_len, dtype=np.int64))
+
+
+def counts(w: Workload) -> dict:
+    """Algorithmic work of one forward, from the definitions of the method."""
+    t = positions(w)
+    c_t = t // w.block_size
+    ksel = np.minimum(w.top_k, c_t + 1)
+    B = w.batch
+    vis_keys = float(B * np.sum(t + 1))
+    sel_blocks = float(B * np.sum(ksel))           # per group
+    index_flops = 2.0 * w.index_dim * w.num_kv_heads * vis_keys
+    main_flops = 4.0 * w.head_dim * w.num_q_heads * w.block_size * sel_blocks
+    esz = 4 if w.dtype == "f32" else 2
+    kidx_bytes = float(B * w.kv_len * w.index_dim * esz)
+    bmax_read = float(B * w.num_kv_heads * np.sum(c_t) * 4)
+    partial_bytes = float(w.num_q_heads * sel_blocks * (w.head_dim * esz + 4))
+    out_bytes = float(w.rows * w.num_q_heads * w.head_dim * esz)
+    return {"index_flops": index_flops, "main_flops": main_flops, "kidx_bytes": kidx_bytes,
+            "bmax_read_bytes": bmax_read, "partial_bytes": partial_bytes,
+            "out_bytes": out_bytes, "sel_blocks_per_group": sel_blocks,
+            "q2k_bytes": float(w.num_kv_heads * w.rows * w.top_k * 4)}
+
+
+def selected_kv_bytes(w: Workload, q2k: torch.Tensor) -> float:
+    """K and V bytes of the distinct (sequence, group, block) triples selected."""
+    Hkv, T, k = q2k.shape
+    b = (torch.arange(T, device=q2k.device) // w.q_len).view(1, T, 1)
+    g = torch.arange(Hkv, device=q2k.device).view(Hkv, 1, 1)
+    key = (b.to(torch.int64) * Hkv + g) * w.nblk + q2k.to(torch.int64)
+    key = key[q2k >= 0]
+    n = int(torch.unique(key).numel())
+    esz = 4 if w.dtype == "f32" else 2
+    return float(n) * w.block_size * w.head_dim * esz * 2
+
+
+def load_peaks() -> tuple:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        if shutil.which("nvidia-smi"):
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self) -> dict:
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9 and p[1].isdigit():
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [int(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": int(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+
+
+# ---------------------------------------------------------------------------
+# oracle on the host cores (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+class RowStore:
+    """Query-side tensors of a few rows behind the [B, Sq, ...] indexing the
+    oracle uses (only the sampled rows are ever read)."""
+
+    def __init__(self, full_shape, rows_np: dict):
+        self.shape = full_shape
+        self._rows = rows_np
+
+    def __getitem__(self, idx):
+        b, i = idx[0], idx[1]
+        x = self._rows[(int(b), int(i))]
+        return x[idx[2:]] if len(idx) > 2 else x
+
+
+_W = {}
+_THREAD_VARS = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+
+
+def _oracle_worker_init(files: dict, meta: dict):
+    _W["k"] = np.load(files["k"], mmap_mode="r")
+    _W["v"] = np.load(files["v"], mmap_mode="r")
+    _W["k_idx"] = np.load(files["k_idx"], mmap_mode="r")
+    _W["meta"] = meta
+
+
+def _oracle_rows(task):
+    from oracle import msa_oracle as O
+    rows, qrows, qirows = task
+    m = _W["meta"]
+    q = RowStore(tuple(m["q_shape"]), qrows)
+    qi = RowStore(tuple(m["qi_shape"]), qirows)
+    O.forward(q, _W["k"], _W["v"], qi, _W["k_idx"], m["q_pos0"], m["block_size"], m["top_k"],
+              rows=rows)
+    return len(rows)
+
+
+def time_oracle(w: Workload, x: dict, n_rows: int, seed: int = 0) -> dict:
+    """Times the oracle forward on ``n_rows`` evenly spread rows with a spawn
+    pool over all host cores and extrapolates to the whole workload."""
+    cores = len(os.sched_getaffinity(0))
+    rows = sample_rows(w, n_rows, seed)
+    tmp = tempfile.mkdtemp(prefix="msa_oracle_")
+    files = {}
+    try:
+        for name in ("k", "v", "k_idx"):
+            files[name] = os.path.join(tmp, name + ".npy")
+            np.save(files[name], x[name].float().cpu().numpy())
+        qrows, qirows = {}, {}
+        qc, qic = x["q"], x["q_idx"]
+        for r in rows:
+            b, i = divmod(r, w.q_len)
+            qrows[(b, i)] = qc[b, i].float().cpu().numpy()
+            qirows[(b, i)] = qic[b, i].float().cpu().numpy()
+        meta = {"q_shape": list(x["q"].shape), "qi_shape": list(x["q_idx"].shape),
+                "q_pos0": w.q_pos0, "block_size": w.block_size, "top_k": w.top_k}
+        nproc = max(1, min(cores, len(rows)))
+        chunks = [rows[i::nproc] for i in range(nproc)]
+        tasks = [(c, {(divmod(r, w.q_len)): qrows[divmod(r, w.q_len)] for r in c},
+                  {(divmod(r, w.q_len)): qirows[divmod(r, w.q_len)] for r in c}) for c in chunks]
+        ctx = mp.get_context("spawn")
+        # one BLAS thread per worker process: the pool already uses every core
+        saved = {k: os.environ.get(k) for k in _THREAD_VARS}
+        os.environ.update({k: "1" for k in _THREAD_VARS})
+        try:
+            pool = ctx.Pool(nproc, initializer=_oracle_worker_init, initargs=(files, meta))
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        with pool:
+            pool.map(_oracle_rows, [(c[:1], t1, t2) for c, t1, t2 in tasks])  # warm imports
+            t0 = time.perf_counter()
+            done = sum(pool.map(_oracle_rows, tasks))
+            wall = time.perf_counter() - t0
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+    # rows are spread evenly over positions, so their mean cost is the workload's
+    full = wall * w.rows / done
+    return {"value": w.rows / full, "unit": "query-tokens/s", "cores": nproc,
+            "kind": "oracle", "sample_wall_s": wall,
+            "sample": f"{done} of {w.rows} query rows of {w.name} spread evenly over positions "
+                      f"(fp64 NumPy oracle, spawn pool of {nproc} processes); whole-workload "
+                      f"time extrapolated as wall * rows / sampled rows"}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def _events(n):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in ev:
+        e.record()  # materialise the underlying CUDA event
+    return ev
+
+
+def run_steps(msa, w, x, ws, out, steps, warmup, stage_timing=True):
+    """Warm-up, then exactly ``steps`` timed forwards.  Returns (ms/step, stage ms)."""
+    kw = dict(q_pos0=w.q_pos0, block_size=w.block_size, top_k=w.top_k, workspace=ws, out=out)
+    for _ in range(warmup):
+        msa.forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], **kw)
+    per = [(_events(1)[0], _events(5)) for _ in range(steps)] if stage_timing else []
+    start, end = _events(2)
+    torch.cuda.synchronize()
+    start.record()
+    for s in range(steps):
+        if stage_timing:
+            per[s][0].record()
+            msa.set_stage_events(per[s][1])
+        msa.forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], **kw)
+    end.record()
+    msa.set_stage_events(None)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    stage = {}
+    if stage_timing:
+        for i, name in enumerate(msa.STAGES):
+            tot = 0.0
+            for s0, evs in per:
+                prev = s0 if i == 0 else evs[i - 1]
+                tot += prev.elapsed_time(evs[i])
+            stage[name] = tot / steps
+    return ms, stage
+
+
+def run_e2e(msa, w, xh, out_h, steps, warmup):
+    """Same metric through the public API with pinned host buffers: every step
+    copies its inputs host->device and its output device->host."""
+    kw = dict(q_pos0=w.q_pos0, block_size=w.block_size, top_k=w.top_k, out=out_h)
+    for _ in range(warmup):
+        msa.forward(xh["q"], xh["k"], xh["v"], xh["q_idx"], xh["k_idx"], **kw)
+    torch.cuda.synchronize()
+    start, end = _events(2)
+    start.record()
+    for _ in range(steps):
+        msa.forward(xh["q"], xh["k"], xh["v"], xh["q_idx"], xh["k_idx"], **kw)
+    end.record()
+    torch.cuda.synchronize()
+    h2d = sum(xh[n].numel() * xh[n].element_size() for n in ("q", "k", "v", "q_idx", "k_idx"))
+    d2h = out_h.numel() * out_h.element_size()
+    return start.elapsed_time(end) / steps, h2d, d2h
+
+
+def kernel_roofline(w, cnt, stage_ms, path, peaks, kv_sel_bytes, sustained=True):
+    """Roofline entry of the slowest stage of the step."""
+    name = max(stage_ms, key=stage_ms.get)
+    ms = stage_ms[name]
+    tflops_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    alu_peak = SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    if name == "index":
+        tc = "index:tc" in path
+        bound, unit, work = ("tensor" if tc else "alu"), "TFLOP/s", cnt["index_flops"]
+        peak = tflops_peak if tc else alu_peak
+        achieved = work / (ms * 1e-3) / 1e12
+    elif name == "attn":
+        tc = "attn:tc" in path
+        bound, unit, work = ("tensor" if tc else "alu"), "TFLOP/s", cnt["main_flops"]
+        peak = tflops_peak if tc else alu_peak
+        achieved = work / (ms * 1e-3) / 1e12
+    else:
+        bound, unit = "hbm", "GB/s"
+        work = {"topk": cnt["bmax_read_bytes"] + cnt["q2k_bytes"],
+                "lists": 3 * cnt["q2k_bytes"],
+                "combine": cnt["partial_bytes"] + cnt["out_bytes"] + cnt["q2k_bytes"]}[name]
+        peak = peaks["hbm_gbs"]
+        achieved = work / (ms * 1e-3) / 1e9
+    return {"kernel": name, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+            "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+            "ms": round(ms, 4), "algorithmic_per_launch": work,
+            "peak_kind": "sustained" if (bound == "tensor" and sustained) else
+                         ("derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock" if bound == "alu"
+                          else "measured")}
+
+
+def path_roofline(cnt, kv_sel_bytes, ms, peaks):
+    F = cnt["index_flops"] + cnt["main_flops"]
+    Bytes = cnt["kidx_bytes"] + kv_sel_bytes
+    t_tensor = F / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = Bytes / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_tensor, t_hbm)
+    return {"flops": F, "bytes": Bytes, "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+            "t_roofline_ms": round(t_roof * 1e3, 4), "t_measured_ms": round(ms, 4),
+            "frac": round(t_roof * 1e3 / ms, 4),
+            "note": "roofline = max(index+main FLOPs / bf16 burst peak, (k_idx + distinct "
+                    "selected K/V bytes) / HBM peak)"}
+
+
+def measure_workload(msa, w, dev, steps, warmup, peaks, with_e2e):
+    x = make_inputs(w, seed=0, device=dev)
+    x.pop("needles")
+    p = msa.problem_of(w)
+    path = msa.kernel_path(p)
+    ws = msa.new_workspace(p, msa.OP_FORWARD, dev)
+    out = torch.empty_like(x["q"])
+    _, q2k = msa.forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], q_pos0=w.q_pos0,
+                         block_size=w.block_size, top_k=w.top_k, workspace=ws, return_q2k=True)
+    kv_sel = selected_kv_bytes(w, q2k)
+    del q2k
+    cnt = counts(w)
+    idx = dev.index if dev.index is not None else 0
+    with ClockSampler(idx) as clk:
+        ms, stage = run_steps(msa, w, x, ws, out, steps, warmup)
+    res = {"w": w, "ms": ms, "stage": stage, "path": path, "cnt": cnt, "kv_sel": kv_sel,
+           "clocks": clk.summary(), "launches": msa.launch_count(p) * steps, "x": x}
+    if with_e2e:
+        xh = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "q_idx", "k_idx")}
+        del ws
+        torch.cuda.empty_cache()
+        out_h = torch.empty(x["q"].shape, dtype=x["q"].dtype).pin_memory()
+        e_ms, h2d, d2h = run_e2e(msa, w, xh, out_h, max(1, steps // 2), 1)
+        res["e2e"] = (e_ms, h2d, d2h)
+    return res
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    """Largest per-rank value (step time) over all ranks; the same on every rank."""
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(rows_per_rank: int, ms_local: float, world: int) -> tuple:
+    """Whole-job throughput of independent per-rank problems: every rank's rows
+    divided by the slowest rank's step time.  Returns (value, max ms)."""
+    ms = max_over_ranks(ms_local, world)
+    return world * rows_per_rank / (ms * 1e-3), ms
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
+    ap.add_argument("--workload", default="prefill_128k", choices=list(WORKLOADS))
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows (0 = auto)")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    w = WORKLOADS[a.workload]
+    peaks, peak_src = load_peaks()
+
+    if a.impl == "reference":
+        # the reference arm is the fp64 oracle on the host cores, rank 0 only
+        if rank != 0:
+            barrier(world)
+            return
+        dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+        x = make_inputs(w, seed=0, device=dev)
+        n_rows = a.cpu_rows or (64 if w.q_len > 1 else w.rows)
+        vals = [time_oracle(w, x, n_rows, seed=s) for s in range(a.warmup + a.steps)]
+        timed = vals[a.warmup:]
+        v = statistics.mean(t["value"] for t in timed)
+        ms = w.rows / v * 1e3
+        cb = dict(timed[-1])
+        cb["value"] = v
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "query-tokens/s",
+                "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.name, "batch": w.batch, "q_len": w.q_len,
+                           "kv_len": w.kv_len, "q_pos0": w.q_pos0, "top_k": w.top_k},
+                "cpu_baseline": cb,
+                "e2e": {"value": v, "unit": "query-tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+                "gpu_launches": 0}
+        print(json.dumps(line), flush=True)
+        barrier(world)
+        return
+
+    from block_sparse_gqa_04_b200 import msa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    msa.load()
+    barrier(world)
+    main_res = measure_workload(msa, w, dev, a.steps, a.warmup, peaks, not a.no_e2e)
+    value, ms = weak_value(w.rows, main_res["ms"], world)
+    cnt = main_res["cnt"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1/d) inputs with planted needle blocks)",
+        "config": {"workload": w.name, "batch": w.batch, "q_len": w.q_len, "kv_len": w.kv_len,
+                   "q_pos0": w.q_pos0, "num_q_heads": w.num_q_heads,
+                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                   "index_dim": w.index_dim, "block_size": w.block_size, "top_k": w.top_k,
+                   "parallelism": f"replicas x{world} (independent problems)",
+                   "kernel_path": main_res["path"],
+                   "l2": "inputs larger than L2 (q alone is %.2f GB per step)" %
+                         (main_res["x"]["q"].numel() * 2 / 1e9)},
+        "clocks": main_res["clocks"],
+        "gpu_launches": main_res["launches"],
+        "stage_ms": {k: round(v, 4) for k, v in main_res["stage"].items()},
+        "roofline": kernel_roofline(w, cnt, main_res["stage"], main_res["path"], peaks,
+                                    main_res["kv_sel"]),
+        "path_roofline": path_roofline(cnt, main_res["kv_sel"], ms, peaks),
+        "peaks": {"source": peak_src, "hbm_gbs": peaks["hbm_gbs"],
+                  "bf16_tflops": peaks["bf16_tflops"],
+                  "bf16_tflops_sustained": peaks.get("bf16_tflops_sustained")},
+    }
+    if "e2e" in main_res:
+        e_ms, h2d, d2h = main_res["e2e"]
+        e_val, e_ms = weak_value(w.rows, e_ms, world)
+        line["e2e"] = {"value": e_val, "unit": "query-tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": e_ms}
+    x_main = main_res.pop("x")
+    if not a.no_decode:
+        wd = WORKLOADS["decode_128k"]
+        del x_main
+        torch.cuda.empty_cache()
+        dres = measure_workload(msa, wd, dev, a.steps, a.warmup, peaks, False)
+        dval, dms = weak_value(wd.rows, dres["ms"], world)
+        dcnt = dres["cnt"]
+        dbytes = dcnt["kidx_bytes"] + dres["kv_sel"]
+        line["decode"] = {
+            "workload": wd.name, "value": dval, "unit": "tokens/s",
+            "ms_per_step": dms, "kernel_path": dres["path"],
+            "stage_ms": {k: round(v, 4) for k, v in dres["stage"].items()},
+            "hbm_roofline": {"bytes": dbytes, "t_roofline_ms": dbytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
+                             "achieved_gbs": dbytes / (dms * 1e-3) / 1e9,
+                             "frac": dbytes / (peaks["hbm_gbs"] * 1e9) / (dms * 1e-3)},
+            "clocks": dres["clocks"]}
+        dres.pop("x")
+        x_main = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        # the oracle runs on host copies of the bench's own inputs
+        xm = make_inputs(w, seed=0, device=dev)
+        xm.pop("needles")
+        n_rows = a.cpu_rows or 256
+        line["cpu_baseline"] = time_oracle(w, xm, n_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,346 @@
+// Index branch on tcgen05 tensor cores: block maxima of the raw index scores
+// q_idx . k_idx with the causal mask and the 128-token max-pool fused into the
+// epilogue, so no token score ever reaches HBM ("Substantial numerical
+// differences with Minimax MSA attention vs Minimax's Reference", section
+// 原因分析: amax over each block, per index head; snilld.dk "Hvad er MSA i
+// praksis": one index-query head per GQA group, one shared index-key head).
+//
+// Shapes: bf16, index_dim 128, block 128, up to 4 groups.  One persistent CTA
+// per SM walks a contiguous share of the (sequence, 128-row query tile, key
+// block) triples that the causal mask leaves (triangle order, so every CTA gets
+// the same number of tiles).  For each triple and each group one MMA unit
+// computes S[128 queries x 128 keys] = q_idx_g . k_idx_block^T in fp32:
+//   * TMEM lanes are query rows.  The index queries of the current query tile
+//     (all groups, 128 x 128 bf16 each) sit in TMEM columns 0..255 as the A
+//     operand, written there once per tile by the epilogue warps;
+//   * the k_idx block (128 keys x 128 dims, 32 KB) is the B operand, streamed
+//     by TMA (128-byte swizzle) through a 4-stage shared-memory ring and shared
+//     by the groups' MMAs, so shared memory only feeds B;
+//   * two 128-column fp32 accumulators alternate, so the epilogue of one unit
+//     overlaps the MMAs of the next.
+// Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
+// 2-5 load index queries into TMEM and run the epilogue (one query row per
+// thread: masked max over the row's 128 columns, one fp32 store per unit).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kStageBytes = 128 * 128 * 2;  // one k_idx block, bf16
+constexpr int kHalfBytes = kStageBytes / 2; // 64 dims (128 B) x 128 keys
+constexpr int kThreads = 192;
+constexpr int kMaxGroups = 4;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCol = 256;           // accumulators follow the A region
+constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, 0, 0);
+constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + 256;
+
+// Blocks query tile m (128 rows) of a sequence can see.
+__host__ __device__ inline int tile_blocks(const Problem& P, int m) {
+  const int last = min(P.Sq - 1, m * 128 + 127);
+  return int((P.q_pos0 + last) / P.Bk) + 1;
+}
+
+// (tile, block) pairs of one sequence that come before query tile m.  Every
+// tile before m is full, so tile m' sees base + m' + 1 blocks.
+__host__ __device__ inline long long pairs_before(const Problem& P, int m) {
+  const long long base = (P.q_pos0 + 127) / P.Bk;
+  return (long long)m * (base + 1) + (long long)m * (m - 1) / 2;
+}
+
+__host__ __device__ inline int mtiles(const Problem& P) { return (P.Sq + 127) / 128; }
+
+__host__ __device__ inline long long pairs_per_seq(const Problem& P) {
+  const int M = mtiles(P);
+  return pairs_before(P, M - 1) + tile_blocks(P, M - 1);
+}
+
+// Walks (b, m, c) over a contiguous range of the linear pair index.
+struct Walk {
+  int b, m, c, nc;
+  __device__ void start(const Problem& P, long long L, long long per_seq) {
+    b = int(L / per_seq);
+    long long l = L % per_seq;
+    int lo = 0, hi = mtiles(P) - 1;
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if (pairs_before(P, mid) <= l) lo = mid; else hi = mid - 1;
+    }
+    m = lo;
+    c = int(l - pairs_before(P, m));
+    nc = tile_blocks(P, m);
+  }
+  // advances; returns true when the next pair starts a new query tile
+  __device__ bool next(const Problem& P) {
+    if (++c < nc) return false;
+    c = 0;
+    if (++m == mtiles(P)) { m = 0; ++b; }
+    nc = tile_blocks(P, m);
+    return true;
+  }
+};
+
+struct Bars {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t a_full;
+  uint64_t a_empty;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
+                const __nv_bfloat16* __restrict__ q_idx, float* __restrict__ bmax,
+                int* __restrict__ status, long long per_seq) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&bars->full[s], 1);
+      tc::mbar_init(&bars->empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&bars->acc_full[s], 1);
+      tc::mbar_init(&bars->acc_empty[s], 4);
+    }
+    tc::mbar_init(&bars->a_full, 4);
+    tc::mbar_init(&bars->a_empty, 1);
+    bars->abort = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) tc::tma_prefetch(&tmap_k);
+  if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  const long long total = per_seq * P.B;
+  const long long L0 = total * blockIdx.x / gridDim.x;
+  const long long L1 = total * (blockIdx.x + 1) / gridDim.x;
+  bool failed = false;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && L0 < L1) {
+      Walk w;
+      w.start(P, L0, per_seq);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (long long L = L0; L < L1; ++L) {
+        if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort)) { failed = true; break; }
+        tc::mbar_arrive_expect_tx(&bars->full[stage], kStageBytes);
+        const int row = w.b * P.Skv + w.c * P.Bk;
+        uint8_t* dst = stages + stage * kStageBytes;
+        tc::tma_load_2d(dst, &tmap_k, &bars->full[stage], 0, row);
+        tc::tma_load_2d(dst + kHalfBytes, &tmap_k, &bars->full[stage], 64, row);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        w.next(P);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && L0 < L1) {
+      Walk w;
+      w.start(P, L0, per_seq);
+      int stage = 0, slot = 0;
+      uint32_t phase = 0, acc_phase = 0, a_phase = 0;
+      bool seg_start = true;
+      for (long long L = L0; L < L1 && !failed; ++L) {
+        if (seg_start) {
+          if (!tc::mbar_wait(&bars->a_full, a_phase, abort)) { failed = true; break; }
+          a_phase ^= 1;
+          tc::tc_fence_after();
+        }
+        if (!tc::mbar_wait(&bars->full[stage], phase, abort)) { failed = true; break; }
+        tc::tc_fence_after();
+        const uint32_t sbase = tc::smem_addr(stages + stage * kStageBytes);
+        for (int g = 0; g < P.Hkv; ++g) {
+          if (!tc::mbar_wait(&bars->acc_empty[slot], acc_phase ^ 1, abort)) {
+            failed = true;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t d = tmem + kAccCol + slot * 128;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t bd = tc::sdesc_sw128(sbase + (kk >> 2) * kHalfBytes + (kk & 3) * 32,
+                                                16, 1024);
+            tc::mma_ts(d, tmem + g * 64 + kk * 8, bd, kIdesc, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&bars->acc_full[slot]);
+          slot ^= 1;
+          if (slot == 0) acc_phase ^= 1;
+        }
+        if (failed) break;
+        tc::mma_commit(&bars->empty[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        seg_start = w.next(P);
+        if (seg_start || L + 1 == L1) tc::mma_commit(&bars->a_empty);
+      }
+    }
+  } else {
+    // ---------------- index-query loader + epilogue ----------------
+    const int quarter = warp & 3;           // TMEM lanes this warp may touch
+    const int row = quarter * 32 + lane;    // query row inside the tile
+    const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+    if (L0 < L1) {
+      Walk w;
+      w.start(P, L0, per_seq);
+      int slot = 0;
+      uint32_t acc_phase = 0, ae_phase = 0;
+      bool seg_start = true, first = true;
+      for (long long L = L0; L < L1 && !failed; ++L) {
+        const int i = w.m * 128 + row;      // query index inside the sequence
+        const bool valid = i < P.Sq;
+        const long long r = (long long)w.b * P.Sq + i;
+        if (seg_start) {
+          if (!first) {
+            if (!__all_sync(MSA_FULL_MASK, tc::mbar_wait(&bars->a_empty, ae_phase, abort))) {
+              failed = true;
+              break;
+            }
+            ae_phase ^= 1;
+            tc::tc_fence_after();
+          }
+          first = false;
+          const uint4* src = reinterpret_cast<const uint4*>(q_idx + r * P.Hkv * 128);
+          for (int g = 0; g < P.Hkv; ++g) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t v[32];
+#pragma unroll
+              for (int x = 0; x < 8; ++x) {
+                uint4 u = valid ? __ldg(src + g * 16 + h * 8 + x) : make_uint4(0, 0, 0, 0);
+                v[4 * x + 0] = u.x;
+                v[4 * x + 1] = u.y;
+                v[4 * x + 2] = u.z;
+                v[4 * x + 3] = u.w;
+              }
+              tc::tmem_st32(tmem + lane_addr + g * 64 + h * 32, v);
+            }
+          }
+          tc::tmem_st_wait();
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&bars->a_full);
+        }
+        const long long t = P.q_pos0 + i;
+        const long long lim = t - (long long)w.c * P.Bk;  // last visible column
+        for (int g = 0; g < P.Hkv; ++g) {
+          if (!__all_sync(MSA_FULL_MASK, tc::mbar_wait(&bars->acc_full[slot], acc_phase, abort))) {
+            failed = true;
+            break;
+          }
+          tc::tc_fence_after();
+          float m = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t v[32];
+            tc::tmem_ld32(tmem + lane_addr + kAccCol + slot * 128 + j * 32, v);
+            tc::tmem_ld_wait();
+            if (lim >= j * 32 + 31) {
+#pragma unroll
+              for (int x = 0; x < 32; ++x) m = fmaxf(m, __uint_as_float(v[x]));
+            } else {
+#pragma unroll
+              for (int x = 0; x < 32; ++x)
+                if (j * 32 + x <= lim) m = fmaxf(m, __uint_as_float(v[x]));
+            }
+          }
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&bars->acc_empty[slot]);
+          if (valid) bmax[((long long)g * P.T + r) * P.nblk + w.c] = m;
+          slot ^= 1;
+          if (slot == 0) acc_phase ^= 1;
+        }
+        seg_start = w.next(P);
+      }
+    }
+  }
+  if (failed) {
+    bars->abort = 1;
+    atomicOr(status, tc::kStatusWaitTimeout);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+bool index_tc_supported(const Problem& P) {
+  return !P.f32 && P.DI == 128 && P.Bk == 128 && P.Hkv <= kMaxGroups && P.Sq > 8 &&
+         (long long)P.B * P.Skv < (1LL << 31);
+}
+
+cudaError_t launch_index_tc(const Problem& P, const void* q_idx, const void* k_idx,
+                            float* bmax, int32_t* status, cudaStream_t s) {
+  auto enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {128, cuuint64_t(P.B) * P.Skv};
+  cuuint64_t strides[1] = {128 * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_idx), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  const long long per_seq = pairs_per_seq(P);
+  const long long total = per_seq * P.B;
+  const int grid = int(std::min<long long>(sm_count(), total));
+  cudaError_t e = cudaFuncSetAttribute(index_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  index_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(
+      map, P, static_cast<const __nv_bfloat16*>(q_idx), bmax, status, per_seq);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

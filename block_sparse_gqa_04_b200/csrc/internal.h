@@ -1,0 +1,80 @@
+// Internal launch interface between the C ABI layer (msa_api.cu) and the
+// kernel files.  Not part of the public header.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace msa {
+
+// Query rows of one sequence handled as one unit of the block -> query lists.
+// The lists are keyed by (sequence, group, query chunk, block) so that the
+// queries gathered by one chunk's work stay resident in L2.
+constexpr int kQueryChunk = 8192;
+
+// Resolved problem, shared by every launcher.
+struct Problem {
+  int B, Sq, Skv, Hq, Hkv, D, DI, Bk, K;
+  int G;            // query heads per group
+  int T;            // B * Sq query rows
+  int nblk;         // ceil(Skv / Bk)
+  int nqc;          // ceil(Sq / kQueryChunk)
+  int qpt;          // gathered queries per 128-row tile = 128 / G
+  long long q_pos0;
+  float scale;      // main-branch logit scale
+  bool f32;         // fp32 tensors (else bf16)
+  long long nlists; // B * Hkv * nqc * nblk
+};
+
+// Views into the caller's workspace.
+struct Lists {
+  int32_t* counts;    // [nlists]
+  int32_t* cursor;    // [nlists]
+  int32_t* list_off;  // [nlists + 1]
+  int32_t* tile_off;  // [nlists + 1]
+  int32_t* entries;   // [Hkv * T * K] packed (row << 5) | slot, grouped by list
+  int32_t* pos;       // [Hkv, T, K] position of (g, row, slot) in entries, or -1
+};
+
+// Partial softmax states, stored in entry order: the G query heads of entry e
+// occupy rows e*G .. e*G+G-1, so one tile of gathered queries writes one
+// contiguous run.
+struct Partials {
+  void* o;            // [entries, G, D] bf16 (bf16 problems) or fp32, normalised
+  float* lse2;        // [entries, G] base-2 log of the softmax normaliser
+};
+
+// --- index branch ---------------------------------------------------------
+cudaError_t launch_fill(float* p, size_t n, float value, cudaStream_t s);
+// Block maxima with SIMT kernels (any dtype / index_dim).
+cudaError_t launch_index_simt(const Problem& P, const void* q_idx, const void* k_idx,
+                              float* bmax, cudaStream_t s);
+// Block maxima with the tcgen05 / TMA kernel (bf16, index_dim 128).
+bool index_tc_supported(const Problem& P);
+cudaError_t launch_index_tc(const Problem& P, const void* q_idx, const void* k_idx,
+                            float* bmax, int32_t* status, cudaStream_t s);
+cudaError_t launch_topk(const Problem& P, const float* bmax, int32_t* q2k, cudaStream_t s);
+
+// --- block -> query lists ---------------------------------------------------
+cudaError_t launch_invert(const Problem& P, const int32_t* q2k, const Lists& L,
+                          int32_t* status, cudaStream_t s);
+
+// --- main branch ------------------------------------------------------------
+cudaError_t launch_attn_simt(const Problem& P, const void* q, const void* k, const void* v,
+                             const Lists& L, const Partials& part, cudaStream_t s);
+bool attn_tc_supported(const Problem& P);
+cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const void* v,
+                           const Lists& L, const Partials& part, int32_t* status,
+                           cudaStream_t s);
+cudaError_t launch_combine(const Problem& P, const int32_t* pos, const Partials& part,
+                           void* out, float* lse, cudaStream_t s);
+
+// Device status bits (workspace status word): 1 = invalid q2k entry given to
+// attend, 2 = a bounded wait inside a tensor-core kernel gave up.
+constexpr int kStatusBadEntry = 1;
+
+// Kernel launches made by each launcher (for msa_launch_count).
+constexpr int kLaunchesInvert = 4;
+
+}  // namespace msa

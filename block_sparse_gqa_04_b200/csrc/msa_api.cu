@@ -1,0 +1,288 @@
+// C ABI of libmsa: argument checks, workspace layout and the launch sequence.
+// Declarations and the contract of every entry point are in include/msa.h.
+#include <math.h>
+#include <string.h>
+
+#include "../../include/msa.h"
+#include "internal.h"
+
+using msa::Problem;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool pow2_divides_128(int g) { return g >= 1 && g <= 128 && (128 % g) == 0; }
+
+// Shape checks shared by every entry point.
+msa_status_t resolve(const msa_problem_t* p, Problem* P) {
+  if (!p) return MSA_ERR_INVALID_ARG;
+  if (p->reserved != 0) return MSA_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->q_len < 0 || p->kv_len < 1 || p->q_pos0 < 0) return MSA_ERR_INVALID_ARG;
+  if (p->q_pos0 + p->q_len > p->kv_len) return MSA_ERR_INVALID_ARG;
+  if (p->num_kv_heads < 1 || p->num_q_heads < 1 || p->num_q_heads % p->num_kv_heads != 0)
+    return MSA_ERR_INVALID_ARG;
+  if (p->block_size < 1 || p->top_k < 1 || p->head_dim < 1 || p->index_dim < 1)
+    return MSA_ERR_INVALID_ARG;
+  if (p->dtype != MSA_BF16 && p->dtype != MSA_F32) return MSA_ERR_INVALID_ARG;
+  if (!(p->softmax_scale >= 0.0f) || isinf(p->softmax_scale)) return MSA_ERR_INVALID_ARG;
+  const int G = p->num_q_heads / p->num_kv_heads;
+  if (p->block_size != 128) return MSA_ERR_UNSUPPORTED;
+  if (p->top_k > 32) return MSA_ERR_UNSUPPORTED;
+  if (p->head_dim != 64 && p->head_dim != 128) return MSA_ERR_UNSUPPORTED;
+  if (p->index_dim != 32 && p->index_dim != 64 && p->index_dim != 128) return MSA_ERR_UNSUPPORTED;
+  if (!pow2_divides_128(G)) return MSA_ERR_UNSUPPORTED;
+  const long long T = (long long)p->batch * p->q_len;
+  if (T * 32 >= (1LL << 31)) return MSA_ERR_UNSUPPORTED;                      // entry packing
+  if ((long long)p->num_kv_heads * T * p->top_k >= (1LL << 31)) return MSA_ERR_UNSUPPORTED;
+  if ((long long)p->batch * p->kv_len >= (1LL << 31)) return MSA_ERR_UNSUPPORTED;
+  P->B = p->batch;
+  P->Sq = p->q_len;
+  P->Skv = p->kv_len;
+  P->Hq = p->num_q_heads;
+  P->Hkv = p->num_kv_heads;
+  P->D = p->head_dim;
+  P->DI = p->index_dim;
+  P->Bk = p->block_size;
+  P->K = p->top_k;
+  P->G = G;
+  P->T = int(T);
+  P->nblk = (p->kv_len + p->block_size - 1) / p->block_size;
+  P->nqc = (p->q_len + msa::kQueryChunk - 1) / msa::kQueryChunk;
+  if (P->nqc < 1) P->nqc = 1;
+  P->qpt = 128 / G;
+  P->q_pos0 = p->q_pos0;
+  P->scale = p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / sqrtf((float)p->head_dim);
+  P->f32 = p->dtype == MSA_F32;
+  P->nlists = (long long)P->B * P->Hkv * P->nqc * P->nblk;
+  if (P->nlists + 1 >= (1LL << 31)) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+// Workspace layout (each region 256-byte aligned, in this order).
+struct Layout {
+  size_t status, bmax, q2k, counts, cursor, list_off, tile_off, entries, pos, part_o, part_lse,
+      total;
+};
+
+Layout layout(const Problem& P, int op) {
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += align_up(bytes); return o; };
+  const size_t T = size_t(P.T);
+  const size_t esz = P.f32 ? 4 : 2;
+  L.status = take(sizeof(int32_t));
+  const bool sel = op == MSA_OP_SELECT || op == MSA_OP_FORWARD;
+  const bool att = op == MSA_OP_ATTEND || op == MSA_OP_FORWARD;
+  L.bmax = sel ? take(size_t(P.Hkv) * T * P.nblk * sizeof(float)) : 0;
+  L.q2k = op == MSA_OP_FORWARD ? take(size_t(P.Hkv) * T * P.K * sizeof(int32_t)) : 0;
+  if (att) {
+    L.counts = take(size_t(P.nlists) * 4);
+    L.cursor = take(size_t(P.nlists) * 4);
+    L.list_off = take(size_t(P.nlists + 1) * 4);
+    L.tile_off = take(size_t(P.nlists + 1) * 4);
+    L.entries = take(size_t(P.Hkv) * T * P.K * 4);
+    L.pos = take(size_t(P.Hkv) * T * P.K * 4);
+    // one partial state per (entry, head of the group): Hkv*T*K*G = T*Hq*K rows
+    L.part_o = take(T * P.Hq * P.K * size_t(P.D) * esz);
+    L.part_lse = take(T * P.Hq * P.K * sizeof(float));
+  }
+  L.total = off;
+  return L;
+}
+
+msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+// Optional stage events (msa_set_stage_events).
+cudaEvent_t const* g_events = nullptr;
+int g_nevents = 0;
+int g_next = 0;
+
+void stage_mark(cudaStream_t s) {
+  if (g_events && g_next < g_nevents) cudaEventRecord(g_events[g_next++], s);
+}
+
+template <typename P_>
+P_* at(void* ws, size_t off) { return reinterpret_cast<P_*>(static_cast<char*>(ws) + off); }
+
+msa_status_t check_ws(const Problem& P, int op, const void* ws, size_t ws_bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return MSA_ERR_INVALID_ARG;
+  if (ws_bytes < layout(P, op).total) return MSA_ERR_WORKSPACE;
+  return MSA_OK;
+}
+
+msa_status_t run_select(const Problem& P, const void* q_idx, const void* k_idx, int32_t* q2k,
+                        float* bscores, void* ws, cudaStream_t s) {
+  const Layout L = layout(P, MSA_OP_SELECT);
+  float* bmax = bscores ? bscores : at<float>(ws, L.bmax);
+  cudaError_t e = cudaSuccess;
+  if (bscores) e = msa::launch_fill(bscores, size_t(P.Hkv) * P.T * P.nblk, -INFINITY, s);
+  if (e == cudaSuccess) {
+    e = msa::index_tc_supported(P)
+            ? msa::launch_index_tc(P, q_idx, k_idx, bmax, at<int32_t>(ws, L.status), s)
+            : msa::launch_index_simt(P, q_idx, k_idx, bmax, s);
+    stage_mark(s);
+  }
+  if (e == cudaSuccess) {
+    e = msa::launch_topk(P, bmax, q2k, s);
+    stage_mark(s);
+  }
+  return cuda_status(e);
+}
+
+msa_status_t run_attend(const Problem& P, const void* q, const void* k, const void* v,
+                        const int32_t* q2k, void* out, float* lse, void* ws, const Layout& L,
+                        cudaStream_t s) {
+  msa::Lists lists{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.cursor),
+                   at<int32_t>(ws, L.list_off), at<int32_t>(ws, L.tile_off),
+                   at<int32_t>(ws, L.entries), at<int32_t>(ws, L.pos)};
+  msa::Partials part{at<void>(ws, L.part_o), at<float>(ws, L.part_lse)};
+  cudaError_t e = msa::launch_invert(P, q2k, lists, at<int32_t>(ws, L.status), s);
+  stage_mark(s);
+  if (e == cudaSuccess) {
+    e = msa::attn_tc_supported(P)
+            ? msa::launch_attn_tc(P, q, k, v, lists, part, at<int32_t>(ws, L.status), s)
+            : msa::launch_attn_simt(P, q, k, v, lists, part, s);
+    stage_mark(s);
+  }
+  if (e == cudaSuccess) {
+    e = msa::launch_combine(P, lists.pos, part, out, lse, s);
+    stage_mark(s);
+  }
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t msa_workspace_size(const msa_problem_t* p, int32_t op) {
+  Problem P;
+  if (resolve(p, &P) != MSA_OK || op < MSA_OP_SELECT || op > MSA_OP_FORWARD) return 0;
+  return layout(P, op).total;
+}
+
+msa_status_t msa_select(const msa_problem_t* p, const void* q_idx, const void* k_idx,
+                        int32_t* q2k, float* block_scores_opt, void* ws, size_t ws_bytes,
+                        void* stream) {
+  Problem P;
+  msa_status_t st = resolve(p, &P);
+  if (st != MSA_OK) return st;
+  if (P.T == 0) return MSA_OK;  // nothing to do; empty tensors may carry null pointers
+  if (!q_idx || !k_idx || !q2k) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q2k) ||
+      (block_scores_opt && !aligned16(block_scores_opt)))
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, MSA_OP_SELECT, ws, ws_bytes)) != MSA_OK) return st;
+  if (P.T == 0) return MSA_OK;
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  return run_select(P, q_idx, k_idx, q2k, block_scores_opt, ws, (cudaStream_t)stream);
+}
+
+msa_status_t msa_attend(const msa_problem_t* p, const void* q, const void* k, const void* v,
+                        const int32_t* q2k, void* out, float* lse_opt, void* ws,
+                        size_t ws_bytes, void* stream) {
+  Problem P;
+  msa_status_t st = resolve(p, &P);
+  if (st != MSA_OK) return st;
+  if (P.T == 0) return MSA_OK;  // nothing to do; empty tensors may carry null pointers
+  if (!q || !k || !v || !q2k || !out) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q2k) || !aligned16(out) ||
+      (lse_opt && !aligned16(lse_opt)))
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, MSA_OP_ATTEND, ws, ws_bytes)) != MSA_OK) return st;
+  if (P.T == 0) return MSA_OK;
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  return run_attend(P, q, k, v, q2k, out, lse_opt, ws, layout(P, MSA_OP_ATTEND),
+                    (cudaStream_t)stream);
+}
+
+msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, const void* v,
+                         const void* q_idx, const void* k_idx, void* out, float* lse_opt,
+                         int32_t* q2k_opt, void* ws, size_t ws_bytes, void* stream) {
+  Problem P;
+  msa_status_t st = resolve(p, &P);
+  if (st != MSA_OK) return st;
+  if (P.T == 0) return MSA_OK;  // nothing to do; empty tensors may carry null pointers
+  if (!q || !k || !v || !q_idx || !k_idx || !out) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_idx) ||
+      !aligned16(k_idx) || !aligned16(out) || (lse_opt && !aligned16(lse_opt)) ||
+      (q2k_opt && !aligned16(q2k_opt)))
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, MSA_OP_FORWARD, ws, ws_bytes)) != MSA_OK) return st;
+  if (P.T == 0) return MSA_OK;
+  const Layout L = layout(P, MSA_OP_FORWARD);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  int32_t* q2k = q2k_opt ? q2k_opt : at<int32_t>(ws, L.q2k);
+  // the select stage only needs the status word and bmax, which sit at the same
+  // offsets in the forward layout
+  st = run_select(P, q_idx, k_idx, q2k, nullptr, ws, s);
+  if (st != MSA_OK) return st;
+  return run_attend(P, q, k, v, q2k, out, lse_opt, ws, L, s);
+}
+
+msa_status_t msa_device_status(const void* ws, int32_t* code, void* stream) {
+  if (!ws || !code) return MSA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MSA_ERR_CUDA;
+  *code = h;
+  return h == 0 ? MSA_OK : MSA_ERR_DEVICE;
+}
+
+int32_t msa_set_stage_events(void* const* events, int32_t n) {
+  g_events = reinterpret_cast<cudaEvent_t const*>(events);
+  g_nevents = events ? n : 0;
+  g_next = 0;
+  return 5;
+}
+
+int32_t msa_launch_count(const msa_problem_t* p, int32_t op) {
+  Problem P;
+  if (resolve(p, &P) != MSA_OK || P.T == 0) return 0;
+  const int sel = 2;                               // index + top-k
+  const int att = msa::kLaunchesInvert + 2;        // lists + attention + combine
+  switch (op) {
+    case MSA_OP_SELECT: return sel;
+    case MSA_OP_ATTEND: return att;
+    case MSA_OP_FORWARD: return sel + att;
+  }
+  return 0;
+}
+
+const char* msa_kernel_path(const msa_problem_t* p, int32_t op) {
+  Problem P;
+  if (resolve(p, &P) != MSA_OK) return "invalid";
+  const bool itc = msa::index_tc_supported(P), atc = msa::attn_tc_supported(P);
+  switch (op) {
+    case MSA_OP_SELECT: return itc ? "index:tc" : "index:simt";
+    case MSA_OP_ATTEND: return atc ? "attn:tc" : "attn:simt";
+    case MSA_OP_FORWARD:
+      return itc ? (atc ? "index:tc attn:tc" : "index:tc attn:simt")
+                 : (atc ? "index:simt attn:tc" : "index:simt attn:simt");
+  }
+  return "invalid";
+}
+
+const char* msa_status_string(msa_status_t s) {
+  switch (s) {
+    case MSA_OK: return "MSA_OK";
+    case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG: null/misaligned pointer or bad shape";
+    case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED: shape outside the kernels' coverage";
+    case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE: workspace too small";
+    case MSA_ERR_CUDA: return "MSA_ERR_CUDA: CUDA launch or call failed";
+    case MSA_ERR_DEVICE: return "MSA_ERR_DEVICE: invalid q2k entry seen on the device";
+  }
+  return "MSA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

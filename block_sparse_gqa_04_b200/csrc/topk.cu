@@ -1,0 +1,105 @@
+// Exp-free top-k block selection, one warp per (GQA group, query row).
+//
+// snilld.dk "Hvad er MSA i praksis": each query keeps k blocks per GQA group
+// and its own block is always kept; section "Teknisk forklaring hvorfor
+// kompleksiteten skifter": softmax preserves the order, so raw block scores are
+// ranked and no exponential is taken.  "Substantial numerical differences ...",
+// section 解决步骤: boost and top-k act per index head, never pooled across
+// heads.  The local block floor(t/Bk) takes one of the k slots; the other
+// min(k, visible) - 1 slots go to the earlier blocks with the largest keys
+// (score, then lower block id); ids are written ascending, -1 padded.
+//
+// Selection runs in two phases.  Phase 1 takes each lane's largest key over its
+// strided share of the row and finds the `need`-th largest of those 32 lane
+// maxima, tau: the lanes holding the top `need` maxima give `need` distinct keys
+// >= tau, so the true top-`need` keys are all >= tau.  The keys >= tau (a few
+// dozen on typical rows) are compacted into shared memory.  Phase 2 picks the
+// top keys among them, one warp-wide maximum at a time, each pass restricted to
+// keys below the previous pick; keys are unique (they carry the block id), so
+// every pass takes exactly one key.  Rows with more candidates than fit in
+// shared memory rescan the row in phase 2 instead.
+#include "common.cuh"
+#include "internal.h"
+
+namespace msa {
+
+constexpr int kTopkWarps = 8;
+constexpr int kCandCap = 128;  // candidates >= tau kept in shared memory per warp
+
+__global__ void __launch_bounds__(256) topk_kernel(Problem P, const float* __restrict__ bmax,
+                                                   int32_t* __restrict__ q2k) {
+  __shared__ uint64_t cand_all[kTopkWarps][kCandCap];
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  const long long wid = (long long)blockIdx.x * kTopkWarps + w;
+  if (wid >= (long long)P.Hkv * P.T) return;
+  uint64_t* cand = cand_all[w];
+  const int g = int(wid / P.T);
+  const int r = int(wid % P.T);
+  const long long t = P.q_pos0 + r % P.Sq;
+  const int c_t = int(t / P.Bk);
+  const int ksel = min(P.K, c_t + 1);
+  const int need = ksel - 1;  // earlier blocks to pick
+  int mine = INT_MAX;         // lane s < need holds the s-th pick
+  if (need == c_t) {
+    // every visible block is selected
+    if (lane < c_t) mine = lane;
+  } else if (need > 0) {
+    const float* row = bmax + ((long long)g * P.T + r) * P.nblk;
+    // phase 1: lane maxima, and tau = the need-th largest of them
+    uint64_t lmax = 0;
+    for (int c = lane; c < c_t; c += 32) {
+      uint64_t key = block_key(row[c], c);
+      lmax = key > lmax ? key : lmax;
+    }
+    uint64_t prev = ~0ull, tau = 0;
+    for (int s = 0; s < need; ++s) {
+      tau = warp_max_u64(lmax < prev ? lmax : 0);
+      prev = tau;
+    }
+    // compact the keys >= tau
+    int count = 0;
+    for (int base = 0; base < c_t; base += 32) {
+      const int c = base + lane;
+      const uint64_t key = c < c_t ? block_key(row[c], c) : 0;
+      const bool take = key >= tau;
+      const unsigned m = __ballot_sync(MSA_FULL_MASK, take);
+      const int pos = count + __popc(m & ((1u << lane) - 1u));
+      if (take && pos < kCandCap) cand[pos] = key;
+      count += __popc(m);
+    }
+    __syncwarp();
+    // phase 2: `need` passes, each taking the largest key below the last pick
+    prev = ~0ull;
+    for (int s = 0; s < need; ++s) {
+      uint64_t best = 0;
+      if (count <= kCandCap) {
+        for (int e = lane; e < count; e += 32) {
+          const uint64_t key = cand[e];
+          if (key < prev && key > best) best = key;
+        }
+      } else {
+        for (int c = lane; c < c_t; c += 32) {
+          const uint64_t key = block_key(row[c], c);
+          if (key >= tau && key < prev && key > best) best = key;
+        }
+      }
+      best = warp_max_u64(best);
+      if (lane == s) mine = key_block(best);
+      prev = best;
+    }
+  }
+  if (lane == need) mine = c_t;
+  const int sorted = warp_sort_asc(mine);
+  if (lane < P.K) q2k[((long long)g * P.T + r) * P.K + lane] = lane < ksel ? sorted : -1;
+}
+
+cudaError_t launch_topk(const Problem& P, const float* bmax, int32_t* q2k, cudaStream_t s) {
+  long long warps = (long long)P.Hkv * P.T;
+  if (warps == 0) return cudaSuccess;
+  long long blocks = (warps + kTopkWarps - 1) / kTopkWarps;
+  topk_kernel<<<unsigned(blocks), 32 * kTopkWarps, 0, s>>>(P, bmax, q2k);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

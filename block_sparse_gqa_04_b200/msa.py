@@ -1,0 +1,253 @@
+"""Python binding of libmsa (argument marshalling only).
+
+Every step of the MSA forward path runs in the CUDA kernels of ``libmsa.so``;
+this module checks tensor shapes, allocates the caller-owned outputs and
+workspace with torch, and calls the C ABI declared in ``include/msa.h`` on
+torch's current CUDA stream.  There is no fallback: if the library is missing
+or the tensors are not CUDA tensors (or pinned host tensors, which are copied
+to the device and back), the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa.so")
+
+MSA_BF16, MSA_F32 = 0, 1
+OP_SELECT, OP_ATTEND, OP_FORWARD = 0, 1, 2
+
+STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
+          3: "MSA_ERR_WORKSPACE", 4: "MSA_ERR_CUDA", 5: "MSA_ERR_DEVICE"}
+
+EXPORTED = ("msa_workspace_size", "msa_select", "msa_attend", "msa_forward",
+            "msa_device_status", "msa_set_stage_events", "msa_launch_count", "msa_kernel_path",
+            "msa_status_string")
+STAGES = ("index", "topk", "lists", "attn", "combine")
+
+
+class MsaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("q_len", ctypes.c_int32), ("kv_len", ctypes.c_int32),
+        ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("index_dim", ctypes.c_int32),
+        ("block_size", ctypes.c_int32), ("top_k", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("q_pos0", ctypes.c_int64), ("softmax_scale", ctypes.c_float),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Loads libmsa.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m block_sparse_gqa_04_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+        pp = ctypes.POINTER(Problem)
+        lib.msa_workspace_size.argtypes = [pp, i32]
+        lib.msa_workspace_size.restype = sz
+        lib.msa_select.argtypes = [pp, vp, vp, vp, vp, vp, sz, vp]
+        lib.msa_select.restype = i32
+        lib.msa_attend.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.msa_attend.restype = i32
+        lib.msa_forward.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.msa_forward.restype = i32
+        lib.msa_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
+        lib.msa_device_status.restype = i32
+        lib.msa_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
+        lib.msa_set_stage_events.restype = i32
+        lib.msa_launch_count.argtypes = [pp, i32]
+        lib.msa_launch_count.restype = i32
+        lib.msa_kernel_path.argtypes = [pp, i32]
+        lib.msa_kernel_path.restype = ctypes.c_char_p
+        lib.msa_status_string.argtypes = [i32]
+        lib.msa_status_string.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def make_problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
+                 block_size=128, top_k=16, dtype=torch.bfloat16, q_pos0=0,
+                 softmax_scale=0.0) -> Problem:
+    return Problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
+                   block_size, top_k, MSA_F32 if dtype == torch.float32 else MSA_BF16,
+                   q_pos0, softmax_scale, 0)
+
+
+def problem_of(w, softmax_scale: float = 0.0) -> Problem:
+    """Problem of a :class:`~block_sparse_gqa_04_b200.workload.Workload`."""
+    return make_problem(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
+                        w.head_dim, w.index_dim, w.block_size, w.top_k, w.torch_dtype,
+                        w.q_pos0, softmax_scale)
+
+
+def workspace_size(p: Problem, op: int = OP_FORWARD) -> int:
+    return int(load().msa_workspace_size(ctypes.byref(p), op))
+
+
+def launch_count(p: Problem, op: int = OP_FORWARD) -> int:
+    return int(load().msa_launch_count(ctypes.byref(p), op))
+
+
+def kernel_path(p: Problem, op: int = OP_FORWARD) -> str:
+    return load().msa_kernel_path(ctypes.byref(p), op).decode()
+
+
+_stage_keep = None
+
+
+def set_stage_events(events) -> None:
+    """Records ``events[i]`` (torch.cuda.Event, already created) after stage i
+    of every later call; ``None`` turns this off.  See msa_set_stage_events."""
+    global _stage_keep
+    if events is None:
+        _stage_keep = None
+        load().msa_set_stage_events(None, 0)
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _stage_keep = arr
+    load().msa_set_stage_events(arr, len(events))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise MsaError(code, where)
+
+
+def new_workspace(p: Problem, op: int, device) -> torch.Tensor:
+    n = workspace_size(p, op)
+    if n == 0:
+        raise MsaError(1, "workspace_size")
+    return torch.empty(n + 256, dtype=torch.uint8, device=device)
+
+
+def _ws_view(ws: torch.Tensor) -> Tuple[int, int]:
+    base = ws.data_ptr()
+    pad = (-base) % 256
+    return base + pad, ws.numel() - pad
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libmsa takes CUDA tensors")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("libmsa takes contiguous tensors")
+
+
+def _dims(q, k, q_idx=None):
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    di = q_idx.shape[3] if q_idx is not None else 32
+    return B, Sq, Hq, D, Skv, Hkv, di
+
+
+def select(q_idx: torch.Tensor, k_idx: torch.Tensor, *, q_pos0: int = 0, block_size: int = 128,
+           top_k: int = 16, return_block_scores: bool = False,
+           workspace: Optional[torch.Tensor] = None):
+    """Index branch: returns q2k [Hkv, B*Sq, top_k] int32 (and block scores)."""
+    _require_cuda(q_idx, k_idx)
+    B, Sq, Hkv, di = q_idx.shape
+    Skv = k_idx.shape[1]
+    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, top_k, q_idx.dtype, q_pos0)
+    dev = q_idx.device
+    q2k = torch.empty((Hkv, B * Sq, top_k), dtype=torch.int32, device=dev)
+    nblk = -(-Skv // block_size)
+    bs = (torch.empty((Hkv, B * Sq, nblk), dtype=torch.float32, device=dev)
+          if return_block_scores else None)
+    ws = workspace if workspace is not None else new_workspace(p, OP_SELECT, dev)
+    wp, wn = _ws_view(ws)
+    _check(load().msa_select(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(q2k), _ptr(bs),
+                             ctypes.c_void_p(wp), wn, _stream(dev)), "msa_select")
+    return (q2k, bs) if return_block_scores else q2k
+
+
+def attend(q, k, v, q2k, *, q_pos0: int = 0, block_size: int = 128,
+           softmax_scale: float = 0.0, return_lse: bool = False,
+           workspace: Optional[torch.Tensor] = None, check_device_status: bool = False):
+    """Main branch over a given selection q2k [Hkv, B*Sq, top_k] (int32)."""
+    _require_cuda(q, k, v, q2k)
+    B, Sq, Hq, D, Skv, Hkv, _ = _dims(q, k)
+    top_k = q2k.shape[2]
+    p = make_problem(B, Sq, Skv, Hq, Hkv, D, 32, block_size, top_k, q.dtype, q_pos0,
+                     softmax_scale)
+    dev = q.device
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=dev) if return_lse else None
+    ws = workspace if workspace is not None else new_workspace(p, OP_ATTEND, dev)
+    wp, wn = _ws_view(ws)
+    _check(load().msa_attend(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q2k), _ptr(out),
+                             _ptr(lse), ctypes.c_void_p(wp), wn, _stream(dev)), "msa_attend")
+    if check_device_status:
+        code = ctypes.c_int32(0)
+        _check(load().msa_device_status(ctypes.c_void_p(wp), ctypes.byref(code), _stream(dev)),
+               "msa_attend (device status)")
+    return (out, lse) if return_lse else out
+
+
+def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, top_k: int = 16,
+            softmax_scale: float = 0.0, return_lse: bool = False, return_q2k: bool = False,
+            workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+            device=None):
+    """Index branch + main branch.  Returns out (and lse, q2k when asked).
+
+    CUDA tensors are used in place.  Host tensors (ideally pinned) are copied to
+    ``device`` (default ``cuda``) before the call and the results copied back.
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device(device or "cuda")
+        nb = q.is_pinned()
+        q, k, v, q_idx, k_idx = (t.to(dev, non_blocking=nb) for t in (q, k, v, q_idx, k_idx))
+    _require_cuda(q, k, v, q_idx, k_idx)
+    B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx)
+    p = make_problem(B, Sq, Skv, Hq, Hkv, D, di, block_size, top_k, q.dtype, q_pos0,
+                     softmax_scale)
+    dev = q.device
+    o = out if (out is not None and not host) else torch.empty_like(q)
+    lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=dev) if return_lse else None
+    q2k = (torch.empty((Hkv, B * Sq, top_k), dtype=torch.int32, device=dev)
+           if return_q2k else None)
+    ws = workspace if workspace is not None else new_workspace(p, OP_FORWARD, dev)
+    wp, wn = _ws_view(ws)
+    _check(load().msa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx),
+                              _ptr(k_idx), _ptr(o), _ptr(lse), _ptr(q2k), ctypes.c_void_p(wp),
+                              wn, _stream(dev)), "msa_forward")
+    if host:
+        if out is not None:
+            out.copy_(o, non_blocking=out.is_pinned())
+            o = out
+        else:
+            o = o.cpu()
+        lse = None if lse is None else lse.cpu()
+        q2k = None if q2k is None else q2k.cpu()
+    res = (o,)
+    if return_lse:
+        res += (lse,)
+    if return_q2k:
+        res += (q2k,)
+    return res[0] if len(res) == 1 else res

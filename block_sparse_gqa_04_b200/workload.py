@@ -5,8 +5,10 @@ imports neither the CUDA binding nor the oracle, so both sides (and the bench)
 can take their inputs from it.
 
 Recipe (the same for every workload):
-  * one ``torch.Generator`` seeded with ``seed`` draws, in this order, Q, K, V,
-    q_idx and k_idx as standard normals in fp32, row chunk by row chunk;
+  * one ``torch.Generator`` on the target device (the GPU for GPU runs, the CPU
+    for CPU-only tests), seeded with ``seed``, draws in this order Q, K, V,
+    q_idx and k_idx as standard normals in fp32, row chunk by row chunk (the
+    two devices' streams differ; each is fixed by the seed);
   * each tensor is multiplied by 1 (``fp32`` workloads) or by 1/sqrt(d)
     (``bf16`` workloads, d = head_dim for Q/K/V and index_dim for the index
     tensors) and rounded once to the workload's dtype (round to nearest even);
@@ -76,13 +78,14 @@ _CHUNK_ELEMS = 1 << 24
 
 def _draw(gen: torch.Generator, shape, scale: float, dtype: torch.dtype) -> torch.Tensor:
     """Standard normals drawn in fp32 row chunk by row chunk, scaled, rounded."""
-    out = torch.empty(shape, dtype=dtype)
+    out = torch.empty(shape, dtype=dtype, device=gen.device)
     flat = out.view(shape[0], -1)
     per_row = flat.shape[1]
     step = max(1, _CHUNK_ELEMS // max(per_row, 1))
     for r0 in range(0, flat.shape[0], step):
         r1 = min(flat.shape[0], r0 + step)
-        x = torch.randn((r1 - r0, per_row), generator=gen, dtype=torch.float32)
+        x = torch.randn((r1 - r0, per_row), generator=gen, dtype=torch.float32,
+                        device=gen.device)
         if scale != 1.0:
             x.mul_(scale)
         flat[r0:r1] = x.to(dtype)
@@ -94,9 +97,9 @@ def needle_upper(w: Workload) -> int:
     return first if first > 0 else (w.q_pos0 + w.q_len - 1) // w.block_size
 
 
-def make_inputs(w: Workload, seed: int = 0) -> Dict[str, torch.Tensor]:
-    """Inputs of workload ``w`` on the CPU: q, k, v, q_idx, k_idx (+ needle ids)."""
-    gen = torch.Generator().manual_seed(seed)
+def make_inputs(w: Workload, seed: int = 0, device="cpu") -> Dict[str, torch.Tensor]:
+    """Inputs of workload ``w`` on ``device``: q, k, v, q_idx, k_idx (+ needle ids)."""
+    gen = torch.Generator(device=device).manual_seed(seed)
     dt = w.torch_dtype
     s_main = 1.0 if w.dtype == "f32" else 1.0 / math.sqrt(w.head_dim)
     s_idx = 1.0 if w.dtype == "f32" else 1.0 / math.sqrt(w.index_dim)
@@ -107,7 +110,8 @@ def make_inputs(w: Workload, seed: int = 0) -> Dict[str, torch.Tensor]:
     q_idx = _draw(gen, (B * Sq, w.num_kv_heads, w.index_dim), s_idx, dt)
     # k_idx stays fp32 until the needles are in, then is rounded once.
     k_idx32 = _draw(gen, (B * Skv, w.index_dim), s_idx, torch.float32)
-    needle_ids = torch.full((B, w.num_kv_heads, max(w.needles, 0)), -1, dtype=torch.int64)
+    needle_ids = torch.full((B, w.num_kv_heads, max(w.needles, 0)), -1, dtype=torch.int64,
+                            device=gen.device)
     if w.needles > 0:
         upper = needle_upper(w)
         if upper < w.needles:
@@ -116,7 +120,7 @@ def make_inputs(w: Workload, seed: int = 0) -> Dict[str, torch.Tensor]:
         kv = k_idx32.view(B, Skv, w.index_dim)
         for b in range(B):
             for g in range(w.num_kv_heads):
-                blocks = torch.randperm(upper, generator=gen)[: w.needles]
+                blocks = torch.randperm(upper, generator=gen, device=gen.device)[: w.needles]
                 needle_ids[b, g] = blocks
                 shift = 0.5 * qi[b, :, g, :].float().mean(dim=0)
                 for c in blocks.tolist():

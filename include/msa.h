@@ -1,0 +1,156 @@
+/*
+ * msa.h - C ABI of libmsa, the B200 (sm_100a) MiniMax Sparse Attention (MSA)
+ * forward path.
+ *
+ * MSA splits attention into two branches.  The index branch scores every
+ * causally visible key token with one index-query head per GQA group against a
+ * single shared index-key head, max-pools the scores to blocks of 128 tokens
+ * and keeps, per (query, GQA group), the top-k blocks with the query's own
+ * block always among them.  The main branch then runs exact softmax attention
+ * of every query head of the group over the causally visible tokens of those
+ * blocks only.  Sources: "MiniMax 稀疏注意力" (hyper.ai page of paper
+ * 2606.13392), section 摘要; "MiniMax lancerer MSA" (snilld.dk), section
+ * "Hvad er MSA i praksis"; "Substantial numerical differences with Minimax MSA
+ * attention vs Minimax's Reference", sections 原因分析 and 解决步骤.
+ *
+ * Conventions for every entry point
+ *  - Tensors are dense, row-major, on the current CUDA device, and start on a
+ *    16-byte boundary:
+ *        q, out   [batch, q_len, num_q_heads, head_dim]
+ *        k, v     [batch, kv_len, num_kv_heads, head_dim]
+ *        q_idx    [batch, q_len, num_kv_heads, index_dim]
+ *        k_idx    [batch, kv_len, index_dim]       (one shared index-key head)
+ *        q2k      [num_kv_heads, batch*q_len, top_k]  int32
+ *        lse      [batch, q_len, num_q_heads]      float32
+ *        block_scores [num_kv_heads, batch*q_len, nblk] float32,
+ *                 nblk = ceil(kv_len / block_size)
+ *    The token-major layout and the q2k list layout are the ones the fix in
+ *    "Substantial numerical differences ...", section 解决步骤, hands to the
+ *    kernel path (q2k[num_kv_heads, bsz*q_len, topk]).
+ *  - Query row r = b*q_len + i sits at absolute position t = q_pos0 + i of
+ *    sequence b and sees keys 0..t of that sequence.  Query head h belongs to
+ *    group g = h / (num_q_heads / num_kv_heads) (contiguous groups, as the
+ *    repeat_interleave expansion in section 解决步骤 implies).
+ *  - The caller owns every buffer, the workspace included.  The library
+ *    allocates no memory, never synchronises the stream, and returns once the
+ *    work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *  - Argument errors are returned synchronously, before any launch, and leave
+ *    every output untouched.  A failed launch returns MSA_ERR_CUDA.  Problems
+ *    found on the device (a q2k entry outside [-1, floor(t/block_size)] given
+ *    to msa_attend) are recorded in the workspace status word, read with
+ *    msa_device_status(); such entries are skipped.
+ *  - q_len == 0 is a valid empty problem: the call returns MSA_OK without
+ *    looking at the pointers or launching anything.
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad size or shape */
+  MSA_ERR_UNSUPPORTED = 2,   /* valid shape outside what the kernels cover    */
+  MSA_ERR_WORKSPACE = 3,     /* ws_bytes smaller than msa_workspace_size()    */
+  MSA_ERR_CUDA = 4,          /* a CUDA call or launch failed                  */
+  MSA_ERR_DEVICE = 5         /* the device recorded an invalid q2k entry      */
+} msa_status_t;
+
+typedef enum { MSA_BF16 = 0, MSA_F32 = 1 } msa_dtype_t;
+
+typedef enum { MSA_OP_SELECT = 0, MSA_OP_ATTEND = 1, MSA_OP_FORWARD = 2 } msa_op_t;
+
+/* One MSA problem.  Supported: block_size 128; top_k 1..32; head_dim 64 or
+ * 128; index_dim 32, 64 or 128; num_q_heads a multiple of num_kv_heads with at
+ * most 128 query heads per group, dividing 128; q_pos0 + q_len <= kv_len;
+ * batch*q_len*32 < 2^31. */
+typedef struct {
+  int32_t batch;          /* sequences                                         */
+  int32_t q_len;          /* query rows per sequence                           */
+  int32_t kv_len;         /* key tokens per sequence                           */
+  int32_t num_q_heads;
+  int32_t num_kv_heads;   /* GQA groups = index-query heads                    */
+  int32_t head_dim;       /* D of q, k, v                                      */
+  int32_t index_dim;      /* d of q_idx, k_idx                                 */
+  int32_t block_size;     /* Bk, tokens per KV block (128)                     */
+  int32_t top_k;          /* blocks kept per (query, group), local one included */
+  int32_t dtype;          /* msa_dtype_t of q, k, v, q_idx, k_idx and out      */
+  int64_t q_pos0;         /* absolute position of query row 0 of every sequence */
+  float softmax_scale;    /* main-branch logit scale; 0 selects 1/sqrt(head_dim) */
+  int32_t reserved;       /* must be 0                                         */
+} msa_problem_t;
+
+/* Bytes of workspace that `op` needs for problem `p` (0 if p is invalid).
+ * The workspace must start on a 256-byte boundary. */
+size_t msa_workspace_size(const msa_problem_t* p, int32_t op);
+
+/* Index branch.  Computes, for every row r and group g, the block maxima of
+ * the raw index scores q_idx[r,g,:] . k_idx[b,j,:] over the visible tokens
+ * j <= t of each block ("Substantial numerical differences ...", section
+ * 原因分析: amax over the block; snilld.dk "Hvad er MSA i praksis": one
+ * index-query head per group, one shared index-key head), then writes q2k[g, r]
+ * = the local block floor(t/Bk) plus the min(top_k, visible blocks) - 1
+ * highest-scoring earlier blocks, ranked on raw scores without exponentials
+ * (snilld.dk, "Teknisk forklaring hvorfor kompleksiteten skifter"), ties to the
+ * lower block id, ids ascending, -1 padded.
+ * block_scores_opt: optional; if not NULL receives the block maxima, with
+ * -inf for every block that row r cannot see. */
+msa_status_t msa_select(const msa_problem_t* p, const void* q_idx, const void* k_idx,
+                        int32_t* q2k, float* block_scores_opt,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Main branch over a given selection q2k (entries -1 are skipped; others must
+ * be visible blocks, 0 <= c <= floor(t/Bk)).  Every query head of group g
+ * attends over the visible tokens of the blocks q2k[g, r, :] with softmax
+ * scale p->softmax_scale (snilld.dk "Hvad er MSA i praksis": scaled
+ * dot-product softmax over exactly those tokens).  Writes out (dtype of q) and,
+ * if lse_opt is not NULL, the natural-log softmax normaliser per (row, head);
+ * a row with no valid block gets zeros and -inf. */
+msa_status_t msa_attend(const msa_problem_t* p, const void* q, const void* k, const void* v,
+                        const int32_t* q2k, void* out, float* lse_opt,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* msa_select followed by msa_attend ("MiniMax 稀疏注意力", section 摘要).
+ * q2k_opt: optional; if not NULL receives the selection, else the selection
+ * lives in the workspace. */
+msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, const void* v,
+                         const void* q_idx, const void* k_idx, void* out, float* lse_opt,
+                         int32_t* q2k_opt, void* ws, size_t ws_bytes, void* stream);
+
+/* Reads the workspace status word written by the last call that used `ws`:
+ * waits for `stream`, stores the device code (0 = fine) in *code and returns
+ * MSA_OK, or MSA_ERR_DEVICE if the code is not 0.  This call synchronises. */
+msa_status_t msa_device_status(const void* ws, int32_t* code, void* stream);
+
+/* Stage timing (a measurement aid, not part of the method).  When `events` is
+ * not NULL, every later call records events[i] (cudaEvent_t values) on its
+ * stream right after its i-th stage, for i < n, so the caller can time each
+ * kernel with cudaEventElapsedTime against an event recorded before the call.
+ * Stages of msa_forward in order: 0 index scores, 1 top-k select, 2 block ->
+ * query lists (four small kernels), 3 KV-outer attention, 4 combine;
+ * msa_select records 0-1 and msa_attend 2-4 (numbered from 0 within the call).
+ * The setting is process-wide and not thread-safe; NULL turns it off.
+ * Returns the number of stages of msa_forward. */
+int32_t msa_set_stage_events(void* const* events, int32_t n);
+
+/* Number of kernel launches one call of `op` makes for problem `p` (without
+ * block_scores_opt, which adds one fill launch). */
+int32_t msa_launch_count(const msa_problem_t* p, int32_t op);
+
+/* Which kernel family a call of `op` runs for `p`: a static string naming the
+ * index-branch and main-branch kernels ("tc" = tcgen05/TMA path, "simt"). */
+const char* msa_kernel_path(const msa_problem_t* p, int32_t op);
+
+/* Human-readable name of a status code (static storage). */
+const char* msa_status_string(msa_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H */

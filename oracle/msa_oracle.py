@@ -55,11 +55,25 @@ import numpy as np
 NEG_INF = -np.inf
 
 
-def _f64(x) -> np.ndarray:
-    """Widen an input to float64 without changing its value."""
+def _np(x) -> np.ndarray:
+    """The stored values as a NumPy array (torch tensors are widened to fp32,
+    which holds every bf16 value exactly)."""
     if hasattr(x, "detach"):  # a torch tensor given by a test
         x = x.detach().float().cpu().numpy()
-    return np.asarray(x, dtype=np.float64)
+    return np.asarray(x)
+
+
+def _f64(x) -> np.ndarray:
+    """Widen an input to float64 without changing its value."""
+    return np.asarray(_np(x), dtype=np.float64)
+
+
+def _take(x, idx: np.ndarray) -> np.ndarray:
+    """Rows ``idx`` of x (NumPy array or torch tensor) as float64."""
+    if hasattr(x, "detach"):
+        import torch  # only when the caller handed in torch tensors
+        return _f64(x[torch.from_numpy(np.ascontiguousarray(idx))])
+    return _f64(np.asarray(x)[idx])
 
 
 def _rows(batch: int, q_len: int, rows: Optional[Iterable[int]]) -> list:
@@ -117,43 +131,45 @@ def select_row(block_max: np.ndarray, t: int, block_size: int, top_k: int) -> np
 
 def block_scores(q_idx, k_idx, q_pos0: int, block_size: int,
                  rows: Optional[Sequence[int]] = None) -> np.ndarray:
-    """Block maxima ``bmax[g, r, c]`` for every row r (or the given rows).
+    """Block maxima ``bmax[g, n, c]`` of the requested rows (default: all rows).
 
-    Blocks c > floor(t/block_size) are not visible to row r and hold -inf.
-    Shape ``[Hkv, B*Sq, nblk]`` with ``nblk = ceil(Skv / block_size)``; rows
-    not requested stay NaN.
+    Axis 1 follows ``rows`` (for a full run it is the row r = b*Sq + i).  Blocks
+    c > floor(t/block_size) are not visible to the row and hold -inf.  Shape
+    ``[Hkv, len(rows), nblk]`` with ``nblk = ceil(Skv / block_size)``.
     """
-    qi = _f64(q_idx)
-    ki = _f64(k_idx)
-    B, Sq, Hkv, _ = qi.shape
-    nblk = -(-ki.shape[1] // block_size)
-    out = np.full((Hkv, B * Sq, nblk), np.nan)
-    for r in _rows(B, Sq, rows):
+    B, Sq, Hkv, _ = q_idx.shape
+    nblk = -(-k_idx.shape[1] // block_size)
+    rl = _rows(B, Sq, rows)
+    out = np.full((Hkv, len(rl), nblk), NEG_INF)
+    kb, kb_of = None, -1
+    for n, r in enumerate(rl):
         b, i = divmod(r, Sq)
         t = q_pos0 + i
+        if b != kb_of:  # widen one sequence's index keys at a time
+            kb, kb_of = _f64(k_idx[b]), b
         # all groups at once: [t+1, di] @ [di, Hkv]
-        s = ki[b, : t + 1] @ qi[b, i].T
-        out[:, r, :] = NEG_INF
+        s = kb[: t + 1] @ _f64(q_idx[b, i]).T
         for g in range(Hkv):
             m = block_maxima_row(s[:, g], block_size)
-            out[g, r, : m.shape[0]] = m
+            out[g, n, : m.shape[0]] = m
     return out
 
 
 def select(q_idx, k_idx, q_pos0: int, block_size: int, top_k: int,
            rows: Optional[Sequence[int]] = None) -> np.ndarray:
-    """Per-(query, GQA group) selection ``q2k[Hkv, B*Sq, top_k]`` (int64).
+    """Per-(query, GQA group) selection ``q2k[Hkv, len(rows), top_k]`` (int64).
 
-    Rows not requested are filled with -2 (never a valid output value).
+    Axis 1 follows ``rows``; for a full run this is the library's
+    ``q2k[Hkv, B*Sq, top_k]`` layout.
     """
-    qi = _f64(q_idx)
-    B, Sq, Hkv, _ = qi.shape
-    bm = block_scores(q_idx, k_idx, q_pos0, block_size, rows)
-    q2k = np.full((Hkv, B * Sq, top_k), -2, dtype=np.int64)
-    for r in _rows(B, Sq, rows):
+    B, Sq, Hkv, _ = q_idx.shape
+    rl = _rows(B, Sq, rows)
+    bm = block_scores(q_idx, k_idx, q_pos0, block_size, rl)
+    q2k = np.empty((Hkv, len(rl), top_k), dtype=np.int64)
+    for n, r in enumerate(rl):
         t = q_pos0 + r % Sq
         for g in range(Hkv):
-            q2k[g, r] = select_row(bm[g, r], t, block_size, top_k)
+            q2k[g, n] = select_row(bm[g, n], t, block_size, top_k)
     return q2k
 
 
@@ -179,8 +195,8 @@ def attend_row(q_heads, k_seq_g, v_seq_g, blocks, t: int, block_size: int,
         hi = min((c + 1) * block_size, t + 1)
         keys.extend(range(lo, hi))
     J = np.array(sorted(keys), dtype=np.int64)
-    K = _f64(k_seq_g)[J]          # [n, D]
-    V = _f64(v_seq_g)[J]
+    K = _take(k_seq_g, J)         # [n, D]
+    V = _take(v_seq_g, J)
     z = scale * (_f64(q_heads) @ K.T)  # [G, n]
     m = z.max(axis=1, keepdims=True)
     w = np.exp(z - m)
@@ -192,30 +208,34 @@ def attend_row(q_heads, k_seq_g, v_seq_g, blocks, t: int, block_size: int,
 
 def attend(q, k, v, q2k, q_pos0: int, block_size: int,
            scale: Optional[float] = None, rows: Optional[Sequence[int]] = None):
-    """Main branch over a given selection: returns (out [B,Sq,Hq,D], lse [B,Sq,Hq]).
+    """Main branch over a given selection.
 
-    Unrequested rows stay NaN.  ``scale`` defaults to 1/sqrt(D) (reading R7).
+    ``q2k`` is ``[Hkv, len(rows), top_k]`` with axis 1 following ``rows``.
+    Returns (out, lse): ``[B, Sq, Hq, D]`` and ``[B, Sq, Hq]`` for a full run,
+    ``[len(rows), Hq, D]`` and ``[len(rows), Hq]`` when rows are given.
+    ``scale`` defaults to 1/sqrt(D) (reading R7).
     """
-    qf = _f64(q)
-    B, Sq, Hq, D = qf.shape
+    B, Sq, Hq, D = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     sel = np.asarray(q2k)
-    out = np.full((B, Sq, Hq, D), np.nan)
-    lse = np.full((B, Sq, Hq), np.nan)
-    kf = _f64(k)
-    vf = _f64(v)
-    for r in _rows(B, Sq, rows):
+    rl = _rows(B, Sq, rows)
+    out = np.empty((len(rl), Hq, D))
+    lse = np.empty((len(rl), Hq))
+    for n, r in enumerate(rl):
         b, i = divmod(r, Sq)
         t = q_pos0 + i
         for g in range(Hkv):
             hs = slice(g * G, (g + 1) * G)
-            o, ls = attend_row(qf[b, i, hs], kf[b, :, g], vf[b, :, g], sel[g, r],
+            # only the gathered key rows are widened (inside attend_row)
+            o, ls = attend_row(_f64(q[b, i, hs]), k[b, :, g], v[b, :, g], sel[g, n],
                                t, block_size, scale)
-            out[b, i, hs] = o
-            lse[b, i, hs] = ls
+            out[n, hs] = o
+            lse[n, hs] = ls
+    if rows is None:
+        return out.reshape(B, Sq, Hq, D), lse.reshape(B, Sq, Hq)
     return out, lse
 
 

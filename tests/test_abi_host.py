@@ -1,0 +1,124 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+entry point that include/msa.h declares, agrees with the header on the problem
+struct's layout, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from block_sparse_gqa_04_b200 import msa, workload
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_gqa_04_b200 import build
+    build.build()
+    return msa.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert names == sorted(msa.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", msa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (msa_\w+)", out))
+    for n in names:
+        assert n in exported, n
+        assert getattr(lib, n) is not None
+
+
+def test_problem_struct_layout_matches_header(tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "msa.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu\\n\", sizeof(msa_problem_t),"
+        " offsetof(msa_problem_t,q_pos0), offsetof(msa_problem_t,softmax_scale),"
+        " offsetof(msa_problem_t,reserved));return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    P = msa.Problem
+    want = [ctypes.sizeof(P), P.q_pos0.offset, P.softmax_scale.offset, P.reserved.offset]
+    assert [int(x) for x in got] == want
+
+
+def test_workspace_sizes(lib):
+    for name, w in workload.WORKLOADS.items():
+        p = msa.problem_of(w)
+        sel = msa.workspace_size(p, msa.OP_SELECT)
+        att = msa.workspace_size(p, msa.OP_ATTEND)
+        fwd = msa.workspace_size(p, msa.OP_FORWARD)
+        assert 0 < sel < fwd and 0 < att < fwd, name
+        # the partial outputs dominate: rows * heads * k * D elements
+        esz = 4 if w.dtype == "f32" else 2
+        assert att >= w.rows * w.num_q_heads * w.top_k * w.head_dim * esz
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("num_q_heads", 63, 1),          # not a multiple of num_kv_heads
+    ("block_size", 64, 2),
+    ("top_k", 33, 2),
+    ("top_k", 0, 1),
+    ("head_dim", 96, 2),
+    ("index_dim", 48, 2),
+    ("q_pos0", 131072, 1),           # q_pos0 + q_len > kv_len
+    ("batch", 0, 1),
+    ("reserved", 1, 1),
+    ("dtype", 7, 1),
+])
+def test_invalid_problems_are_rejected_on_the_host(lib, field, value, code):
+    p = msa.problem_of(workload.WORKLOADS["prefill_32k"])
+    setattr(p, field, value)
+    assert msa.workspace_size(p, msa.OP_FORWARD) == 0
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected before any launch
+    st = lib.msa_forward(ctypes.byref(p), fake, fake, fake, fake, fake, fake, None, None, fake,
+                         1 << 40, None)
+    assert st == code
+
+
+def test_null_misaligned_and_small_workspace(lib):
+    p = msa.problem_of(workload.WORKLOADS["tiny"])
+    need = msa.workspace_size(p, msa.OP_FORWARD)
+    a = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    ws = ctypes.c_void_p(1 << 24)
+    f = lib.msa_forward
+    assert f(ctypes.byref(p), None, a, a, a, a, a, None, None, ws, need, None) == 1
+    assert f(ctypes.byref(p), mis, a, a, a, a, a, None, None, ws, need, None) == 1
+    assert f(ctypes.byref(p), a, a, a, a, a, a, None, None, ctypes.c_void_p((1 << 24) + 16),
+             need, None) == 1                                   # workspace not 256-aligned
+    assert f(ctypes.byref(p), a, a, a, a, a, a, None, None, ws, need - 1, None) == 3
+    assert lib.msa_select(ctypes.byref(p), a, None, a, None, ws, need, None) == 1
+    assert lib.msa_attend(ctypes.byref(p), a, a, a, None, a, None, ws, need, None) == 1
+    assert lib.msa_device_status(None, None, None) == 1
+
+
+def test_empty_problem_launches_nothing(lib):
+    p = msa.problem_of(workload.WORKLOADS["tiny"].with_(q_len=0))
+    need = msa.workspace_size(p, msa.OP_FORWARD)
+    a = ctypes.c_void_p(1 << 20)
+    assert lib.msa_forward(ctypes.byref(p), a, a, a, a, a, a, None, None, ctypes.c_void_p(1 << 24),
+                           need, None) == 0
+    assert msa.launch_count(p) == 0
+
+
+def test_status_strings_and_launch_counts(lib):
+    for code, name in msa.STATUS.items():
+        assert lib.msa_status_string(code).decode().startswith(name)
+    p = msa.problem_of(workload.WORKLOADS["prefill_128k"])
+    assert msa.launch_count(p, msa.OP_SELECT) + msa.launch_count(p, msa.OP_ATTEND) == \
+        msa.launch_count(p, msa.OP_FORWARD)
+    assert "index" in msa.kernel_path(p) and "attn" in msa.kernel_path(p)

@@ -57,9 +57,10 @@ def test_golden_block_maxima_and_selection():
     sel = O.select(q_idx, k_idx, 0, Bk, k, rows=rows)
     for r in gd["rows"]:
         n = len(r["block_max"])
-        assert bm[r["group"], r["t"], :n].tolist() == r["block_max"], r["why"]
-        assert np.all(np.isneginf(bm[r["group"], r["t"], n:]))
-        assert sel[r["group"], r["t"]].tolist() == r["selection"], r["why"]
+        at = rows.index(r["t"])
+        assert bm[r["group"], at, :n].tolist() == r["block_max"], r["why"]
+        assert np.all(np.isneginf(bm[r["group"], at, n:]))
+        assert sel[r["group"], at].tolist() == r["selection"], r["why"]
 
 
 def test_golden_attention_closed_forms():
@@ -313,10 +314,11 @@ def test_row_subset_matches_full_run():
     full = O.forward(q, kk, v, qi, ki, 0, 16, 3)
     rows = [0, 17, 89, 90, 133, 179]
     part = O.forward(q, kk, v, qi, ki, 0, 16, 3, rows=rows)
-    for r in rows:
+    for n, r in enumerate(rows):
         b, i = divmod(r, 90)
-        assert np.array_equal(full[0][b, i], part[0][b, i])
-        assert np.array_equal(full[2][:, r], part[2][:, r])
+        assert np.array_equal(full[0][b, i], part[0][n])
+        assert np.array_equal(full[1][b, i], part[1][n])
+        assert np.array_equal(full[2][:, r], part[2][:, n])
 
 
 # ---------------------------------------------------------------------------
@@ -380,15 +382,16 @@ def test_planted_mistakes_are_caught(mutant, monkeypatch):
             qi, ki = O._f64(q_idx), O._f64(k_idx)
             B, Sq, Hkv, _ = qi.shape
             nblk = -(-ki.shape[1] // Bk)
-            out = np.full((Hkv, B * Sq, nblk), -np.inf)
-            for r in O._rows(B, Sq, rows):
+            rl = O._rows(B, Sq, rows)
+            out = np.full((Hkv, len(rl), nblk), -np.inf)
+            for n, r in enumerate(rl):
                 b, i = divmod(r, Sq)
                 t = q_pos0 + i
                 end = min(ki.shape[1], (t // Bk + 1) * Bk)
                 s = ki[b, :end] @ qi[b, i].T
                 for g in range(Hkv):
                     m = orig_bmax_row(s[:, g], Bk)
-                    out[g, r, : m.shape[0]] = m
+                    out[g, n, : m.shape[0]] = m
             return out
         monkeypatch.setattr(O, "block_scores", bs)
     elif mutant == "gqa_modulo":
@@ -397,16 +400,19 @@ def test_planted_mistakes_are_caught(mutant, monkeypatch):
             B, Sq, Hq, D = qf.shape
             Hkv = k.shape[2]
             scale = 1.0 / math.sqrt(D) if scale is None else scale
-            out = np.full((B, Sq, Hq, D), np.nan)
-            lse = np.full((B, Sq, Hq), np.nan)
-            for r in O._rows(B, Sq, rows):
+            rl = O._rows(B, Sq, rows)
+            out = np.full((len(rl), Hq, D), np.nan)
+            lse = np.full((len(rl), Hq), np.nan)
+            for n, r in enumerate(rl):
                 b, i = divmod(r, Sq)
                 for h in range(Hq):
                     g = h % Hkv   # wrong: interleaved instead of contiguous groups
                     o, ls = orig_attend_row(qf[b, i, h:h + 1], O._f64(k)[b, :, g],
-                                            O._f64(v)[b, :, g], np.asarray(q2k)[g, r],
+                                            O._f64(v)[b, :, g], np.asarray(q2k)[g, n],
                                             q_pos0 + i, Bk, scale)
-                    out[b, i, h], lse[b, i, h] = o[0], ls[0]
+                    out[n, h], lse[n, h] = o[0], ls[0]
+            if rows is None:
+                return out.reshape(B, Sq, Hq, D), lse.reshape(B, Sq, Hq)
             return out, lse
         monkeypatch.setattr(O, "attend", att)
     elif mutant == "missing_causal_in_local":
