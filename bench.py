@@ -412,11 +412,19 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows (0 = auto)")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="prefill length override (a smaller case of the same structure, "
+                         "e.g. for profiling); needles scale with the length")
     a = ap.parse_args()
     if a.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     world, rank, local = dist_setup()
     w = WORKLOADS[a.workload]
+    if a.seq:
+        if w.q_pos0 != 0 or w.batch != 1:
+            raise SystemExit("--seq applies to the prefill workloads")
+        w = w.with_(name=f"{w.name}@{a.seq}", q_len=a.seq, kv_len=a.seq,
+                    needles=max(1, w.needles * a.seq // w.q_len))
     peaks, peak_src = load_peaks()
 
     if a.impl == "reference":

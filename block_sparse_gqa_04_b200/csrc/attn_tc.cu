@@ -16,12 +16,14 @@
 //   * the softmax warps read their row, apply the scale and the causal cut of
 //     the local block, and write P (bf16) back over S in TMEM;
 //   * O = P V runs with P from TMEM and V as an MN-major shared-memory operand;
-//   * the softmax warps normalise O by the row sum, stage the bf16 rows in
-//     shared memory and bulk-store them (each warp its own 32 rows, which are
-//     contiguous in the entry-ordered partial states); the base-2
-//     log-normaliser goes with them.
-// TMEM holds two (S|P, O) buffers of 256 columns, so the S MMA of the next tile
-// runs while the softmax of this one is computed.
+//   * the softmax warps normalise O by the row sum, stage the bf16 rows in the
+//     tile's own Q buffer (free once S is done) and store them with TMA (each
+//     warp its own 32 rows, which are contiguous in the entry-ordered partial
+//     states); the base-2 log-normaliser goes with them.
+// Two softmax warpgroups take alternate tiles, each with its own TMEM buffer
+// pair (S|P, O) of 256 columns, so two tiles are in their softmax while the
+// tensor cores run the MMAs of their neighbours.  The softmax works on
+// 32-column chunks, which keeps the code small and the registers few.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -33,79 +35,48 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 192;                 // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr int kThreads = 320;                 // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
 constexpr int kRows = 128;
 constexpr int kQBytes = kRows * 128 * 2;      // 32 KB: 128 rows x 128 dims
 constexpr int kQHalf = kQBytes / 2;           // one 64-dim half
 constexpr int kKVBytes = 2 * kQBytes;         // K then V
-constexpr int kOutBytes = kRows * 128 * 2;    // staging of one tile's bf16 rows
+constexpr int kQStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdescS = tc::idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t kIdescO = tc::idesc_bf16_f32(128, 128, 0, 1);  // V is MN-major
 constexpr int kGroup = 16;                    // query heads per group
 constexpr int kQPerTile = kRows / kGroup;     // 8 gathered queries
 
+// Tiles are dealt to CTAs block-cyclically in chunks of kChunk consecutive
+// tiles: chunk k goes to CTA k % grid.  Consecutive tiles of a list stay on
+// one CTA (K/V is loaded once per chunk), while at any moment all CTAs work
+// inside the same narrow window of the tile order, i.e. on the same query
+// chunk of the same group, whose Q rows then stay resident in L2.
+constexpr int kChunk = 8;
+constexpr int kDesc = 4;  // tile descriptors in flight
+
+// What the producer warp tells the MMA warp and the softmax warps about a tile.
+struct TileDesc {
+  int c, e0, n, flags;     // flags: 1 new list, 2 last tile of its list here, kv stage << 2
+  int rows[kQPerTile];     // query rows of the gathered queries
+};
+
 struct Bars {
   uint64_t kv_full[2], kv_empty[2];
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[kQStages], q_empty[kQStages];
   uint64_t s_full[2], p_full[2], o_full[2], buf_empty[2];
+  uint64_t d_full[kDesc], d_empty[kDesc];
+  TileDesc desc[kDesc];
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 + 2 * kQBytes + 2 * kKVBytes + kOutBytes + 256;
+constexpr size_t kSmemBytes = 1024 + kQStages * kQBytes + 2 * kKVBytes + sizeof(Bars) + 64;
 
-__device__ __forceinline__ long long find_list(const int32_t* __restrict__ tile_off,
-                                               long long nlists, int tile) {
-  long long lo = 0, hi = nlists;  // tile_off[lo] <= tile < tile_off[hi]
-  while (hi - lo > 1) {
-    long long mid = (lo + hi) >> 1;
-    if (__ldg(tile_off + mid) <= tile) lo = mid; else hi = mid;
-  }
-  return lo;
+// The j-th tile of this CTA.
+__device__ __forceinline__ long long tile_of(int j) {
+  return ((long long)(j / kChunk) * gridDim.x + blockIdx.x) * kChunk + j % kChunk;
 }
-
-// Walks the tiles [t0, t1) in order, tracking the list each one belongs to.
-struct TileWalk {
-  const Problem* P;
-  const int32_t* tile_off;
-  const int32_t* list_off;
-  int tile, t1;
-  long long lid;
-  int c, g, b, e0, n;
-  bool new_list;
-  __device__ void decode() {
-    c = int(lid % P->nblk);
-    const long long rest = lid / P->nblk;
-    g = int((rest / P->nqc) % P->Hkv);
-    b = int(rest / ((long long)P->nqc * P->Hkv));
-    e0 = __ldg(list_off + lid) + (tile - __ldg(tile_off + lid)) * kQPerTile;
-    n = min(kQPerTile, __ldg(list_off + lid + 1) - e0);
-  }
-  __device__ void start(const Problem& Pr, const Lists& L, int a, int z) {
-    P = &Pr;
-    tile_off = L.tile_off;
-    list_off = L.list_off;
-    tile = a;
-    t1 = z;
-    lid = find_list(tile_off, Pr.nlists, a);
-    new_list = true;
-    decode();
-  }
-  // true if the tile after this one (in range) belongs to another list
-  __device__ bool last_of_list() const {
-    return tile + 1 >= t1 || tile + 1 >= __ldg(tile_off + lid + 1);
-  }
-  __device__ void next() {
-    ++tile;
-    new_list = false;
-    while (tile >= __ldg(tile_off + lid + 1)) {
-      ++lid;
-      new_list = true;
-    }
-    decode();
-  }
-};
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   return __all_sync(MSA_FULL_MASK, tc::mbar_wait(bar, parity, abort));
@@ -116,34 +87,69 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+
+// Maximum of 32 values (four independent chains of three-input maxima).
+__device__ __forceinline__ float max32(const uint32_t (&v)[32], float m) {
+  float a[4] = {m, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int x = 0; x < 32; x += 2)
+    a[(x >> 1) & 3] = max3(a[(x >> 1) & 3], __uint_as_float(v[x]), __uint_as_float(v[x + 1]));
+  return fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_v,
                const __grid_constant__ CUtensorMap tmap_o32,
                const __grid_constant__ CUtensorMap tmap_o16, Problem P, Lists L,
-               __nv_bfloat16* __restrict__ part_o, float* __restrict__ part_lse,
-               int* __restrict__ status) {
+               float* __restrict__ part_lse, int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qbuf = smem;                          // [2][32 KB]
-  uint8_t* kvbuf = qbuf + 2 * kQBytes;           // [2][K 32 KB | V 32 KB]
-  uint8_t* obuf = kvbuf + 2 * kKVBytes;          // 32 KB staging
-  Bars* bars = reinterpret_cast<Bars*>(obuf + kOutBytes);
+  uint8_t* qbuf = smem;                          // [3][32 KB]: Q, then output staging
+  uint8_t* kvbuf = qbuf + kQStages * kQBytes;    // [2][K 32 KB | V 32 KB]
+  Bars* bars = reinterpret_cast<Bars*>(kvbuf + 2 * kKVBytes);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      tc::mbar_init(&bars->q_full[s], 1);
+      tc::mbar_init(&bars->q_empty[s], 4);  // the four warps that stored the tile
+    }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->kv_full[s], 1);
       tc::mbar_init(&bars->kv_empty[s], 1);
-      tc::mbar_init(&bars->q_full[s], 1);
-      tc::mbar_init(&bars->q_empty[s], 1);
       tc::mbar_init(&bars->s_full[s], 1);
       tc::mbar_init(&bars->p_full[s], 4);
       tc::mbar_init(&bars->o_full[s], 1);
       tc::mbar_init(&bars->buf_empty[s], 4);
+    }
+    for (int d = 0; d < kDesc; ++d) {
+      tc::mbar_init(&bars->d_full[d], 1);
+      tc::mbar_init(&bars->d_empty[d], 5);  // the MMA thread and the four softmax warps
     }
     bars->abort = 0;
     tc::fence_mbar_init();
@@ -160,215 +166,270 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-
   const int total = __ldg(L.tile_off + P.nlists);
-  const int t0 = int((long long)total * blockIdx.x / gridDim.x);
-  const int t1 = int((long long)total * (blockIdx.x + 1) / gridDim.x);
   bool failed = false;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0 && t0 < t1) {
-      TileWalk w;
-      w.start(P, L, t0, t1);
-      int kv_stage = 0, q_stage = 0;
-      uint32_t kv_phase = 0, q_phase = 0;
-      for (int i = t0; i < t1; ++i) {
-        if (w.new_list) {
-          if (!tc::mbar_wait(&bars->kv_empty[kv_stage], kv_phase ^ 1, abort)) {
-            failed = true;
-            break;
+    // ---------------- producer: tile descriptors + TMA ----------------
+    // Lane l holds the record of tile jb + l of this CTA (prefetched one batch
+    // ahead); lane 0 waits for buffer space and issues the copies tile by tile.
+    const TileRec* recs = reinterpret_cast<const TileRec*>(L.tiles);
+    int kv_stage = 0, q_stage = 0;
+    uint32_t kv_phase = 0, q_phase = 0;
+    int prev_lid = -1;
+    auto fetch = [&](int j, TileRec& r) -> bool {
+      const long long tile = tile_of(j);
+      if (tile >= total) return false;
+      const uint4* src = reinterpret_cast<const uint4*>(recs + tile);
+      uint4* dst = reinterpret_cast<uint4*>(&r);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) dst[x] = __ldg(src + x);
+      return true;
+    };
+    TileRec cur, nxt;
+    bool cur_ok = fetch(lane, cur);
+    for (int jb = 0; !failed; jb += 32) {
+      if (!__any_sync(MSA_FULL_MASK, cur_ok)) break;
+      const bool nxt_ok = fetch(jb + 32 + lane, nxt);  // in flight while this batch is issued
+      const int j = jb + lane;
+      const long long nt = tile_of(j + 1);
+      const int last = cur_ok && !(nt < total && nt < cur.tend);
+      int lid_prev = __shfl_up_sync(MSA_FULL_MASK, cur.lid, 1);
+      if (lane == 0) lid_prev = prev_lid;
+      const int new_list = cur_ok && cur.lid != lid_prev;
+      prev_lid = __shfl_sync(MSA_FULL_MASK, cur.lid, 31);
+      for (int jj = 0; jj < 32; ++jj) {
+        if (!__shfl_sync(MSA_FULL_MASK, cur_ok, jj)) break;
+        const int jt = jb + jj;
+        const int tc_ = __shfl_sync(MSA_FULL_MASK, cur.c, jj);
+        const int tg = __shfl_sync(MSA_FULL_MASK, cur.g, jj);
+        const int tb = __shfl_sync(MSA_FULL_MASK, cur.b, jj);
+        const int te0 = __shfl_sync(MSA_FULL_MASK, cur.e0, jj);
+        const int tn = __shfl_sync(MSA_FULL_MASK, cur.n, jj);
+        const int tnew = __shfl_sync(MSA_FULL_MASK, new_list, jj);
+        const int tlast = __shfl_sync(MSA_FULL_MASK, last, jj);
+        int trow[kQPerTile];
+#pragma unroll
+        for (int e = 0; e < kQPerTile; ++e) trow[e] = __shfl_sync(MSA_FULL_MASK, cur.rows[e], jj);
+        bool good = true;
+        if (lane == 0) {
+          if (tnew) {
+            good = tc::mbar_wait(&bars->kv_empty[kv_stage], kv_phase ^ 1, abort);
+            if (good) {
+              uint64_t* fb = &bars->kv_full[kv_stage];
+              tc::mbar_arrive_expect_tx(fb, kKVBytes);
+              uint8_t* dst = kvbuf + kv_stage * kKVBytes;
+              const int key0 = tb * P.Skv + tc_ * P.Bk;
+              tc::tma_load_3d(dst, &tmap_k, fb, 0, tg, key0);
+              tc::tma_load_3d(dst + kQHalf, &tmap_k, fb, 64, tg, key0);
+              tc::tma_load_3d(dst + kQBytes, &tmap_v, fb, 0, tg, key0);
+              tc::tma_load_3d(dst + kQBytes + kQHalf, &tmap_v, fb, 64, tg, key0);
+            }
           }
-          uint64_t* fb = &bars->kv_full[kv_stage];
-          tc::mbar_arrive_expect_tx(fb, kKVBytes);
-          uint8_t* dst = kvbuf + kv_stage * kKVBytes;
-          const int key0 = w.b * P.Skv + w.c * P.Bk;
-          tc::tma_load_3d(dst, &tmap_k, fb, 0, w.g, key0);
-          tc::tma_load_3d(dst + kQHalf, &tmap_k, fb, 64, w.g, key0);
-          tc::tma_load_3d(dst + kQBytes, &tmap_v, fb, 0, w.g, key0);
-          tc::tma_load_3d(dst + kQBytes + kQHalf, &tmap_v, fb, 64, w.g, key0);
+          good = good && tc::mbar_wait(&bars->q_empty[q_stage], q_phase ^ 1, abort);
+          if (good) {
+            uint64_t* fb = &bars->q_full[q_stage];
+            tc::mbar_arrive_expect_tx(fb, uint32_t(tn) * 2 * kGroup * 128);
+            uint8_t* dst = qbuf + q_stage * kQBytes;
+#pragma unroll
+            for (int e = 0; e < kQPerTile; ++e) {
+              if (e < tn) {
+                const int qrow = trow[e] * P.Hq + tg * kGroup;
+                tc::tma_load_2d(dst + e * (kGroup * 128), &tmap_q, fb, 0, qrow);
+                tc::tma_load_2d(dst + kQHalf + e * (kGroup * 128), &tmap_q, fb, 64, qrow);
+              }
+            }
+          }
+          const int d = jt % kDesc;
+          good = good && tc::mbar_wait(&bars->d_empty[d], ((jt / kDesc) & 1) ^ 1, abort);
+          if (good) {
+            TileDesc& D = bars->desc[d];
+            D.c = tc_;
+            D.e0 = te0;
+            D.n = tn;
+            D.flags = (tnew ? 1 : 0) | (tlast ? 2 : 0) | ((tnew ? kv_stage : (kv_stage ^ 1)) << 2);
+#pragma unroll
+            for (int e = 0; e < kQPerTile; ++e) D.rows[e] = trow[e];
+            tc::mbar_arrive(&bars->d_full[d]);
+          }
+        }
+        if (!__shfl_sync(MSA_FULL_MASK, good, 0)) { failed = true; break; }
+        if (tnew) {
           kv_stage ^= 1;
           if (kv_stage == 0) kv_phase ^= 1;
         }
-        if (!tc::mbar_wait(&bars->q_empty[q_stage], q_phase ^ 1, abort)) {
-          failed = true;
-          break;
-        }
-        int rows[kQPerTile];
-#pragma unroll
-        for (int e = 0; e < kQPerTile; ++e)
-          rows[e] = e < w.n ? (__ldg(L.entries + w.e0 + e) >> 5) : 0;
-        uint64_t* fb = &bars->q_full[q_stage];
-        tc::mbar_arrive_expect_tx(fb, uint32_t(w.n) * 2 * kGroup * 128);
-        uint8_t* dst = qbuf + q_stage * kQBytes;
-#pragma unroll
-        for (int e = 0; e < kQPerTile; ++e) {
-          if (e < w.n) {
-            const int qrow = rows[e] * P.Hq + w.g * kGroup;
-            tc::tma_load_2d(dst + e * (kGroup * 128), &tmap_q, fb, 0, qrow);
-            tc::tma_load_2d(dst + kQHalf + e * (kGroup * 128), &tmap_q, fb, 64, qrow);
-          }
-        }
-        q_stage ^= 1;
-        if (q_stage == 0) q_phase ^= 1;
-        if (i + 1 < t1) w.next();
+        if (++q_stage == kQStages) { q_stage = 0; q_phase ^= 1; }
       }
+      cur = nxt;
+      cur_ok = nxt_ok;
     }
+    if (lane != 0) failed = false;  // lane 0 speaks for the warp
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0 && t0 < t1) {
-      TileWalk w;
-      w.start(P, L, t0, t1);
-      int kv_stage = 0, q_stage = 0;
-      uint32_t kv_phase = 0, q_phase = 0;
-      int tile_kv[2] = {0, 0};
-      bool tile_last[2] = {false, false};
-      // issues S = Q K^T of tile i into buffer i & 1
-      auto issue_s = [&](int i) -> bool {
-        const int buf = i & 1;
-        if (w.new_list) {
-          if (!tc::mbar_wait(&bars->kv_full[kv_stage], kv_phase, abort)) return false;
-          tile_kv[buf] = kv_stage;
-          kv_stage ^= 1;
-          if (kv_stage == 0) kv_phase ^= 1;
+    // Event loop: issue S = Q K^T of the next tile as soon as its descriptor,
+    // K/V, Q and TMEM buffer are ready, and O = P V of the oldest tile as soon
+    // as its P is in TMEM, whichever comes first.  At most two tiles are in
+    // flight (one per TMEM buffer).
+    if (lane == 0) {
+      uint32_t kv_phase[2] = {0, 0};
+      int ns = 0, np = 0;
+      uint32_t idle = 0;
+      while (tile_of(np) < total) {
+        bool progress = false;
+        if (ns < np + 2 && tile_of(ns) < total) {
+          const int d = ns % kDesc, buf = ns & 1, qs = ns % kQStages;
+          if (tc::mbar_test(&bars->d_full[d], (ns / kDesc) & 1)) {
+            const int flags = bars->desc[d].flags;
+            const int kvs = flags >> 2;
+            const bool ready =
+                (!(flags & 1) || tc::mbar_test(&bars->kv_full[kvs], kv_phase[kvs])) &&
+                tc::mbar_test(&bars->q_full[qs], (ns / kQStages) & 1) &&
+                tc::mbar_test(&bars->buf_empty[buf], ((ns >> 1) & 1) ^ 1);
+            if (ready) {
+              tc::tc_fence_after();
+              const uint32_t qa = tc::smem_addr(qbuf + qs * kQBytes);
+              const uint32_t ka = tc::smem_addr(kvbuf + kvs * kKVBytes);
+              const uint32_t dt = tmem + buf * 256;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * kQHalf + (kk & 3) * 32;
+                tc::mma_ss(dt, tc::sdesc_sw128(qa + off, 16, 1024),
+                           tc::sdesc_sw128(ka + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+              }
+              tc::mma_commit(&bars->s_full[buf]);
+              if (flags & 1) kv_phase[kvs] ^= 1;
+              ++ns;
+              progress = true;
+            }
+          }
+        }
+        if (np < ns && tc::mbar_test(&bars->p_full[np & 1], (np >> 1) & 1)) {
+          tc::tc_fence_after();
+          const int buf = np & 1, d = np % kDesc;
+          const int flags = bars->desc[d].flags;
+          const int kvs = flags >> 2;
+          const uint32_t va = tc::smem_addr(kvbuf + kvs * kKVBytes + kQBytes);
+          const uint32_t o = tmem + buf * 256 + 128;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            tc::mma_ts(o, tmem + buf * 256 + kk * 8, tc::sdesc_sw128(va + kk * 2048, kQHalf, 1024),
+                       kIdescO, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&bars->o_full[buf]);
+          if (flags & 2) tc::mma_commit(&bars->kv_empty[kvs]);
+          tc::mbar_arrive(&bars->d_empty[d]);
+          ++np;
+          progress = true;
+        }
+        if (progress) {
+          idle = 0;
         } else {
-          tile_kv[buf] = tile_kv[buf ^ 1];
+          if (++idle > tc::kWaitLimit || (idle > 64 && *abort)) { failed = true; break; }
+          if (idle > 64) __nanosleep(32);
         }
-        tile_last[buf] = w.last_of_list();
-        if (!tc::mbar_wait(&bars->q_full[q_stage], q_phase, abort)) return false;
-        if (!tc::mbar_wait(&bars->buf_empty[buf], (((i - t0) >> 1) & 1) ^ 1, abort)) return false;
-        tc::tc_fence_after();
-        const uint32_t qa = tc::smem_addr(qbuf + q_stage * kQBytes);
-        const uint32_t ka = tc::smem_addr(kvbuf + tile_kv[buf] * kKVBytes);
-        const uint32_t d = tmem + buf * 256;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          tc::mma_ss(d, tc::sdesc_sw128(qa + off, 16, 1024), tc::sdesc_sw128(ka + off, 16, 1024),
-                     kIdescS, kk > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&bars->s_full[buf]);
-        tc::mma_commit(&bars->q_empty[q_stage]);
-        q_stage ^= 1;
-        if (q_stage == 0) q_phase ^= 1;
-        return true;
-      };
-      if (!issue_s(t0)) failed = true;
-      for (int i = t0; i < t1 && !failed; ++i) {
-        const int buf = i & 1;
-        const int kvs = tile_kv[buf];
-        const bool last = tile_last[buf];
-        if (i + 1 < t1) {
-          w.next();
-          if (!issue_s(i + 1)) { failed = true; break; }
-        }
-        if (!tc::mbar_wait(&bars->p_full[buf], ((i - t0) >> 1) & 1, abort)) { failed = true; break; }
-        tc::tc_fence_after();
-        const uint32_t va = tc::smem_addr(kvbuf + kvs * kKVBytes + kQBytes);
-        const uint32_t o = tmem + buf * 256 + 128;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          tc::mma_ts(o, tmem + buf * 256 + kk * 8, tc::sdesc_sw128(va + kk * 2048, kQHalf, 1024),
-                     kIdescO, kk > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&bars->o_full[buf]);
-        if (last) tc::mma_commit(&bars->kv_empty[kvs]);
       }
     }
   } else {
-    // ---------------- softmax + epilogue ----------------
+    // ---------------- softmax + epilogue (two warpgroups) ----------------
+    const int wg = (warp - 2) >> 2;          // tiles j with j % 2 == wg, TMEM buffer wg
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+    const uint32_t sbase = tmem + lane_addr + wg * 256;  // S|P at +0, O at +128
     const float sl2 = P.scale * 1.4426950408889634f;
-    if (t0 < t1) {
-      TileWalk w;
-      w.start(P, L, t0, t1);
-      for (int i = t0; i < t1; ++i) {
-        const int buf = i & 1;
-        const uint32_t par = ((i - t0) >> 1) & 1;
-        const int el = row / kGroup, hh = row % kGroup;
-        const bool valid = el < w.n;
-        const int packed = valid ? __ldg(L.entries + w.e0 + el) : 0;
-        const int r = packed >> 5;
-        const long long t = P.q_pos0 + r % P.Sq;
-        const int lim = int(min(127LL, t - (long long)w.c * P.Bk));  // last visible column
-        if (!warp_wait(&bars->s_full[buf], par, abort)) { failed = true; break; }
-        tc::tc_fence_after();
-        float s[128];
+    const int el = row / kGroup, hh = row % kGroup;
+    for (int j = wg; tile_of(j) < total; j += 2) {
+      const int d = j % kDesc, qs = j % kQStages;
+      const uint32_t par = (j >> 1) & 1;
+      if (!warp_wait(&bars->d_full[d], (j / kDesc) & 1, abort)) { failed = true; break; }
+      const TileDesc& D = bars->desc[d];
+      const int c = D.c, e0 = D.e0, n = D.n;
+      const bool valid = el < n;
+      const long long t = P.q_pos0 + (valid ? D.rows[el] : 0) % P.Sq;
+      // last visible column of this row in block c (127 = the whole block)
+      const int lim = valid ? int(min(127LL, t - (long long)c * P.Bk)) : 127;
+      const bool full = __all_sync(MSA_FULL_MASK, lim >= 127);
+      if (!warp_wait(&bars->s_full[wg], par, abort)) { failed = true; break; }
+      tc::tc_fence_after();
+      // pass 1: row maximum
+      float m = -INFINITY;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t v[32];
+        tc::tmem_ld32(sbase + q4 * 32, v);
+        tc::tmem_ld_wait();
+        if (!full) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t v[32];
-          tc::tmem_ld32(tmem + lane_addr + buf * 256 + j * 32, v);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) s[j * 32 + x] = __uint_as_float(v[x]);
+          for (int x = 0; x < 32; ++x)
+            if (q4 * 32 + x > lim) v[x] = __float_as_uint(-INFINITY);
         }
-        float m = -INFINITY;
+        m = max32(v, m);
+      }
+      const float ms = m * sl2;
+      // pass 2: P = 2^(S*scale*log2e - max) in bf16, written over S, and its sum
+      float l = 0.f;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t v[32];
+        tc::tmem_ld32(sbase + q4 * 32, v);
+        tc::tmem_ld_wait();
+        uint32_t pw[16];
+        float l2[2] = {0.f, 0.f};
 #pragma unroll
-        for (int x = 0; x < 128; ++x)
-          if (x <= lim) m = fmaxf(m, s[x]);
-        const float ms = m * sl2;
-        float l = 0.f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t v[32];
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const int c0 = 64 * h + 2 * x;
-            const float p0 = c0 <= lim ? exp2f(fmaf(s[c0], sl2, -ms)) : 0.f;
-            const float p1 = c0 + 1 <= lim ? exp2f(fmaf(s[c0 + 1], sl2, -ms)) : 0.f;
-            l += p0 + p1;
-            v[x] = pack_bf16(p0, p1);
+        for (int x = 0; x < 32; x += 2) {
+          float p0 = ex2(fmaf(__uint_as_float(v[x]), sl2, -ms));
+          float p1 = ex2(fmaf(__uint_as_float(v[x + 1]), sl2, -ms));
+          if (!full) {
+            p0 = q4 * 32 + x <= lim ? p0 : 0.f;
+            p1 = q4 * 32 + x + 1 <= lim ? p1 : 0.f;
           }
-          tc::tmem_st32(tmem + lane_addr + buf * 256 + h * 32, v);
+          l2[(x >> 1) & 1] += p0 + p1;
+          pw[x >> 1] = pack_bf16(p0, p1);
         }
-        tc::tmem_st_wait();
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->p_full[buf]);
-        if (!warp_wait(&bars->o_full[buf], par, abort)) { failed = true; break; }
-        tc::tc_fence_after();
+        l += l2[0] + l2[1];
+        tmem_st16(sbase + q4 * 16, pw);  // P columns 16*q4.. cover S columns already read
+      }
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->p_full[wg]);
+      if (!warp_wait(&bars->o_full[wg], par, abort)) { failed = true; break; }
+      tc::tc_fence_after();
+      // Stage the normalised bf16 O row in this tile's Q buffer (S is done with
+      // it).  Each warp owns 32 consecutive rows (two gathered queries,
+      // contiguous in the entry-ordered partial states) and stores them itself
+      // with TMA.  The staging uses the 128-byte swizzle (16-byte chunk k of a
+      // row goes to chunk k ^ (row % 8)), which the TMA store undoes.
+      uint8_t* wst = qbuf + qs * kQBytes + quarter * 8192;
+      const float inv = 1.f / l;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t v[32];
+        tc::tmem_ld32(sbase + 128 + q4 * 32, v);
+        tc::tmem_ld_wait();
+        uint8_t* half = wst + (q4 >> 1) * 4096 + lane * 128;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t v[32];
-          tc::tmem_ld32(tmem + lane_addr + buf * 256 + 128 + j * 32, v);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) s[j * 32 + x] = __uint_as_float(v[x]);
+        for (int k8 = 0; k8 < 4; ++k8) {
+          uint4 u;
+          u.x = pack_bf16(__uint_as_float(v[8 * k8 + 0]) * inv, __uint_as_float(v[8 * k8 + 1]) * inv);
+          u.y = pack_bf16(__uint_as_float(v[8 * k8 + 2]) * inv, __uint_as_float(v[8 * k8 + 3]) * inv);
+          u.z = pack_bf16(__uint_as_float(v[8 * k8 + 4]) * inv, __uint_as_float(v[8 * k8 + 5]) * inv);
+          u.w = pack_bf16(__uint_as_float(v[8 * k8 + 6]) * inv, __uint_as_float(v[8 * k8 + 7]) * inv);
+          const int chunk = (q4 & 1) * 4 + k8;
+          *reinterpret_cast<uint4*>(half + ((chunk ^ (lane & 7)) << 4)) = u;
         }
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->buf_empty[buf]);
-        // Stage the normalised bf16 row.  Each warp owns 32 consecutive rows (two
-        // gathered queries, contiguous in the entry-ordered partial states) and
-        // stores them itself with TMA, so the epilogue needs no barrier across
-        // warps.  The staging uses the 128-byte swizzle (16-byte chunk j of a
-        // row goes to chunk j ^ (row % 8)), which the TMA store undoes.
-        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        __syncwarp();
-        const float inv = 1.f / l;
-        uint8_t* wst = obuf + quarter * 8192;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int c0 = 64 * h + 8 * j;
-            uint4 u;
-            u.x = pack_bf16(s[c0 + 0] * inv, s[c0 + 1] * inv);
-            u.y = pack_bf16(s[c0 + 2] * inv, s[c0 + 3] * inv);
-            u.z = pack_bf16(s[c0 + 4] * inv, s[c0 + 5] * inv);
-            u.w = pack_bf16(s[c0 + 6] * inv, s[c0 + 7] * inv);
-            *reinterpret_cast<uint4*>(wst + h * 4096 + lane * 128 + ((j ^ (lane & 7)) << 4)) = u;
-          }
-        }
-        if (valid) part_lse[(long long)(w.e0 + el) * kGroup + hh] = ms + log2f(l);
-        tc::fence_async_smem();
-        __syncwarp();
-        const int nrows = min(32, w.n * kGroup - quarter * 32);  // 0, 16 or 32
-        if (lane == 0 && nrows > 0) {
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->buf_empty[wg]);
+      if (valid) part_lse[(long long)(e0 + el) * kGroup + hh] = ms + __log2f(l);
+      tc::fence_async_smem();
+      __syncwarp();
+      const int nrows = min(32, n * kGroup - quarter * 32);  // 0, 16 or 32
+      if (lane == 0) {
+        if (nrows > 0) {
           const CUtensorMap* map = nrows == 32 ? &tmap_o32 : &tmap_o16;
-          const int grow = w.e0 * kGroup + quarter * 32;
+          const int grow = e0 * kGroup + quarter * 32;
 #pragma unroll
           for (int h = 0; h < 2; ++h)
             asm volatile(
@@ -377,11 +438,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 "r"(64 * h), "r"(grow), "r"(tc::smem_addr(wst + h * 4096))
                 : "memory");
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
-        if (i + 1 < t1) w.next();
+        // the Q buffer may be refilled once the store has read it
+        tc::mbar_arrive(&bars->q_empty[qs]);
+        tc::mbar_arrive(&bars->d_empty[d]);
       }
-      if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   if (failed) {
     bars->abort = 1;
@@ -476,7 +540,7 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
                                        int(kSmemBytes));
   if (e != cudaSuccess) return e;
   attn_tc_kernel<<<sm_count(), kThreads, kSmemBytes, s>>>(
-      mq, mk, mv, mo32, mo16, P, L, static_cast<__nv_bfloat16*>(part.o), part.lse2, status);
+      mq, mk, mv, mo32, mo16, P, L, part.lse2, status);
   return cudaGetLastError();
 }
 

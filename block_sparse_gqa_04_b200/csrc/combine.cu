@@ -6,12 +6,57 @@
 // exact softmax over the union of the slots' tokens is
 //     O = sum_s w_s o_s,   w_s = 2^(lse_s - M) / sum_u 2^(lse_u - M),
 // with M = max_s lse_s, and its natural-log normaliser is (M + log2 sum) ln 2.
-// One warp per (row, head); lane s reads slot s's lse, each lane owns D/32
-// output elements.
+//
+// One thread per (row, head, 8 output elements).  The partial states are in
+// entry order, [entry][head of group][D], so for one slot the threads of a
+// (row, group) read one contiguous run of G*D elements with 16-byte loads.
 #include "common.cuh"
 #include "internal.h"
 
 namespace msa {
+
+template <typename PT>
+struct Vec8;
+template <>
+struct Vec8<__nv_bfloat16> {
+  uint4 u;
+  __device__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ void to_f32(float (&f)[8]) const {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(h[i]);
+      f[2 * i] = x.x;
+      f[2 * i + 1] = x.y;
+    }
+  }
+  __device__ static void store(__nv_bfloat16* p, const float (&f)[8]) {
+    uint4 u;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+template <>
+struct Vec8<float> {
+  float4 a, b;
+  __device__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ void to_f32(float (&f)[8]) const {
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+  __device__ static void store(float* p, const float (&f)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+};
 
 template <typename PT, typename OT, int D>
 __global__ void __launch_bounds__(256) combine_kernel(Problem P, const int32_t* __restrict__ pos,
@@ -19,58 +64,55 @@ __global__ void __launch_bounds__(256) combine_kernel(Problem P, const int32_t* 
                                                       const float* __restrict__ part_lse,
                                                       OT* __restrict__ out,
                                                       float* __restrict__ lse_out) {
-  constexpr int EPL = D / 32;
-  const int lane = threadIdx.x & 31;
-  const long long wid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (wid >= (long long)P.T * P.Hq) return;
-  const int r = int(wid / P.Hq), h = int(wid % P.Hq);
-  const int g = h / P.G, hh = h % P.G;
-  // lane s < K looks after slot s: its partial sits at entry position pos[g, r, s]
-  long long prow = -1;
-  float ls = -INFINITY;
-  if (lane < P.K) {
-    const int e = pos[((long long)g * P.T + r) * P.K + lane];
-    if (e >= 0) {
-      prow = (long long)e * P.G + hh;
-      ls = part_lse[prow];
+  constexpr int CH = D / 8;  // 8-element chunks per head row
+  const long long n = (long long)P.T * P.Hq * CH;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int ch = int(idx % CH);
+    const long long rh = idx / CH;          // r * Hq + h
+    const int h = int(rh % P.Hq);
+    const int r = int(rh / P.Hq);
+    const int g = h / P.G, hh = h % P.G;
+    const int32_t* ps = pos + ((long long)g * P.T + r) * P.K;
+    float M = -INFINITY;
+    for (int s = 0; s < P.K; ++s) {
+      const int e = __ldg(ps + s);
+      if (e >= 0) M = fmaxf(M, __ldg(part_lse + (long long)e * P.G + hh));
     }
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    float sum = 0.f;
+    if (M != -INFINITY) {
+      for (int s = 0; s < P.K; ++s) {
+        const int e = __ldg(ps + s);
+        if (e < 0) continue;
+        const long long prow = (long long)e * P.G + hh;
+        const float w = exp2f(__ldg(part_lse + prow) - M);
+        sum += w;
+        Vec8<PT> v;
+        v.load(part_o + prow * D + ch * 8);
+        float f[8];
+        v.to_f32(f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, f[i], acc[i]);
+      }
+      const float inv = 1.f / sum;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] *= inv;
+    }
+    Vec8<OT>::store(out + rh * D + ch * 8, acc);
+    if (lse_out && ch == 0)
+      lse_out[rh] = M == -INFINITY ? -INFINITY : (M + log2f(sum)) * 0.6931471805599453f;
   }
-  const float M = warp_max_f32(ls);
-  float o[EPL];
-#pragma unroll
-  for (int x = 0; x < EPL; ++x) o[x] = 0.f;
-  OT* dst = out + ((long long)r * P.Hq + h) * D + lane * EPL;
-  if (M == -INFINITY) {  // no valid slot
-#pragma unroll
-    for (int x = 0; x < EPL; ++x) dst[x] = from_f32<OT>(0.f);
-    if (lse_out && lane == 0) lse_out[(long long)r * P.Hq + h] = -INFINITY;
-    return;
-  }
-  const float w = ls == -INFINITY ? 0.f : exp2f(ls - M);
-  const float sum = warp_sum_f32(w);
-  const float inv = 1.f / sum;
-  unsigned valid = __ballot_sync(MSA_FULL_MASK, w > 0.f);
-  while (valid) {
-    const int s = __ffs(valid) - 1;
-    valid &= valid - 1;
-    const float ws = __shfl_sync(MSA_FULL_MASK, w, s) * inv;
-    const long long ps = __shfl_sync(MSA_FULL_MASK, prow, s);
-    float pv[EPL];
-    load_vec<PT, EPL>(part_o + ps * D + lane * EPL, pv);
-#pragma unroll
-    for (int x = 0; x < EPL; ++x) o[x] = fmaf(ws, pv[x], o[x]);
-  }
-#pragma unroll
-  for (int x = 0; x < EPL; ++x) dst[x] = from_f32<OT>(o[x]);
-  if (lse_out && lane == 0)
-    lse_out[(long long)r * P.Hq + h] = (M + log2f(sum)) * 0.6931471805599453f;
 }
 
 template <typename T, int D>
 static cudaError_t launch_t(const Problem& P, const int32_t* pos, const Partials& part,
                             void* out, float* lse, cudaStream_t s) {
-  long long warps = (long long)P.T * P.Hq;
-  long long blocks = (warps + 7) / 8;
+  const long long n = (long long)P.T * P.Hq * (D / 8);
+  long long blocks = (n + 255) / 256;
+  if (blocks > 148LL * 32) blocks = 148LL * 32;
   combine_kernel<T, T, D><<<unsigned(blocks), 256, 0, s>>>(P, pos, (const T*)part.o,
                                                            part.lse2, (T*)out, lse);
   return cudaGetLastError();

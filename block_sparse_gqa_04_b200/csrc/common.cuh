@@ -21,12 +21,34 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
   return __float2bfloat16_rn(x);
 }
 
-// Loads N consecutive elements starting at p (N*sizeof(T) bytes, aligned to that
-// size or 16 bytes) into fp32 registers.
+// Loads N consecutive elements starting at p into fp32 registers, in the widest
+// chunks (16, 8 or 4 bytes) that N * sizeof(T) allows; p must be aligned to
+// that chunk size (callers pass rows whose offsets are multiples of N).
 template <typename T, int N>
 __device__ __forceinline__ void load_vec(const T* __restrict__ p, float (&out)[N]) {
+  constexpr int bytes = N * int(sizeof(T));
+  if constexpr (bytes % 16 == 0) {
+    constexpr int per = 16 / sizeof(T);
 #pragma unroll
-  for (int i = 0; i < N; ++i) out[i] = to_f32(p[i]);
+    for (int c = 0; c < N / per; ++c) {
+      const uint4 u = *reinterpret_cast<const uint4*>(p + c * per);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int i = 0; i < per; ++i) out[c * per + i] = to_f32(e[i]);
+    }
+  } else if constexpr (bytes % 8 == 0) {
+    constexpr int per = 8 / sizeof(T);
+#pragma unroll
+    for (int c = 0; c < N / per; ++c) {
+      const uint2 u = *reinterpret_cast<const uint2*>(p + c * per);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int i = 0; i < per; ++i) out[c * per + i] = to_f32(e[i]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) out[i] = to_f32(p[i]);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -49,13 +71,13 @@ __device__ __forceinline__ int key_block(uint64_t key) {
   return int(0xffffffffu - uint32_t(key & 0xffffffffu));
 }
 
+// Warp-wide maximum of 64-bit keys: the maximum high word, then the maximum
+// low word among the lanes holding that high word (two redux instructions).
 __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    uint64_t w = __shfl_xor_sync(MSA_FULL_MASK, v, o);
-    v = w > v ? w : v;
-  }
-  return v;
+  const uint32_t hi = uint32_t(v >> 32), lo = uint32_t(v);
+  const uint32_t mh = __reduce_max_sync(MSA_FULL_MASK, hi);
+  const uint32_t ml = __reduce_max_sync(MSA_FULL_MASK, hi == mh ? lo : 0u);
+  return (uint64_t(mh) << 32) | ml;
 }
 
 __device__ __forceinline__ float warp_max_f32(float v) {

@@ -249,21 +249,27 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
             break;
           }
           tc::tc_fence_after();
-          float m = -INFINITY;
+          // all 128 columns in flight at once, then a tree of maxima (eight
+          // independent chains) instead of one 128-long dependent chain
+          uint32_t v[4][32];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t v[32];
-            tc::tmem_ld32(tmem + lane_addr + kAccCol + slot * 128 + j * 32, v);
-            tc::tmem_ld_wait();
-            if (lim >= j * 32 + 31) {
+          for (int j = 0; j < 4; ++j)
+            tc::tmem_ld32(tmem + lane_addr + kAccCol + slot * 128 + j * 32, v[j]);
+          tc::tmem_ld_wait();
+          float mx[8];
 #pragma unroll
-              for (int x = 0; x < 32; ++x) m = fmaxf(m, __uint_as_float(v[x]));
-            } else {
+          for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
+          if (__all_sync(MSA_FULL_MASK, lim >= 127)) {
 #pragma unroll
-              for (int x = 0; x < 32; ++x)
-                if (j * 32 + x <= lim) m = fmaxf(m, __uint_as_float(v[x]));
-            }
+            for (int x = 0; x < 128; ++x)
+              mx[x & 7] = fmaxf(mx[x & 7], __uint_as_float(v[x >> 5][x & 31]));
+          } else {
+#pragma unroll
+            for (int x = 0; x < 128; ++x)
+              if (x <= lim) mx[x & 7] = fmaxf(mx[x & 7], __uint_as_float(v[x >> 5][x & 31]));
           }
+          const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
           tc::tc_fence_before();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&bars->acc_empty[slot]);

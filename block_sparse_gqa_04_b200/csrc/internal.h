@@ -35,7 +35,25 @@ struct Lists {
   int32_t* tile_off;  // [nlists + 1]
   int32_t* entries;   // [Hkv * T * K] packed (row << 5) | slot, grouped by list
   int32_t* pos;       // [Hkv, T, K] position of (g, row, slot) in entries, or -1
+  int32_t* tiles;     // [max_tiles] TileRec, one per 128-row tile (tensor-core path)
 };
+
+// One 128-row tile of gathered queries: everything the KV-outer kernel needs to
+// stage it, precomputed so that kernel's producer reads one record per tile.
+struct TileRec {
+  int c, g, b;        // block, group, sequence
+  int e0, n;          // first entry and number of gathered queries (<= 8)
+  int tend;           // first tile of the next list
+  int lid;            // list id (low 31 bits)
+  int pad;
+  int rows[8];        // query rows of the gathered queries
+};
+static_assert(sizeof(TileRec) == 64, "TileRec is 64 bytes");
+
+// Upper bound on the number of 128-row tiles.
+inline long long max_tiles(const Problem& P) {
+  return (long long)P.Hkv * P.T * P.K / P.qpt + P.nlists + 1;
+}
 
 // Partial softmax states, stored in entry order: the G query heads of entry e
 // occupy rows e*G .. e*G+G-1, so one tile of gathered queries writes one
@@ -59,6 +77,8 @@ cudaError_t launch_topk(const Problem& P, const float* bmax, int32_t* q2k, cudaS
 // --- block -> query lists ---------------------------------------------------
 cudaError_t launch_invert(const Problem& P, const int32_t* q2k, const Lists& L,
                           int32_t* status, cudaStream_t s);
+// Fills L.tiles from the list offsets (one record per tile).
+cudaError_t launch_tile_records(const Problem& P, const Lists& L, cudaStream_t s);
 
 // --- main branch ------------------------------------------------------------
 cudaError_t launch_attn_simt(const Problem& P, const void* q, const void* k, const void* v,

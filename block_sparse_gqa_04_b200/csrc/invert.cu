@@ -113,6 +113,33 @@ __global__ void scatter_kernel(Problem P, const int32_t* __restrict__ q2k, Lists
   }
 }
 
+// One thread per tile: find its list (binary search over the tile offsets)
+// and write the tile's record.
+__global__ void tile_records_kernel(Problem P, Lists L) {
+  const int total = L.tile_off[P.nlists];
+  for (int tile = blockIdx.x * blockDim.x + threadIdx.x; tile < total;
+       tile += gridDim.x * blockDim.x) {
+    long long lo = 0, hi = P.nlists;  // tile_off[lo] <= tile < tile_off[hi]
+    while (hi - lo > 1) {
+      const long long mid = (lo + hi) >> 1;
+      if (L.tile_off[mid] <= tile) lo = mid; else hi = mid;
+    }
+    TileRec rec;
+    rec.c = int(lo % P.nblk);
+    const long long rest = lo / P.nblk;
+    rec.g = int((rest / P.nqc) % P.Hkv);
+    rec.b = int(rest / ((long long)P.nqc * P.Hkv));
+    rec.e0 = L.list_off[lo] + (tile - L.tile_off[lo]) * P.qpt;
+    rec.n = min(P.qpt, L.list_off[lo + 1] - rec.e0);
+    rec.tend = L.tile_off[lo + 1];
+    rec.lid = int(lo & 0x7fffffff);
+    rec.pad = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) rec.rows[e] = e < rec.n ? (L.entries[rec.e0 + e] >> 5) : 0;
+    reinterpret_cast<TileRec*>(L.tiles)[tile] = rec;
+  }
+}
+
 static unsigned grid_for(long long n, int threads) {
   long long b = (n + threads - 1) / threads;
   if (b > 148LL * 64) b = 148LL * 64;
@@ -126,6 +153,11 @@ cudaError_t launch_invert(const Problem& P, const int32_t* q2k, const Lists& L,
   count_kernel<<<grid_for(n, 256), 256, 0, s>>>(P, q2k, L, status);
   scan_kernel<<<1, 1024, 0, s>>>(P, L);
   scatter_kernel<<<grid_for(n, 256), 256, 0, s>>>(P, q2k, L);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_records(const Problem& P, const Lists& L, cudaStream_t s) {
+  tile_records_kernel<<<grid_for(max_tiles(P), 256), 256, 0, s>>>(P, L);
   return cudaGetLastError();
 }
 

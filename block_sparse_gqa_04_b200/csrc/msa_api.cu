@@ -65,8 +65,8 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
 
 // Workspace layout (each region 256-byte aligned, in this order).
 struct Layout {
-  size_t status, bmax, q2k, counts, cursor, list_off, tile_off, entries, pos, part_o, part_lse,
-      total;
+  size_t status, bmax, q2k, counts, cursor, list_off, tile_off, entries, pos, tiles, part_o,
+      part_lse, total;
 };
 
 Layout layout(const Problem& P, int op) {
@@ -87,6 +87,7 @@ Layout layout(const Problem& P, int op) {
     L.tile_off = take(size_t(P.nlists + 1) * 4);
     L.entries = take(size_t(P.Hkv) * T * P.K * 4);
     L.pos = take(size_t(P.Hkv) * T * P.K * 4);
+    L.tiles = take(size_t(msa::max_tiles(P)) * sizeof(msa::TileRec));
     // one partial state per (entry, head of the group): Hkv*T*K*G = T*Hq*K rows
     L.part_o = take(T * P.Hq * P.K * size_t(P.D) * esz);
     L.part_lse = take(T * P.Hq * P.K * sizeof(float));
@@ -139,13 +140,15 @@ msa_status_t run_attend(const Problem& P, const void* q, const void* k, const vo
                         cudaStream_t s) {
   msa::Lists lists{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.cursor),
                    at<int32_t>(ws, L.list_off), at<int32_t>(ws, L.tile_off),
-                   at<int32_t>(ws, L.entries), at<int32_t>(ws, L.pos)};
+                   at<int32_t>(ws, L.entries), at<int32_t>(ws, L.pos),
+                   at<int32_t>(ws, L.tiles)};
   msa::Partials part{at<void>(ws, L.part_o), at<float>(ws, L.part_lse)};
+  const bool tc = msa::attn_tc_supported(P);
   cudaError_t e = msa::launch_invert(P, q2k, lists, at<int32_t>(ws, L.status), s);
+  if (e == cudaSuccess && tc) e = msa::launch_tile_records(P, lists, s);
   stage_mark(s);
   if (e == cudaSuccess) {
-    e = msa::attn_tc_supported(P)
-            ? msa::launch_attn_tc(P, q, k, v, lists, part, at<int32_t>(ws, L.status), s)
+    e = tc ? msa::launch_attn_tc(P, q, k, v, lists, part, at<int32_t>(ws, L.status), s)
             : msa::launch_attn_simt(P, q, k, v, lists, part, s);
     stage_mark(s);
   }
@@ -250,7 +253,8 @@ int32_t msa_launch_count(const msa_problem_t* p, int32_t op) {
   Problem P;
   if (resolve(p, &P) != MSA_OK || P.T == 0) return 0;
   const int sel = 2;                               // index + top-k
-  const int att = msa::kLaunchesInvert + 2;        // lists + attention + combine
+  // lists (+ tile records on the tensor-core path) + attention + combine
+  const int att = msa::kLaunchesInvert + (msa::attn_tc_supported(P) ? 1 : 0) + 2;
   switch (op) {
     case MSA_OP_SELECT: return sel;
     case MSA_OP_ATTEND: return att;
