@@ -112,10 +112,38 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+// Two-wide fp32 helpers (sm_100 packed FMA / add / mul on a 64-bit pair).
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  return (uint64_t(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// bf16x2 of the two fp32 halves (low half -> low 16 bits), round to nearest even
+__device__ __forceinline__ uint32_t to_bf16x2(uint64_t x) {
+  return pack_bf16(__uint_as_float(uint32_t(x)), __uint_as_float(uint32_t(x >> 32)));
+}
+// 2^x for both bf16 halves
+__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
+  uint32_t y;
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
   return y;
+}
+// the two bf16 halves widened to fp32 (exact)
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t p) {
+  return (uint64_t(p & 0xffff0000u) << 32) | uint64_t(p << 16);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -366,29 +394,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         m = max32(v, m);
       }
       const float ms = m * sl2;
-      // pass 2: P = 2^(S*scale*log2e - max) in bf16, written over S, and its sum
-      float l = 0.f;
+      // pass 2: P = 2^(S*scale*log2e - max), written over S, and its sum, two
+      // columns at a time: the scaled logits (packed fp32x2 FMA) are rounded to
+      // bf16 and exponentiated with the bf16x2 exp2, which gives P in the bf16
+      // the P V product takes at half the exp2-unit cost
+      const uint64_t sl2x2 = f2(sl2, sl2), nmsx2 = f2(-ms, -ms);
+      uint64_t lsum[2] = {0, 0};
 #pragma unroll 1
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t v[32];
         tc::tmem_ld32(sbase + q4 * 32, v);
         tc::tmem_ld_wait();
+        if (!full) {
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if (q4 * 32 + x > lim) v[x] = __float_as_uint(-INFINITY);
+        }
         uint32_t pw[16];
-        float l2[2] = {0.f, 0.f};
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(v[x]), sl2, -ms));
-          float p1 = ex2(fmaf(__uint_as_float(v[x + 1]), sl2, -ms));
-          if (!full) {
-            p0 = q4 * 32 + x <= lim ? p0 : 0.f;
-            p1 = q4 * 32 + x + 1 <= lim ? p1 : 0.f;
-          }
-          l2[(x >> 1) & 1] += p0 + p1;
-          pw[x >> 1] = pack_bf16(p0, p1);
+          const uint64_t z = fma2((uint64_t(v[x + 1]) << 32) | v[x], sl2x2, nmsx2);
+          const uint32_t pp = ex2_bf16x2(to_bf16x2(z));
+          lsum[(x >> 1) & 1] = add2(lsum[(x >> 1) & 1], bf16x2_to_f2(pp));
+          pw[x >> 1] = pp;
         }
-        l += l2[0] + l2[1];
         tmem_st16(sbase + q4 * 16, pw);  // P columns 16*q4.. cover S columns already read
       }
+      const uint64_t lsx = add2(lsum[0], lsum[1]);
+      const float l = __uint_as_float(uint32_t(lsx)) + __uint_as_float(uint32_t(lsx >> 32));
       tc::tmem_st_wait();
       tc::tc_fence_before();
       __syncwarp();
@@ -402,6 +435,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       // row goes to chunk k ^ (row % 8)), which the TMA store undoes.
       uint8_t* wst = qbuf + qs * kQBytes + quarter * 8192;
       const float inv = 1.f / l;
+      const uint64_t invx2 = f2(inv, inv);
 #pragma unroll 1
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t v[32];
@@ -411,10 +445,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
         for (int k8 = 0; k8 < 4; ++k8) {
           uint4 u;
-          u.x = pack_bf16(__uint_as_float(v[8 * k8 + 0]) * inv, __uint_as_float(v[8 * k8 + 1]) * inv);
-          u.y = pack_bf16(__uint_as_float(v[8 * k8 + 2]) * inv, __uint_as_float(v[8 * k8 + 3]) * inv);
-          u.z = pack_bf16(__uint_as_float(v[8 * k8 + 4]) * inv, __uint_as_float(v[8 * k8 + 5]) * inv);
-          u.w = pack_bf16(__uint_as_float(v[8 * k8 + 6]) * inv, __uint_as_float(v[8 * k8 + 7]) * inv);
+          u.x = to_bf16x2(mul2((uint64_t(v[8 * k8 + 1]) << 32) | v[8 * k8 + 0], invx2));
+          u.y = to_bf16x2(mul2((uint64_t(v[8 * k8 + 3]) << 32) | v[8 * k8 + 2], invx2));
+          u.z = to_bf16x2(mul2((uint64_t(v[8 * k8 + 5]) << 32) | v[8 * k8 + 4], invx2));
+          u.w = to_bf16x2(mul2((uint64_t(v[8 * k8 + 7]) << 32) | v[8 * k8 + 6], invx2));
           const int chunk = (q4 & 1) * 4 + k8;
           *reinterpret_cast<uint4*>(half + ((chunk ^ (lane & 7)) << 4)) = u;
         }

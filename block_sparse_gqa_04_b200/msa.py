@@ -212,11 +212,13 @@ def attend(q, k, v, q2k, *, q_pos0: int = 0, block_size: int = 128,
 def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, top_k: int = 16,
             softmax_scale: float = 0.0, return_lse: bool = False, return_q2k: bool = False,
             workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-            device=None):
+            device=None, check_device_status: bool = False):
     """Index branch + main branch.  Returns out (and lse, q2k when asked).
 
     CUDA tensors are used in place.  Host tensors (ideally pinned) are copied to
     ``device`` (default ``cuda``) before the call and the results copied back.
+    ``check_device_status`` waits for the call and raises if the device
+    recorded a problem (a bounded wait that gave up).
     """
     host = not q.is_cuda
     if host:
@@ -237,6 +239,10 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
     _check(load().msa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx),
                               _ptr(k_idx), _ptr(o), _ptr(lse), _ptr(q2k), ctypes.c_void_p(wp),
                               wn, _stream(dev)), "msa_forward")
+    if check_device_status:
+        code = ctypes.c_int32(0)
+        _check(load().msa_device_status(ctypes.c_void_p(wp), ctypes.byref(code), _stream(dev)),
+               "msa_forward (device status)")
     if host:
         if out is not None:
             out.copy_(o, non_blocking=out.is_pinned())

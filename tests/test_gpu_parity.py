@@ -14,8 +14,8 @@ import torch
 from block_sparse_gqa_04_b200 import msa
 from block_sparse_gqa_04_b200.workload import WORKLOADS, Workload, make_inputs, sample_rows
 from oracle import msa_oracle as O
-from parity_util import (assert_close_out, check_selection, check_selection_properties,
-                         to_np)
+from parity_util import (assert_close_lse, assert_close_out, check_selection,
+                         check_selection_properties, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -63,7 +63,7 @@ def _positions(w: Workload, rows):
 def _run_forward(w: Workload, gpu):
     return msa.forward(gpu["q"], gpu["k"], gpu["v"], gpu["q_idx"], gpu["k_idx"],
                        q_pos0=w.q_pos0, block_size=w.block_size, top_k=w.top_k,
-                       return_lse=True, return_q2k=True)
+                       return_lse=True, return_q2k=True, check_device_status=True)
 
 
 def _forward_parity(w: Workload, rows=None):
@@ -82,7 +82,7 @@ def _forward_parity(w: Workload, rows=None):
     go = to_np(out).reshape(w.rows, w.num_q_heads, w.head_dim)[rl]
     gl = to_np(lse).reshape(w.rows, w.num_q_heads)[rl]
     assert_close_out(go, oo, w.dtype)
-    np.testing.assert_allclose(gl, ol, rtol=1e-4 if w.dtype == "f32" else 2e-3, atol=1e-4)
+    assert_close_lse(gl, ol, w.dtype)
     return dec, agree, und
 
 
@@ -107,7 +107,7 @@ def test_attend_with_oracle_selection(name):
                           block_size=w.block_size, return_lse=True, check_device_status=True)
     oo, ol = O.attend(cpu["q"], cpu["k"], cpu["v"], oq2k, w.q_pos0, w.block_size)
     assert_close_out(to_np(out), oo, w.dtype)
-    np.testing.assert_allclose(to_np(lse), ol, rtol=1e-4 if w.dtype == "f32" else 2e-3, atol=1e-4)
+    assert_close_lse(to_np(lse), ol, w.dtype)
 
 
 @pytest.mark.parametrize("name", ["tiny", "bf16_ragged", "chunk_unaligned", "decode_small",
