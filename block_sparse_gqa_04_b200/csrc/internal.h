@@ -36,6 +36,7 @@ struct Lists {
   int32_t* entries;   // [Hkv * T * K] packed (row << 5) | slot, grouped by list
   int32_t* pos;       // [Hkv, T, K] position of (g, row, slot) in entries, or -1
   int32_t* tiles;     // [max_tiles] TileRec, one per 128-row tile (tensor-core path)
+  int32_t* seg_sums;  // [2 * ceil(nlists / 2048)] scan scratch
 };
 
 // One 128-row tile of gathered queries: everything the KV-outer kernel needs to
@@ -72,6 +73,11 @@ cudaError_t launch_index_simt(const Problem& P, const void* q_idx, const void* k
 bool index_tc_supported(const Problem& P);
 cudaError_t launch_index_tc(const Problem& P, const void* q_idx, const void* k_idx,
                             float* bmax, int32_t* status, cudaStream_t s);
+// Block maxima for a few query rows per sequence (decode): a TMA-fed stream over
+// k_idx (bf16, index_dim 128).
+bool index_decode_supported(const Problem& P);
+cudaError_t launch_index_decode(const Problem& P, const void* q_idx, const void* k_idx,
+                                float* bmax, int32_t* status, cudaStream_t s);
 cudaError_t launch_topk(const Problem& P, const float* bmax, int32_t* q2k, cudaStream_t s);
 
 // --- block -> query lists ---------------------------------------------------
@@ -95,6 +101,6 @@ cudaError_t launch_combine(const Problem& P, const int32_t* pos, const Partials&
 constexpr int kStatusBadEntry = 1;
 
 // Kernel launches made by each launcher (for msa_launch_count).
-constexpr int kLaunchesInvert = 4;
+constexpr int kLaunchesInvert = 5;
 
 }  // namespace msa

@@ -8,7 +8,8 @@
 //   prep     zero the counters
 //   count    histogram of list ids (invalid q2k entries flag the status word)
 //   scan     exclusive prefix sums of the counts (entry offsets) and of the
-//            128-row tiles each list needs (tile offsets)
+//            128-row tiles each list needs (tile offsets), in two passes over
+//            segments of lists (segment sums, then offsets)
 //   scatter  place each entry at its list offset + an atomic cursor, and record
 //            that position per (group, row, slot) for the combine
 // The order inside a list is not fixed, which does not change any result: the
@@ -54,43 +55,88 @@ __global__ void count_kernel(Problem P, const int32_t* __restrict__ q2k, Lists L
   }
 }
 
-// One CTA of 1024 threads; each thread owns a contiguous run of lists.
-__global__ void __launch_bounds__(1024) scan_kernel(Problem P, Lists L) {
-  __shared__ int s_e[1024];
-  __shared__ int s_t[1024];
-  const long long n = P.nlists;
-  const int tid = threadIdx.x;
-  const long long per = (n + 1023) / 1024;
-  const long long lo = min(n, per * tid), hi = min(n, lo + per);
-  int se = 0, st = 0;
-  for (long long i = lo; i < hi; ++i) {
-    const int c = L.counts[i];
-    se += c;
-    st += (c + P.qpt - 1) / P.qpt;
+// Two-kernel exclusive scan of the list counts (entry offsets) and of the
+// tiles each list needs (tile offsets).  scan_sums: CTA s sums segment s of
+// kScanSeg lists.  scan_apply: CTA s adds the sums of the segments before it
+// and scans its own segment.
+constexpr int kScanSeg = 2048;  // lists per segment (256 threads x 8)
+
+__device__ __forceinline__ int tiles_of(int count, int qpt) { return (count + qpt - 1) / qpt; }
+
+// block-wide inclusive scan of (a, b) pairs over 256 threads
+__device__ __forceinline__ void block_scan2(int& a, int& b, int* sa, int* sb) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int xa = __shfl_up_sync(MSA_FULL_MASK, a, o), xb = __shfl_up_sync(MSA_FULL_MASK, b, o);
+    if (lane >= o) { a += xa; b += xb; }
   }
-  s_e[tid] = se;
-  s_t[tid] = st;
+  if (lane == 31) { sa[w] = a; sb[w] = b; }
   __syncthreads();
-  // Hillis-Steele inclusive scan over the 1024 partial sums
-  for (int off = 1; off < 1024; off <<= 1) {
-    int ae = tid >= off ? s_e[tid - off] : 0;
-    int at = tid >= off ? s_t[tid - off] : 0;
-    __syncthreads();
-    s_e[tid] += ae;
-    s_t[tid] += at;
-    __syncthreads();
+  if (w == 0) {
+    int ta = lane < 8 ? sa[lane] : 0, tb = lane < 8 ? sb[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const int xa = __shfl_up_sync(MSA_FULL_MASK, ta, o), xb = __shfl_up_sync(MSA_FULL_MASK, tb, o);
+      if (lane >= o) { ta += xa; tb += xb; }
+    }
+    if (lane < 8) { sa[lane] = ta; sb[lane] = tb; }
   }
-  int ee = s_e[tid] - se, et = s_t[tid] - st;  // exclusive
-  for (long long i = lo; i < hi; ++i) {
-    const int c = L.counts[i];
-    L.list_off[i] = ee;
-    L.tile_off[i] = et;
-    ee += c;
-    et += (c + P.qpt - 1) / P.qpt;
+  __syncthreads();
+  if (w > 0) { a += sa[w - 1]; b += sb[w - 1]; }
+}
+
+__global__ void __launch_bounds__(256) scan_sums_kernel(Problem P, Lists L, int2* seg_sums) {
+  __shared__ int sa[8], sb[8];
+  const long long lo = (long long)blockIdx.x * kScanSeg;
+  int e = 0, t = 0;
+  for (int k = 0; k < kScanSeg / 256; ++k) {
+    const long long i = lo + k * 256 + threadIdx.x;
+    if (i < P.nlists) {
+      const int c = L.counts[i];
+      e += c;
+      t += tiles_of(c, P.qpt);
+    }
   }
-  if (tid == 1023) {
-    L.list_off[n] = s_e[1023];
-    L.tile_off[n] = s_t[1023];
+  block_scan2(e, t, sa, sb);
+  if (threadIdx.x == 255) seg_sums[blockIdx.x] = make_int2(e, t);
+}
+
+__global__ void __launch_bounds__(256) scan_apply_kernel(Problem P, Lists L,
+                                                         const int2* __restrict__ seg_sums) {
+  __shared__ int sa[8], sb[8];
+  __shared__ int base_e, base_t;
+  // offsets of this segment: the sums of all segments before it
+  int e = 0, t = 0;
+  for (int s = threadIdx.x; s < blockIdx.x; s += 256) {
+    e += seg_sums[s].x;
+    t += seg_sums[s].y;
+  }
+  block_scan2(e, t, sa, sb);
+  if (threadIdx.x == 255) { base_e = e; base_t = t; }
+  __syncthreads();
+  int run_e = base_e, run_t = base_t;
+  const long long lo = (long long)blockIdx.x * kScanSeg;
+  for (int k = 0; k < kScanSeg / 256; ++k) {
+    const long long i = lo + k * 256 + threadIdx.x;
+    const int c = i < P.nlists ? L.counts[i] : 0;
+    int ie = c, it = tiles_of(c, P.qpt);
+    __syncthreads();  // sa/sb reuse
+    block_scan2(ie, it, sa, sb);
+    if (i < P.nlists) {
+      L.list_off[i] = run_e + ie - c;
+      L.tile_off[i] = run_t + it - tiles_of(c, P.qpt);
+    }
+    // the last thread's inclusive sums advance the running offsets
+    __shared__ int tot_e, tot_t;
+    if (threadIdx.x == 255) { tot_e = ie; tot_t = it; }
+    __syncthreads();
+    run_e += tot_e;
+    run_t += tot_t;
+  }
+  if (lo + kScanSeg >= P.nlists && threadIdx.x == 0) {
+    L.list_off[P.nlists] = run_e;
+    L.tile_off[P.nlists] = run_t;
   }
 }
 
@@ -149,9 +195,11 @@ static unsigned grid_for(long long n, int threads) {
 cudaError_t launch_invert(const Problem& P, const int32_t* q2k, const Lists& L,
                           int32_t* status, cudaStream_t s) {
   const long long n = (long long)P.Hkv * P.T * P.K;
+  const unsigned segs = unsigned((P.nlists + kScanSeg - 1) / kScanSeg);
   prep_kernel<<<grid_for(P.nlists, 256), 256, 0, s>>>(P, L);
   count_kernel<<<grid_for(n, 256), 256, 0, s>>>(P, q2k, L, status);
-  scan_kernel<<<1, 1024, 0, s>>>(P, L);
+  scan_sums_kernel<<<segs, 256, 0, s>>>(P, L, reinterpret_cast<int2*>(L.seg_sums));
+  scan_apply_kernel<<<segs, 256, 0, s>>>(P, L, reinterpret_cast<const int2*>(L.seg_sums));
   scatter_kernel<<<grid_for(n, 256), 256, 0, s>>>(P, q2k, L);
   return cudaGetLastError();
 }

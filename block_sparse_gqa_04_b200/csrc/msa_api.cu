@@ -65,8 +65,8 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
 
 // Workspace layout (each region 256-byte aligned, in this order).
 struct Layout {
-  size_t status, bmax, q2k, counts, cursor, list_off, tile_off, entries, pos, tiles, part_o,
-      part_lse, total;
+  size_t status, bmax, q2k, counts, cursor, list_off, tile_off, entries, pos, tiles, seg_sums,
+      part_o, part_lse, total;
 };
 
 Layout layout(const Problem& P, int op) {
@@ -88,6 +88,7 @@ Layout layout(const Problem& P, int op) {
     L.entries = take(size_t(P.Hkv) * T * P.K * 4);
     L.pos = take(size_t(P.Hkv) * T * P.K * 4);
     L.tiles = take(size_t(msa::max_tiles(P)) * sizeof(msa::TileRec));
+    L.seg_sums = take(size_t((P.nlists + 2047) / 2048) * 8);
     // one partial state per (entry, head of the group): Hkv*T*K*G = T*Hq*K rows
     L.part_o = take(T * P.Hq * P.K * size_t(P.D) * esz);
     L.part_lse = take(T * P.Hq * P.K * sizeof(float));
@@ -123,9 +124,10 @@ msa_status_t run_select(const Problem& P, const void* q_idx, const void* k_idx, 
   cudaError_t e = cudaSuccess;
   if (bscores) e = msa::launch_fill(bscores, size_t(P.Hkv) * P.T * P.nblk, -INFINITY, s);
   if (e == cudaSuccess) {
-    e = msa::index_tc_supported(P)
-            ? msa::launch_index_tc(P, q_idx, k_idx, bmax, at<int32_t>(ws, L.status), s)
-            : msa::launch_index_simt(P, q_idx, k_idx, bmax, s);
+    int32_t* status = at<int32_t>(ws, L.status);
+    e = msa::index_tc_supported(P)       ? msa::launch_index_tc(P, q_idx, k_idx, bmax, status, s)
+        : msa::index_decode_supported(P) ? msa::launch_index_decode(P, q_idx, k_idx, bmax, status, s)
+                                         : msa::launch_index_simt(P, q_idx, k_idx, bmax, s);
     stage_mark(s);
   }
   if (e == cudaSuccess) {
@@ -141,7 +143,7 @@ msa_status_t run_attend(const Problem& P, const void* q, const void* k, const vo
   msa::Lists lists{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.cursor),
                    at<int32_t>(ws, L.list_off), at<int32_t>(ws, L.tile_off),
                    at<int32_t>(ws, L.entries), at<int32_t>(ws, L.pos),
-                   at<int32_t>(ws, L.tiles)};
+                   at<int32_t>(ws, L.tiles), at<int32_t>(ws, L.seg_sums)};
   msa::Partials part{at<void>(ws, L.part_o), at<float>(ws, L.part_lse)};
   const bool tc = msa::attn_tc_supported(P);
   cudaError_t e = msa::launch_invert(P, q2k, lists, at<int32_t>(ws, L.status), s);
@@ -266,13 +268,16 @@ int32_t msa_launch_count(const msa_problem_t* p, int32_t op) {
 const char* msa_kernel_path(const msa_problem_t* p, int32_t op) {
   Problem P;
   if (resolve(p, &P) != MSA_OK) return "invalid";
-  const bool itc = msa::index_tc_supported(P), atc = msa::attn_tc_supported(P);
+  const bool atc = msa::attn_tc_supported(P);
+  const int ik = msa::index_tc_supported(P) ? 0 : msa::index_decode_supported(P) ? 1 : 2;
+  static const char* sel[3] = {"index:tc", "index:stream", "index:simt"};
+  static const char* fwd[3][2] = {{"index:tc attn:simt", "index:tc attn:tc"},
+                                  {"index:stream attn:simt", "index:stream attn:tc"},
+                                  {"index:simt attn:simt", "index:simt attn:tc"}};
   switch (op) {
-    case MSA_OP_SELECT: return itc ? "index:tc" : "index:simt";
+    case MSA_OP_SELECT: return sel[ik];
     case MSA_OP_ATTEND: return atc ? "attn:tc" : "attn:simt";
-    case MSA_OP_FORWARD:
-      return itc ? (atc ? "index:tc attn:tc" : "index:tc attn:simt")
-                 : (atc ? "index:simt attn:tc" : "index:simt attn:simt");
+    case MSA_OP_FORWARD: return fwd[ik][atc ? 1 : 0];
   }
   return "invalid";
 }
