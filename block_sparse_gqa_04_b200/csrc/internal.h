@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/msa.h"
+
 namespace msa {
 
 // Query rows of one sequence handled as one unit of the block -> query lists.
@@ -26,6 +28,9 @@ struct Problem {
   bool f32;         // fp32 tensors (else bf16)
   long long nlists; // B * Hkv * nqc * nblk
 };
+
+// Shape checks of the C ABI: fills *P from *p or returns why it cannot.
+msa_status_t resolve_problem(const msa_problem_t* p, Problem* P);
 
 // Views into the caller's workspace.
 struct Lists {

@@ -163,6 +163,10 @@ msa_status_t run_attend(const Problem& P, const void* q, const void* k, const vo
 
 }  // namespace
 
+namespace msa {
+msa_status_t resolve_problem(const msa_problem_t* p, Problem* P) { return resolve(p, P); }
+}  // namespace msa
+
 extern "C" {
 
 size_t msa_workspace_size(const msa_problem_t* p, int32_t op) {
@@ -290,6 +294,9 @@ const char* msa_status_string(msa_status_t s) {
     case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE: workspace too small";
     case MSA_ERR_CUDA: return "MSA_ERR_CUDA: CUDA launch or call failed";
     case MSA_ERR_DEVICE: return "MSA_ERR_DEVICE: invalid q2k entry seen on the device";
+    case MSA_ERR_TOO_LARGE:
+      return "MSA_ERR_TOO_LARGE: block maxima exceed the 4 MiB static scratch of "
+             "msa_select_static";
   }
   return "MSA_ERR_UNKNOWN";
 }

@@ -22,11 +22,12 @@ MSA_BF16, MSA_F32 = 0, 1
 OP_SELECT, OP_ATTEND, OP_FORWARD = 0, 1, 2
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
-          3: "MSA_ERR_WORKSPACE", 4: "MSA_ERR_CUDA", 5: "MSA_ERR_DEVICE"}
+          3: "MSA_ERR_WORKSPACE", 4: "MSA_ERR_CUDA", 5: "MSA_ERR_DEVICE",
+          6: "MSA_ERR_TOO_LARGE"}
 
 EXPORTED = ("msa_workspace_size", "msa_select", "msa_attend", "msa_forward",
             "msa_device_status", "msa_set_stage_events", "msa_launch_count", "msa_kernel_path",
-            "msa_status_string")
+            "msa_status_string", "msa_select_static")
 STAGES = ("index", "topk", "lists", "attn", "combine")
 
 
@@ -78,6 +79,8 @@ def load() -> ctypes.CDLL:
         lib.msa_kernel_path.restype = ctypes.c_char_p
         lib.msa_status_string.argtypes = [i32]
         lib.msa_status_string.restype = ctypes.c_char_p
+        lib.msa_select_static.argtypes = [pp, vp, vp, vp, vp, vp]
+        lib.msa_select_static.restype = i32
         _lib = lib
     return _lib
 
@@ -184,6 +187,28 @@ def select(q_idx: torch.Tensor, k_idx: torch.Tensor, *, q_pos0: int = 0, block_s
     _check(load().msa_select(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(q2k), _ptr(bs),
                              ctypes.c_void_p(wp), wn, _stream(dev)), "msa_select")
     return (q2k, bs) if return_block_scores else q2k
+
+
+def select_static(q_idx: torch.Tensor, k_idx: torch.Tensor, q2k: torch.Tensor, *,
+                  q_pos0: int = 0, block_size: int = 128,
+                  device_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Index branch through msa_select_static, which allocates nothing: the
+    caller passes the output q2k [Hkv, B*Sq, top_k] int32 (and optionally a
+    one-element int32 device tensor that receives the device status word).
+    For callers that cannot lend the library device memory; the library's
+    fixed scratch is shared, so calls must not overlap on the GPU."""
+    _require_cuda(q_idx, k_idx, q2k, device_status)
+    B, Sq, Hkv, di = q_idx.shape
+    Skv = k_idx.shape[1]
+    if q2k.dtype != torch.int32 or tuple(q2k.shape[:2]) != (Hkv, B * Sq):
+        raise ValueError("q2k must be int32 [Hkv, B*Sq, top_k]")
+    if device_status is not None and device_status.dtype != torch.int32:
+        raise ValueError("device_status must be an int32 tensor")
+    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, q2k.shape[2], q_idx.dtype, q_pos0)
+    _check(load().msa_select_static(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(q2k),
+                                    _ptr(device_status), _stream(q_idx.device)),
+           "msa_select_static")
+    return q2k
 
 
 def attend(q, k, v, q2k, *, q_pos0: int = 0, block_size: int = 128,

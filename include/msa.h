@@ -58,7 +58,8 @@ typedef enum {
   MSA_ERR_UNSUPPORTED = 2,   /* valid shape outside what the kernels cover    */
   MSA_ERR_WORKSPACE = 3,     /* ws_bytes smaller than msa_workspace_size()    */
   MSA_ERR_CUDA = 4,          /* a CUDA call or launch failed                  */
-  MSA_ERR_DEVICE = 5         /* the device recorded an invalid q2k entry      */
+  MSA_ERR_DEVICE = 5,        /* the device recorded an invalid q2k entry      */
+  MSA_ERR_TOO_LARGE = 6      /* problem exceeds msa_select_static's scratch   */
 } msa_status_t;
 
 typedef enum { MSA_BF16 = 0, MSA_F32 = 1 } msa_dtype_t;
@@ -121,6 +122,31 @@ msa_status_t msa_attend(const msa_problem_t* p, const void* q, const void* k, co
 msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, const void* v,
                          const void* q_idx, const void* k_idx, void* out, float* lse_opt,
                          int32_t* q2k_opt, void* ws, size_t ws_bytes, void* stream);
+
+/* msa_select without a workspace: the same index branch and selection,
+ * writing the same q2k, with its scratch in a fixed 256-byte-aligned device
+ * buffer inside this library (status word + block maxima), so the call
+ * allocates no memory at all and takes no workspace.  The pages have no
+ * counterpart of this entry point; it is for callers that cannot hand the
+ * library device memory: a host runtime that has reserved the whole device up
+ * front (a KV-cache pool, say) and has no allocator left to lend, or a C caller
+ * without a device allocator.
+ *  - Limit: the block maxima, num_kv_heads * batch * q_len * nblk * 4 bytes,
+ *    must fit in 4 MiB (e.g. 32 decode rows at 1M tokens with 4 groups);
+ *    larger problems return MSA_ERR_TOO_LARGE before anything is launched.
+ *  - Setup: the first call on each device (with that device current) looks up
+ *    the buffer's address with cudaGetSymbolAddress, which may load the
+ *    library's device code; make that first call before any stream capture.
+ *  - The buffer is shared by every call on a device: calls whose work overlaps
+ *    on the GPU (other streams, other threads) race on it and must be
+ *    serialised by the caller.
+ *  - Each call clears the status word first (the only scratch that must start
+ *    at zero).  device_status_opt: optional device int32; if not NULL it
+ *    receives, in stream order, the call's status word (0 = fine; 2 = a bounded
+ *    wait inside a tensor-core kernel gave up).
+ * Other arguments and errors as msa_select. */
+msa_status_t msa_select_static(const msa_problem_t* p, const void* q_idx, const void* k_idx,
+                               int32_t* q2k, int32_t* device_status_opt, void* stream);
 
 /* Reads the workspace status word written by the last call that used `ws`:
  * waits for `stream`, stores the device code (0 = fine) in *code and returns
