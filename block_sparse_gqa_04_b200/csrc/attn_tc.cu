@@ -11,7 +11,8 @@
 // One persistent CTA per SM takes a contiguous share of the tiles.  Per tile:
 //   * TMA loads the block's K and V (128 keys x 128 dims each, 128-byte swizzle)
 //     into one of two buffers, once per list, and gathers the 8 queries' Q rows
-//     (16 heads x 128 dims, contiguous in memory) with two boxes per query;
+//     (16 heads x 128 dims, contiguous in memory) with two boxes per query,
+//     issued by sixteen lanes at once;
 //   * S = Q K^T (both K-major in shared memory) lands in TMEM, one row per lane;
 //   * the softmax warps read their row, apply the scale and the causal cut of
 //     the local block, and write P (bf16) back over S in TMEM;
@@ -22,8 +23,10 @@
 //     states); the base-2 log-normaliser goes with them.
 // Two softmax warpgroups take alternate tiles, each with its own TMEM buffer
 // pair (S|P, O) of 256 columns, so two tiles are in their softmax while the
-// tensor cores run the MMAs of their neighbours.  The softmax works on
-// 32-column chunks, which keeps the code small and the registers few.
+// tensor cores run the MMAs of their neighbours; a buffer's next S = Q K^T is
+// issued as soon as its previous P V has completed, so it overlaps the
+// previous tile's epilogue.  Each softmax thread holds its whole S row (and
+// later its O row) in registers, so a tile costs one TMEM round trip each.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -202,6 +205,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     // Lane l holds the record of tile jb + l of this CTA (prefetched one batch
     // ahead); lane 0 waits for buffer space and issues the copies tile by tile.
     const TileRec* recs = reinterpret_cast<const TileRec*>(L.tiles);
+    // the Q rows of the current query chunk are gathered once per selected
+    // block: keep them in L2 ahead of the streaming partial-state writes
+    const uint64_t q_policy = tc::policy_evict_last();
     int kv_stage = 0, q_stage = 0;
     uint32_t kv_phase = 0, q_phase = 0;
     int prev_lid = -1;
@@ -255,19 +261,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
           }
           good = good && tc::mbar_wait(&bars->q_empty[q_stage], q_phase ^ 1, abort);
-          if (good) {
-            uint64_t* fb = &bars->q_full[q_stage];
-            tc::mbar_arrive_expect_tx(fb, uint32_t(tn) * 2 * kGroup * 128);
-            uint8_t* dst = qbuf + q_stage * kQBytes;
+          if (good) tc::mbar_arrive_expect_tx(&bars->q_full[q_stage], uint32_t(tn) * 2 * kGroup * 128);
+        }
+        // the Q boxes of the tile, issued together: lane 2e + h copies half h
+        // of query e (one copy per lane instead of sixteen from one lane)
+        if (__shfl_sync(MSA_FULL_MASK, good, 0) && lane < 2 * tn) {
+          const int e = lane >> 1, h = lane & 1;
+          int qr = trow[0];
 #pragma unroll
-            for (int e = 0; e < kQPerTile; ++e) {
-              if (e < tn) {
-                const int qrow = trow[e] * P.Hq + tg * kGroup;
-                tc::tma_load_2d(dst + e * (kGroup * 128), &tmap_q, fb, 0, qrow);
-                tc::tma_load_2d(dst + kQHalf + e * (kGroup * 128), &tmap_q, fb, 64, qrow);
-              }
-            }
-          }
+          for (int x = 1; x < kQPerTile; ++x) qr = e == x ? trow[x] : qr;
+          tc::tma_load_2d_hint(qbuf + q_stage * kQBytes + h * kQHalf + e * (kGroup * 128), &tmap_q,
+                               &bars->q_full[q_stage], 64 * h, qr * P.Hq + tg * kGroup, q_policy);
+        }
+        if (lane == 0) {
           const int d = jt % kDesc;
           good = good && tc::mbar_wait(&bars->d_empty[d], ((jt / kDesc) & 1) ^ 1, abort);
           if (good) {
@@ -297,7 +303,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     // Event loop: issue S = Q K^T of the next tile as soon as its descriptor,
     // K/V, Q and TMEM buffer are ready, and O = P V of the oldest tile as soon
     // as its P is in TMEM, whichever comes first.  At most two tiles are in
-    // flight (one per TMEM buffer).
+    // flight (one per TMEM buffer).  The barriers are tested without blocking
+    // (a blocking test of one would hide the other becoming ready).
     if (lane == 0) {
       uint32_t kv_phase[2] = {0, 0};
       int ns = 0, np = 0;
@@ -306,13 +313,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         bool progress = false;
         if (ns < np + 2 && tile_of(ns) < total) {
           const int d = ns % kDesc, buf = ns & 1, qs = ns % kQStages;
-          if (tc::mbar_test(&bars->d_full[d], (ns / kDesc) & 1)) {
+          if (tc::mbar_poll(&bars->d_full[d], (ns / kDesc) & 1)) {
             const int flags = bars->desc[d].flags;
             const int kvs = flags >> 2;
+            // S overwrites only the S|P columns of its buffer, which are free
+            // once the P V product of the buffer's previous tile has completed;
+            // the O columns may still be draining in the epilogue
             const bool ready =
-                (!(flags & 1) || tc::mbar_test(&bars->kv_full[kvs], kv_phase[kvs])) &&
-                tc::mbar_test(&bars->q_full[qs], (ns / kQStages) & 1) &&
-                tc::mbar_test(&bars->buf_empty[buf], ((ns >> 1) & 1) ^ 1);
+                (!(flags & 1) || tc::mbar_poll(&bars->kv_full[kvs], kv_phase[kvs])) &&
+                tc::mbar_poll(&bars->q_full[qs], (ns / kQStages) & 1) &&
+                tc::mbar_poll(&bars->o_full[buf], ((ns >> 1) & 1) ^ 1);
             if (ready) {
               tc::tc_fence_after();
               const uint32_t qa = tc::smem_addr(qbuf + qs * kQBytes);
@@ -331,7 +341,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
           }
         }
-        if (np < ns && tc::mbar_test(&bars->p_full[np & 1], (np >> 1) & 1)) {
+        // O = P V needs its P and the O columns drained by the epilogue of the
+        // buffer's previous tile
+        if (np < ns && tc::mbar_poll(&bars->p_full[np & 1], (np >> 1) & 1) &&
+            tc::mbar_poll(&bars->buf_empty[np & 1], ((np >> 1) & 1) ^ 1)) {
           tc::tc_fence_after();
           const int buf = np & 1, d = np % kDesc;
           const int flags = bars->desc[d].flags;
@@ -353,7 +366,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
           idle = 0;
         } else {
           if (++idle > tc::kWaitLimit || (idle > 64 && *abort)) { failed = true; break; }
-          if (idle > 64) __nanosleep(32);
+          if (idle > 8) __nanosleep(20);
         }
       }
     }
@@ -379,46 +392,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       const bool full = __all_sync(MSA_FULL_MASK, lim >= 127);
       if (!warp_wait(&bars->s_full[wg], par, abort)) { failed = true; break; }
       tc::tc_fence_after();
-      // pass 1: row maximum
-      float m = -INFINITY;
-#pragma unroll 1
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t v[32];
-        tc::tmem_ld32(sbase + q4 * 32, v);
-        tc::tmem_ld_wait();
-        if (!full) {
+      // the whole S row in registers: four loads, one wait
+      uint32_t v[4][32];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tc::tmem_ld32(sbase + q4 * 32, v[q4]);
+      tc::tmem_ld_wait();
+      if (!full) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
           for (int x = 0; x < 32; ++x)
-            if (q4 * 32 + x > lim) v[x] = __float_as_uint(-INFINITY);
-        }
-        m = max32(v, m);
+            if (q4 * 32 + x > lim) v[q4][x] = __float_as_uint(-INFINITY);
       }
+      float m = max32(v[0], -INFINITY);
+      m = fmaxf(fmaxf(m, max32(v[1], -INFINITY)), fmaxf(max32(v[2], -INFINITY),
+                                                       max32(v[3], -INFINITY)));
       const float ms = m * sl2;
-      // pass 2: P = 2^(S*scale*log2e - max), written over S, and its sum, two
-      // columns at a time: the scaled logits (packed fp32x2 FMA) are rounded to
-      // bf16 and exponentiated with the bf16x2 exp2, which gives P in the bf16
-      // the P V product takes at half the exp2-unit cost
+      // P = 2^(S*scale*log2e - max), written over S, and its sum, two columns
+      // at a time: the scaled logits (packed fp32x2 FMA) are rounded to bf16
+      // and exponentiated with the bf16x2 exp2, which gives P in the bf16 the
+      // P V product takes at half the exp2-unit cost
       const uint64_t sl2x2 = f2(sl2, sl2), nmsx2 = f2(-ms, -ms);
       uint64_t lsum[2] = {0, 0};
-#pragma unroll 1
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t v[32];
-        tc::tmem_ld32(sbase + q4 * 32, v);
-        tc::tmem_ld_wait();
-        if (!full) {
 #pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (q4 * 32 + x > lim) v[x] = __float_as_uint(-INFINITY);
-        }
+      for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t pw[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          const uint64_t z = fma2((uint64_t(v[x + 1]) << 32) | v[x], sl2x2, nmsx2);
+          const uint64_t z = fma2((uint64_t(v[q4][x + 1]) << 32) | v[q4][x], sl2x2, nmsx2);
           const uint32_t pp = ex2_bf16x2(to_bf16x2(z));
           lsum[(x >> 1) & 1] = add2(lsum[(x >> 1) & 1], bf16x2_to_f2(pp));
           pw[x >> 1] = pp;
         }
-        tmem_st16(sbase + q4 * 16, pw);  // P columns 16*q4.. cover S columns already read
+        tmem_st16(sbase + q4 * 16, pw);  // P columns 16*q4.. (S is all in registers)
       }
       const uint64_t lsx = add2(lsum[0], lsum[1]);
       const float l = __uint_as_float(uint32_t(lsx)) + __uint_as_float(uint32_t(lsx >> 32));
@@ -436,19 +442,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       uint8_t* wst = qbuf + qs * kQBytes + quarter * 8192;
       const float inv = 1.f / l;
       const uint64_t invx2 = f2(inv, inv);
-#pragma unroll 1
+      uint32_t o[4][32];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tc::tmem_ld32(sbase + 128 + q4 * 32, o[q4]);
+      tc::tmem_ld_wait();
+#pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t v[32];
-        tc::tmem_ld32(sbase + 128 + q4 * 32, v);
-        tc::tmem_ld_wait();
         uint8_t* half = wst + (q4 >> 1) * 4096 + lane * 128;
 #pragma unroll
         for (int k8 = 0; k8 < 4; ++k8) {
+          const uint32_t* w8 = o[q4] + 8 * k8;
           uint4 u;
-          u.x = to_bf16x2(mul2((uint64_t(v[8 * k8 + 1]) << 32) | v[8 * k8 + 0], invx2));
-          u.y = to_bf16x2(mul2((uint64_t(v[8 * k8 + 3]) << 32) | v[8 * k8 + 2], invx2));
-          u.z = to_bf16x2(mul2((uint64_t(v[8 * k8 + 5]) << 32) | v[8 * k8 + 4], invx2));
-          u.w = to_bf16x2(mul2((uint64_t(v[8 * k8 + 7]) << 32) | v[8 * k8 + 6], invx2));
+          u.x = to_bf16x2(mul2((uint64_t(w8[1]) << 32) | w8[0], invx2));
+          u.y = to_bf16x2(mul2((uint64_t(w8[3]) << 32) | w8[2], invx2));
+          u.z = to_bf16x2(mul2((uint64_t(w8[5]) << 32) | w8[4], invx2));
+          u.w = to_bf16x2(mul2((uint64_t(w8[7]) << 32) | w8[6], invx2));
           const int chunk = (q4 & 1) * 4 + k8;
           *reinterpret_cast<uint4*>(half + ((chunk ^ (lane & 7)) << 4)) = u;
         }
@@ -464,13 +472,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         if (nrows > 0) {
           const CUtensorMap* map = nrows == 32 ? &tmap_o32 : &tmap_o16;
           const int grow = e0 * kGroup + quarter * 32;
+          // partial states are read once, by the combine: first out of L2
+          const uint64_t o_policy = tc::policy_evict_first();
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            asm volatile(
-                "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                    reinterpret_cast<uint64_t>(map)),
-                "r"(64 * h), "r"(grow), "r"(tc::smem_addr(wst + h * 4096))
-                : "memory");
+          for (int h = 0; h < 2; ++h) tc::tma_store_2d_hint(map, wst + h * 4096, 64 * h, grow, o_policy);
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
           asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }

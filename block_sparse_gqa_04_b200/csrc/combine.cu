@@ -10,6 +10,10 @@
 // One thread per (row, head, 8 output elements).  The partial states are in
 // entry order, [entry][head of group][D], so for one slot the threads of a
 // (row, group) read one contiguous run of G*D elements with 16-byte loads.
+// Slots are merged in batches with a running maximum (the same exact merge,
+// rescaled whenever the maximum grows), so that each thread issues the loads
+// of a whole batch before it uses any of them: the kernel is bound by HBM and
+// needs many bytes in flight per SM.
 #include "common.cuh"
 #include "internal.h"
 
@@ -58,6 +62,10 @@ struct Vec8<float> {
   }
 };
 
+// Slots merged per batch: their loads are all issued before any is used, so a
+// thread keeps kBatch 16-byte partial loads in flight.
+constexpr int kBatch = 8;
+
 template <typename PT, typename OT, int D>
 __global__ void __launch_bounds__(256) combine_kernel(Problem P, const int32_t* __restrict__ pos,
                                                       const PT* __restrict__ part_o,
@@ -74,29 +82,51 @@ __global__ void __launch_bounds__(256) combine_kernel(Problem P, const int32_t* 
     const int r = int(rh / P.Hq);
     const int g = h / P.G, hh = h % P.G;
     const int32_t* ps = pos + ((long long)g * P.T + r) * P.K;
-    float M = -INFINITY;
-    for (int s = 0; s < P.K; ++s) {
-      const int e = __ldg(ps + s);
-      if (e >= 0) M = fmaxf(M, __ldg(part_lse + (long long)e * P.G + hh));
-    }
+    // running merge: M = max lse so far, acc and sum scaled by 2^-M
+    float M = -INFINITY, sum = 0.f;
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    float sum = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < P.K; ++s) {
-        const int e = __ldg(ps + s);
-        if (e < 0) continue;
-        const long long prow = (long long)e * P.G + hh;
-        const float w = exp2f(__ldg(part_lse + prow) - M);
-        sum += w;
-        Vec8<PT> v;
-        v.load(part_o + prow * D + ch * 8);
-        float f[8];
-        v.to_f32(f);
+    for (int s0 = 0; s0 < P.K; s0 += kBatch) {
+      int e[kBatch];
+      float l[kBatch];
+      Vec8<PT> v[kBatch];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, f[i], acc[i]);
+      for (int u = 0; u < kBatch; ++u) e[u] = s0 + u < P.K ? __ldg(ps + s0 + u) : -1;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (e[u] >= 0) {
+          const long long prow = (long long)e[u] * P.G + hh;
+          l[u] = __ldg(part_lse + prow);
+          v[u].load(part_o + prow * D + ch * 8);
+        } else {
+          l[u] = -INFINITY;
+        }
       }
+      float bm = l[0];
+#pragma unroll
+      for (int u = 1; u < kBatch; ++u) bm = fmaxf(bm, l[u]);
+      if (bm == -INFINITY) continue;  // no valid slot in this batch
+      if (bm > M) {
+        const float sc = exp2f(M - bm);  // 0 while M is -inf
+        sum *= sc;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] *= sc;
+        M = bm;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (e[u] >= 0) {
+          const float w = exp2f(l[u] - M);
+          sum += w;
+          float f[8];
+          v[u].to_f32(f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, f[i], acc[i]);
+        }
+      }
+    }
+    if (M != -INFINITY) {
       const float inv = 1.f / sum;
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] *= inv;

@@ -6,15 +6,23 @@
 // one shared index-key head).
 //
 // With one query per sequence the work is a stream over k_idx (0.25 KB per key)
-// with a handful of dot products per key, so it is bound by HBM, not by any
-// arithmetic unit.  Persistent CTAs stream contiguous ranges of (sequence,
-// block) items of 32 KB through a ring of shared-memory stages filled by TMA (128-byte swizzle, which
-// also makes each thread's 16-byte reads of its own key row conflict-free).
-// Two teams of four warps take alternate items; in a team, thread k owns key k
-// of the block and forms its dot products with every (row, group) index query
-// (packed fp32x2 FMAs against queries broadcast from shared memory); the
-// block maximum per (row, group) is a warp redux plus a max over the four
-// warps.
+// with a handful of dot products per key, so it is bound by HBM.  The dot
+// products run on the tensor cores so that no SM spends more than a few
+// cycles per key: for each (sequence, block) item one tcgen05 MMA computes
+//     D[128 keys x N] = k_idx_block[128 keys x 128 dims] . Q[N x 128 dims]^T
+// with the block's keys on the TMEM lanes and the sequence's RG = rows x groups
+// index queries (zero-padded to N columns) on the TMEM columns.
+//   * warp 0 streams the k_idx block by TMA (128-byte swizzle) into a ring of
+//     shared-memory stages and writes the sequence's queries next to it in the
+//     same swizzled K-major layout (they stay in registers while the sequence
+//     does not change);
+//   * warp 1 issues the MMAs (A = keys, B = queries, both K-major) into one of
+//     four N-column TMEM accumulators;
+//   * warps 2-5 (one TMEM lane quarter each) read their keys' N scores, mask
+//     the keys a row cannot see, reduce each column with a warp redux over
+//     orderable keys and combine the four warps' maxima through shared memory.
+// Persistent CTAs take contiguous ranges of items, so consecutive items mostly
+// share one sequence.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -26,166 +34,236 @@
 namespace msa {
 namespace {
 
-constexpr int kStages = 5;
-constexpr int kBlkBytes = 128 * 128 * 2;   // one block of k_idx
-constexpr int kHalfBytes = kBlkBytes / 2;
-constexpr int kTeamThreads = 128;
-constexpr int kThreads = 2 * kTeamThreads + 32;  // two teams + a producer warp
-constexpr int kMaxRG = 16;                 // (rows per sequence) x groups handled
+constexpr int kKBytes = 128 * 128 * 2;  // one block of k_idx
+constexpr int kKHalf = kKBytes / 2;     // 64 dims (128 B) x 128 keys
+constexpr int kThreads = 192;
+constexpr int kSlots = 4;               // TMEM accumulators
+constexpr int kMaxRG = 32;              // (rows per sequence) x groups handled
 
+template <int N>
+struct Cfg {
+  static constexpr int kStages = N <= 16 ? 6 : 5;
+  static constexpr int kQHalf = N * 128;                 // 64 dims x N padded queries
+  static constexpr int kStageBytes = kKBytes + 2 * kQHalf;
+  static constexpr uint32_t kTmemCols = kSlots * N < 32 ? 32 : kSlots * N;
+  static constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, N, 0, 0);
+  static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+};
+
+template <int N>
 struct Shared {
-  uint64_t full[kStages], empty[kStages];
-  float q[2][kMaxRG][128];                 // per team: index queries of its sequence, fp32
-  uint32_t red[2][4][kMaxRG];              // per team: warp maxima (orderable keys)
+  uint64_t full[Cfg<N>::kStages], empty[Cfg<N>::kStages];
+  uint64_t acc_full[kSlots], acc_empty[kSlots];
+  uint32_t red[kSlots][4][N];   // per accumulator: the four warps' column maxima
+  int qseq[Cfg<N>::kStages];    // sequence whose queries each stage holds (-1: none)
+  uint32_t tmem_base;
   int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 + kStages * kBlkBytes + sizeof(Shared) + 64;
-static_assert(kSmemBytes <= 232448, "more dynamic shared memory than a B200 CTA can have");
-
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
+template <int N>
+constexpr size_t smem_bytes() {
+  return 1024 + Cfg<N>::kStages * Cfg<N>::kStageBytes + sizeof(Shared<N>) + 64;
 }
+static_assert(smem_bytes<16>() <= 232448, "more dynamic shared memory than a B200 CTA can have");
+static_assert(smem_bytes<32>() <= 232448, "more dynamic shared memory than a B200 CTA can have");
 
-__device__ __forceinline__ void team_sync(int team) {
-  asm volatile("bar.sync %0, %1;" ::"r"(team + 1), "r"(kTeamThreads) : "memory");
-}
-
-// Team barrier that also returns whether any thread of the team passed `v`.
-__device__ __forceinline__ bool team_any(int team, bool v) {
+// Barrier of the four epilogue warps that also returns whether any of their
+// threads passed `v` (so that they leave together on a failed wait).
+__device__ __forceinline__ bool epi_any(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "barrier.red.or.pred q, 1, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(uint32_t(v)), "r"(team + 1), "r"(kTeamThreads)
+      : "r"(uint32_t(v))
       : "memory");
   return r != 0;
 }
 
-// RG = (query rows per sequence) x groups, fixed at compile time so that only
-// the live dot products are formed.
-template <int RG>
+template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
 index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
                     const __nv_bfloat16* __restrict__ q_idx, float* __restrict__ bmax,
                     int* __restrict__ status, int nvis) {
+  using C = Cfg<N>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  Shared* sh = reinterpret_cast<Shared*>(smem + kStages * kBlkBytes);
+  Shared<N>* sh = reinterpret_cast<Shared<N>*>(smem + S * C::kStageBytes);
   volatile int* abort = &sh->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int RG = P.Sq * P.Hkv;
+
+  // zero the padded query rows RG..N-1 of every stage once; only rows < RG are
+  // rewritten later
+  for (int e = threadIdx.x; e < S * 2 * (N - RG) * 8; e += kThreads) {
+    const int st = e / (2 * (N - RG) * 8), rem = e % (2 * (N - RG) * 8);
+    const int h = rem / ((N - RG) * 8), x = rem % ((N - RG) * 8);
+    *reinterpret_cast<uint4*>(stages + st * C::kStageBytes + kKBytes + h * C::kQHalf +
+                              RG * 128 + x * 16) = make_uint4(0, 0, 0, 0);
+  }
+  tc::fence_async_smem();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&sh->full[s], 1);
-      tc::mbar_init(&sh->empty[s], 4);  // the four warps of the team that used it
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(&sh->full[s], 2);   // TMA bytes + the queries written by warp 0
+      tc::mbar_init(&sh->empty[s], 1);
+      sh->qseq[s] = -1;
+    }
+    for (int s = 0; s < kSlots; ++s) {
+      tc::mbar_init(&sh->acc_full[s], 1);
+      tc::mbar_init(&sh->acc_empty[s], 4);
     }
     sh->abort = 0;
     tc::fence_mbar_init();
   }
+  if (warp == 0 && lane == 0) tc::tma_prefetch(&tmap_k);
+  if (warp == 1) tc::tmem_alloc(&sh->tmem_base, C::kTmemCols);
+  tc::tc_fence_before();
   __syncthreads();
-  // each CTA streams a contiguous range of (sequence, block) items, so it stays
-  // on one sequence's index queries and reads consecutive blocks
+  tc::tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
   const long long items = (long long)P.B * nvis;
   const long long i0 = items * blockIdx.x / gridDim.x;
   const long long i1 = items * (blockIdx.x + 1) / gridDim.x;
   bool failed = false;
-  if (warp == 8) {
-    // ---------------- producer ----------------
+
+  if (warp == 0) {
+    // ---------------- producer: k_idx by TMA, queries from registers ----------------
+    constexpr int kQv = N / 2;          // 16-byte query chunks per lane (RG * 16 / 32 at most)
+    uint4 qv[kQv];
+    int qb = -1;
+    int k = 0;
+    for (long long it = i0; it < i1; ++it, ++k) {
+      const int s = k % S;
+      const uint32_t ph = (k / S) & 1;
+      const int b = int(it / nvis), c = int(it % nvis);
+      if (b != qb) {
+        const uint4* src = reinterpret_cast<const uint4*>(q_idx + (long long)b * RG * 128);
+#pragma unroll
+        for (int x = 0; x < kQv; ++x) {
+          const int e = lane + 32 * x;
+          qv[x] = e < RG * 16 ? __ldg(src + e) : make_uint4(0, 0, 0, 0);
+        }
+        qb = b;
+      }
+      bool ok = true;
+      if (lane == 0) ok = tc::mbar_wait(&sh->empty[s], ph ^ 1, abort);
+      if (!__shfl_sync(MSA_FULL_MASK, ok, 0)) { failed = true; break; }
+      uint8_t* st = stages + s * C::kStageBytes;
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&sh->full[s], kKBytes);
+        const int row = b * P.Skv + c * 128;
+        tc::tma_load_2d(st, &tmap_k, &sh->full[s], 0, row);
+        tc::tma_load_2d(st + kKHalf, &tmap_k, &sh->full[s], 64, row);
+      }
+      // query chunk e = (row n, 16-byte chunk j of its 256 B): K-major, 128-byte
+      // swizzle, the layout TMA gives the key block.  A stage that already
+      // holds this sequence's queries keeps them.
+      const bool put_q = sh->qseq[s] != b;
+      if (put_q) {
+#pragma unroll
+        for (int x = 0; x < kQv; ++x) {
+          const int e = lane + 32 * x;
+          if (e < RG * 16) {
+            const int n = e >> 4, j = e & 15;
+            *reinterpret_cast<uint4*>(st + kKBytes + (j >> 3) * C::kQHalf + n * 128 +
+                                      (((j & 7) ^ (n & 7)) << 4)) = qv[x];
+          }
+        }
+        tc::fence_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) {
+        if (put_q) sh->qseq[s] = b;
+        tc::mbar_arrive(&sh->full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      tc::tma_prefetch(&tmap_k);
       int k = 0;
       for (long long it = i0; it < i1; ++it, ++k) {
-        const int s = k % kStages;
-        if (!tc::mbar_wait(&sh->empty[s], ((k / kStages) & 1) ^ 1, abort)) { failed = true; break; }
-        const int b = int(it / nvis), c = int(it % nvis);
-        tc::mbar_arrive_expect_tx(&sh->full[s], kBlkBytes);
-        const int row = b * P.Skv + c * 128;
-        tc::tma_load_2d(stages + s * kBlkBytes, &tmap_k, &sh->full[s], 0, row);
-        tc::tma_load_2d(stages + s * kBlkBytes + kHalfBytes, &tmap_k, &sh->full[s], 64, row);
+        const int s = k % S, slot = k % kSlots;
+        if (!tc::mbar_wait(&sh->full[s], (k / S) & 1, abort)) { failed = true; break; }
+        if (!tc::mbar_wait(&sh->acc_empty[slot], ((k / kSlots) & 1) ^ 1, abort)) {
+          failed = true;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t kb = tc::smem_addr(stages + s * C::kStageBytes);
+        const uint32_t qbase = kb + kKBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ad = tc::sdesc_sw128(kb + (kk >> 2) * kKHalf + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              tc::sdesc_sw128(qbase + (kk >> 2) * C::kQHalf + (kk & 3) * 32, 16, 1024);
+          tc::mma_ss(tmem + slot * N, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&sh->acc_full[slot]);
+        tc::mma_commit(&sh->empty[s]);
       }
     }
   } else {
-    // ---------------- teams ----------------
-    const int team = warp >> 2, kw = warp & 3;
-    const int key = kw * 32 + lane;          // key of the block this thread owns
-    int qb = -1;                             // sequence whose queries sit in sh->q[team]
-    int k = team;
-    for (long long it = i0 + team; it < i1; it += 2, k += 2) {
-      const int s = k % kStages;
+    // ---------------- epilogue: masked column maxima ----------------
+    const int quarter = warp & 3;            // TMEM lanes this warp may touch
+    const int key = quarter * 32 + lane;     // key of the block on this thread's lane
+    const int et = threadIdx.x - 64;         // 0..127 over the epilogue warps
+    int k = 0;
+    for (long long it = i0; it < i1; ++it, ++k) {
+      const int slot = k % kSlots;
       const int b = int(it / nvis), c = int(it % nvis);
-      if (b != qb) {
-        team_sync(team);
-        for (int e = threadIdx.x - team * kTeamThreads; e < RG * 128; e += kTeamThreads)
-          sh->q[team][e >> 7][e & 127] =
-              __bfloat162float(q_idx[(long long)b * RG * 128 + e]);
-        team_sync(team);
-        qb = b;
-      }
-      // the whole team gives up together, so no warp is left at a team barrier
-      if (team_any(team, !tc::mbar_wait(&sh->full[s], (k / kStages) & 1, abort))) {
-        failed = true;
-        break;
-      }
-      const uint8_t* kr = stages + s * kBlkBytes + key * 128;
-      uint64_t acc[RG];
+      bool ok = true;
+      if (lane == 0) ok = tc::mbar_wait(&sh->acc_full[slot], (k / kSlots) & 1, abort);
+      ok = __shfl_sync(MSA_FULL_MASK, ok, 0);
+      if (ok) {
+        tc::tc_fence_after();
+        uint32_t v[N];
 #pragma unroll
-      for (int x = 0; x < RG; ++x) acc[x] = 0;
-#pragma unroll 4
-      for (int j = 0; j < 16; ++j) {
-        // 16-byte chunk j of this key: half j / 8, swizzled position (j % 8) ^ (key % 8)
-        const uint4 u = *reinterpret_cast<const uint4*>(kr + (j >> 3) * kHalfBytes +
-                                                        (((j & 7) ^ (key & 7)) << 4));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-        uint64_t kp[4];
+        for (int h = 0; h < N / 16; ++h)
+          tc::tmem_ld16(tmem + (uint32_t(quarter * 32) << 16) + slot * N + h * 16, v + h * 16);
+        tc::tmem_ld_wait();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sh->acc_empty[slot]);
+        const long long j = (long long)c * 128 + key;  // key position in the sequence
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
-          kp[x] = (uint64_t(w[x] & 0xffff0000u) << 32) | uint64_t(w[x] << 16);
-#pragma unroll
-        for (int x = 0; x < RG; ++x) {
-          const uint4* qp = reinterpret_cast<const uint4*>(&sh->q[team][x][8 * j]);
-          const uint4 q0 = qp[0], q1 = qp[1];
-          acc[x] = fma2(kp[0], (uint64_t(q0.y) << 32) | q0.x, acc[x]);
-          acc[x] = fma2(kp[1], (uint64_t(q0.w) << 32) | q0.z, acc[x]);
-          acc[x] = fma2(kp[2], (uint64_t(q1.y) << 32) | q1.x, acc[x]);
-          acc[x] = fma2(kp[3], (uint64_t(q1.w) << 32) | q1.z, acc[x]);
+        for (int n = 0; n < N; ++n) {
+          if (n < RG) {
+            const bool vis = j <= P.q_pos0 + n / P.Hkv;
+            const uint32_t m =
+                __reduce_max_sync(MSA_FULL_MASK, vis ? orderable(__uint_as_float(v[n])) : 0u);
+            if (lane == 0) sh->red[slot][quarter][n] = m;
+          }
         }
       }
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sh->empty[s]);  // this warp is done with the stage
-      const long long j = (long long)c * 128 + key;    // key position in the sequence
-#pragma unroll
-      for (int x = 0; x < RG; ++x) {
-        const int i = x / P.Hkv;
-        const bool vis = j < P.Skv && j <= P.q_pos0 + i;
-        const float sc = __uint_as_float(uint32_t(acc[x])) + __uint_as_float(uint32_t(acc[x] >> 32));
-        const uint32_t m = __reduce_max_sync(MSA_FULL_MASK, vis ? orderable(sc) : 0u);
-        if (lane == 0) sh->red[team][kw][x] = m;
-      }
-      team_sync(team);
-      const int t = threadIdx.x - team * kTeamThreads;
-      if (t < RG) {
-        const uint32_t m = max(max(sh->red[team][0][t], sh->red[team][1][t]),
-                               max(sh->red[team][2][t], sh->red[team][3][t]));
-        const int i = t / P.Hkv, g = t % P.Hkv;
+      // publishes red[slot]; every epilogue thread leaves together on a failure
+      if (epi_any(!ok)) { failed = true; break; }
+      if (et < RG) {
+        const uint32_t m = max(max(sh->red[slot][0][et], sh->red[slot][1][et]),
+                               max(sh->red[slot][2][et], sh->red[slot][3][et]));
+        const int i = et / P.Hkv, g = et % P.Hkv;
         // back from the orderable key; 0 means no visible key in the block
-        const float v = m == 0u ? -INFINITY
-                                : __uint_as_float((m & 0x80000000u) ? (m & 0x7fffffffu) : ~m);
+        const float val = m == 0u ? -INFINITY
+                                  : __uint_as_float((m & 0x80000000u) ? (m & 0x7fffffffu) : ~m);
         if ((long long)c * 128 <= P.q_pos0 + i)
-          bmax[((long long)g * P.T + (long long)b * P.Sq + i) * P.nblk + c] = v;
+          bmax[((long long)g * P.T + (long long)b * P.Sq + i) * P.nblk + c] = val;
       }
-      team_sync(team);  // red[] is reused by the next item
     }
   }
   if (failed) {
     sh->abort = 1;
     atomicOr(status, tc::kStatusWaitTimeout);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -215,19 +293,27 @@ int sm_count() {
 
 }  // namespace
 
-// (rows per sequence) x groups: the widths the kernel is instantiated for
-static int rg_width(const Problem& P) {
+bool index_decode_supported(const Problem& P) {
   const int rg = P.Sq * P.Hkv;
-  return (rg == 4 || rg == 8 || rg == 16) ? rg : 0;
+  return !P.f32 && P.DI == 128 && P.Bk == 128 && P.Sq <= 8 && rg >= 1 && rg <= kMaxRG &&
+         (long long)P.B * P.Skv < (1LL << 31);
 }
 
-bool index_decode_supported(const Problem& P) {
-  return !P.f32 && P.DI == 128 && P.Bk == 128 && P.Sq <= 8 && rg_width(P) != 0 &&
-         (long long)P.B * P.Skv < (1LL << 31);
+template <int N>
+static cudaError_t launch_n(const CUtensorMap& map, const Problem& P, const void* q_idx,
+                            float* bmax, int32_t* status, int nvis, int grid, cudaStream_t s) {
+  constexpr size_t smem = smem_bytes<N>();
+  cudaError_t e = cudaFuncSetAttribute(index_decode_kernel<N>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  index_decode_kernel<N><<<grid, kThreads, smem, s>>>(
+      map, P, static_cast<const __nv_bfloat16*>(q_idx), bmax, status, nvis);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_index_decode(const Problem& P, const void* q_idx, const void* k_idx,
                                 float* bmax, int32_t* status, cudaStream_t s) {
+  if (!index_decode_supported(P)) return cudaErrorNotSupported;
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap map;
@@ -241,20 +327,10 @@ cudaError_t launch_index_decode(const Problem& P, const void* q_idx, const void*
     return cudaErrorInvalidValue;
   const int nvis = int((P.q_pos0 + P.Sq - 1) / P.Bk) + 1;
   const long long items = (long long)P.B * nvis;
-  const int grid = int(std::min<long long>(sm_count(), (items + 1) / 2));
-  auto kern = index_decode_kernel<4>;
-  switch (P.Sq * P.Hkv) {
-    case 4: kern = index_decode_kernel<4>; break;
-    case 8: kern = index_decode_kernel<8>; break;
-    case 16: kern = index_decode_kernel<16>; break;
-    default: return cudaErrorNotSupported;
-  }
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(kSmemBytes));
-  if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemBytes, s>>>(map, P, static_cast<const __nv_bfloat16*>(q_idx), bmax,
-                                          status, nvis);
-  return cudaGetLastError();
+  const int grid = int(std::min<long long>(sm_count(), items));
+  const int rg = P.Sq * P.Hkv;
+  return rg <= 16 ? launch_n<16>(map, P, q_idx, bmax, status, nvis, grid, s)
+                  : launch_n<32>(map, P, q_idx, bmax, status, nvis, grid, s);
 }
 
 }  // namespace msa

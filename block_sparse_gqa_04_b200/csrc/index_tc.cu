@@ -19,8 +19,10 @@
 //   * two 128-column fp32 accumulators alternate, so the epilogue of one unit
 //     overlaps the MMAs of the next.
 // Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
-// 2-5 load index queries into TMEM and run the epilogue (one query row per
+// 2-9 load index queries into TMEM and run the epilogue (one query row per
 // thread: masked max over the row's 128 columns, one fp32 store per unit).
+// The epilogue is two warpgroups, one per accumulator, so that two units drain
+// at once while the tensor cores fill the next.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -35,7 +37,7 @@ namespace {
 constexpr int kStages = 4;
 constexpr int kStageBytes = 128 * 128 * 2;  // one k_idx block, bf16
 constexpr int kHalfBytes = kStageBytes / 2; // 64 dims (128 B) x 128 keys
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;               // TMA, MMA, two epilogue warpgroups
 constexpr int kMaxGroups = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 256;           // accumulators follow the A region
@@ -119,7 +121,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       tc::mbar_init(&bars->acc_full[s], 1);
       tc::mbar_init(&bars->acc_empty[s], 4);
     }
-    tc::mbar_init(&bars->a_full, 4);
+    tc::mbar_init(&bars->a_full, 8);
     tc::mbar_init(&bars->a_empty, 1);
     bars->abort = 0;
     tc::fence_mbar_init();
@@ -196,15 +198,16 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       }
     }
   } else {
-    // ---------------- index-query loader + epilogue ----------------
+    // ---------------- index-query loader + epilogue (two warpgroups) ----------------
+    const int ewg = (warp - 2) >> 2;        // accumulator slot this warpgroup drains
     const int quarter = warp & 3;           // TMEM lanes this warp may touch
     const int row = quarter * 32 + lane;    // query row inside the tile
     const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
     if (L0 < L1) {
       Walk w;
       w.start(P, L0, per_seq);
-      int slot = 0;
-      uint32_t acc_phase = 0, ae_phase = 0;
+      uint32_t ae_phase = 0;
+      int k = 0;                            // unit counter, the same on every warp
       bool seg_start = true, first = true;
       for (long long L = L0; L < L1 && !failed; ++L) {
         const int i = w.m * 128 + row;      // query index inside the sequence
@@ -220,8 +223,9 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
             tc::tc_fence_after();
           }
           first = false;
+          // each warpgroup writes the index queries of every other group
           const uint4* src = reinterpret_cast<const uint4*>(q_idx + r * P.Hkv * 128);
-          for (int g = 0; g < P.Hkv; ++g) {
+          for (int g = ewg; g < P.Hkv; g += 2) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               uint32_t v[32];
@@ -243,8 +247,10 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
         }
         const long long t = P.q_pos0 + i;
         const long long lim = t - (long long)w.c * P.Bk;  // last visible column
-        for (int g = 0; g < P.Hkv; ++g) {
-          if (!__all_sync(MSA_FULL_MASK, tc::mbar_wait(&bars->acc_full[slot], acc_phase, abort))) {
+        for (int g = 0; g < P.Hkv; ++g, ++k) {
+          if ((k & 1) != ewg) continue;     // the other warpgroup's unit
+          const uint32_t par = (k >> 1) & 1;
+          if (!__all_sync(MSA_FULL_MASK, tc::mbar_wait(&bars->acc_full[ewg], par, abort))) {
             failed = true;
             break;
           }
@@ -254,8 +260,11 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
           uint32_t v[4][32];
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            tc::tmem_ld32(tmem + lane_addr + kAccCol + slot * 128 + j * 32, v[j]);
+            tc::tmem_ld32(tmem + lane_addr + kAccCol + ewg * 128 + j * 32, v[j]);
           tc::tmem_ld_wait();
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&bars->acc_empty[ewg]);
           float mx[8];
 #pragma unroll
           for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
@@ -270,12 +279,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
           }
           const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&bars->acc_empty[slot]);
           if (valid) bmax[((long long)g * P.T + r) * P.nblk + w.c] = m;
-          slot ^= 1;
-          if (slot == 0) acc_phase ^= 1;
         }
         seg_start = w.next(P);
       }

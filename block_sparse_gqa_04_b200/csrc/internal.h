@@ -90,6 +90,11 @@ cudaError_t launch_invert(const Problem& P, const int32_t* q2k, const Lists& L,
                           int32_t* status, cudaStream_t s);
 // Fills L.tiles from the list offsets (one record per tile).
 cudaError_t launch_tile_records(const Problem& P, const Lists& L, cudaStream_t s);
+// One query row per sequence with the tensor-core attention kernel: entries,
+// positions and tile records in one launch (every list has at most one entry).
+bool lists_direct(const Problem& P);
+cudaError_t launch_lists_direct(const Problem& P, const int32_t* q2k, const Lists& L,
+                                int32_t* status, cudaStream_t s);
 
 // --- main branch ------------------------------------------------------------
 cudaError_t launch_attn_simt(const Problem& P, const void* q, const void* k, const void* v,

@@ -186,6 +186,93 @@ __global__ void tile_records_kernel(Problem P, Lists L) {
   }
 }
 
+// One query row per sequence (decode): every list holds at most one entry, so
+// the counting sort degenerates.  One CTA walks the entries in order, keeps
+// the valid ones (a block-wide prefix count gives each its position), and
+// writes the entry, its position and a one-query tile record directly.  Only
+// the tile count at tile_off[nlists] is written of the offsets: the
+// tensor-core attention kernel and the combine read nothing else.
+constexpr int kDirectThreads = 1024;
+constexpr long long kDirectMaxEntries = 1 << 16;
+
+__global__ void __launch_bounds__(kDirectThreads) direct_lists_kernel(Problem P,
+                                                                      const int32_t* __restrict__ q2k,
+                                                                      Lists L, int32_t* status) {
+  __shared__ int wsum[kDirectThreads / 32];
+  __shared__ int run;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const long long n = (long long)P.Hkv * P.T * P.K;
+  if (threadIdx.x == 0) run = 0;
+  __syncthreads();
+  for (long long base = 0; base < n; base += kDirectThreads) {
+    const long long e = base + threadIdx.x;
+    int g = 0, r = 0, slot = 0, c = -1, st = 0;
+    if (e < n) {
+      g = int(e / ((long long)P.T * P.K));
+      r = int((e / P.K) % P.T);
+      slot = int(e % P.K);
+      c = q2k[e];
+      st = entry_state(P, r, c);
+      if (st < 0) atomicOr(status, kStatusBadEntry);
+    }
+    const int valid = st > 0 ? 1 : 0;
+    int incl = valid;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(MSA_FULL_MASK, incl, o);
+      if (lane >= o) incl += x;
+    }
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      int x = wsum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(MSA_FULL_MASK, x, o);
+        if (lane >= o) x += y;
+      }
+      wsum[lane] = x;  // inclusive sums over warps
+    }
+    __syncthreads();
+    const int p = run + (w > 0 ? wsum[w - 1] : 0) + incl - valid;
+    if (e < n) {
+      if (valid) {
+        L.entries[p] = (r << 5) | slot;
+        L.pos[e] = p;
+        TileRec rec;
+        rec.c = c;
+        rec.g = g;
+        rec.b = r / P.Sq;
+        rec.e0 = p;
+        rec.n = 1;
+        rec.tend = p + 1;
+        rec.lid = p;
+        rec.pad = 0;
+        rec.rows[0] = r;
+#pragma unroll
+        for (int x = 1; x < 8; ++x) rec.rows[x] = 0;
+        reinterpret_cast<TileRec*>(L.tiles)[p] = rec;
+      } else {
+        L.pos[e] = -1;
+      }
+    }
+    __syncthreads();  // everyone has read run and wsum
+    if (threadIdx.x == 0) run += wsum[kDirectThreads / 32 - 1];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) L.tile_off[P.nlists] = run;
+}
+
+bool lists_direct(const Problem& P) {
+  return P.Sq == 1 && attn_tc_supported(P) && (long long)P.Hkv * P.T * P.K <= kDirectMaxEntries;
+}
+
+cudaError_t launch_lists_direct(const Problem& P, const int32_t* q2k, const Lists& L,
+                                int32_t* status, cudaStream_t s) {
+  direct_lists_kernel<<<1, kDirectThreads, 0, s>>>(P, q2k, L, status);
+  return cudaGetLastError();
+}
+
 static unsigned grid_for(long long n, int threads) {
   long long b = (n + threads - 1) / threads;
   if (b > 148LL * 64) b = 148LL * 64;

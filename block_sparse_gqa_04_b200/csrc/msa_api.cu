@@ -146,8 +146,13 @@ msa_status_t run_attend(const Problem& P, const void* q, const void* k, const vo
                    at<int32_t>(ws, L.tiles), at<int32_t>(ws, L.seg_sums)};
   msa::Partials part{at<void>(ws, L.part_o), at<float>(ws, L.part_lse)};
   const bool tc = msa::attn_tc_supported(P);
-  cudaError_t e = msa::launch_invert(P, q2k, lists, at<int32_t>(ws, L.status), s);
-  if (e == cudaSuccess && tc) e = msa::launch_tile_records(P, lists, s);
+  cudaError_t e;
+  if (msa::lists_direct(P)) {
+    e = msa::launch_lists_direct(P, q2k, lists, at<int32_t>(ws, L.status), s);
+  } else {
+    e = msa::launch_invert(P, q2k, lists, at<int32_t>(ws, L.status), s);
+    if (e == cudaSuccess && tc) e = msa::launch_tile_records(P, lists, s);
+  }
   stage_mark(s);
   if (e == cudaSuccess) {
     e = tc ? msa::launch_attn_tc(P, q, k, v, lists, part, at<int32_t>(ws, L.status), s)
@@ -260,7 +265,9 @@ int32_t msa_launch_count(const msa_problem_t* p, int32_t op) {
   if (resolve(p, &P) != MSA_OK || P.T == 0) return 0;
   const int sel = 2;                               // index + top-k
   // lists (+ tile records on the tensor-core path) + attention + combine
-  const int att = msa::kLaunchesInvert + (msa::attn_tc_supported(P) ? 1 : 0) + 2;
+  const int att = (msa::lists_direct(P) ? 1
+                                         : msa::kLaunchesInvert + (msa::attn_tc_supported(P) ? 1 : 0)) +
+                  2;
   switch (op) {
     case MSA_OP_SELECT: return sel;
     case MSA_OP_ATTEND: return att;

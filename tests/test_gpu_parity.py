@@ -26,6 +26,11 @@ SMALL = {
     "chunk_unaligned": Workload("chunk_unaligned", 1, 300, 2000, 1700, 64, 4, 128, 128, 128, 16,
                                 "bf16", 2),
     "decode_small": Workload("decode_small", 5, 1, 3000, 2999, 64, 4, 128, 128, 128, 16, "bf16", 3),
+    # a few query rows per sequence (the decode index kernel's 16- and 32-wide
+    # query tiles; rows of one sequence straddle a block boundary)
+    "decode_rows4": Workload("decode_rows4", 3, 4, 3000, 2942, 32, 4, 128, 128, 128, 8, "bf16", 2),
+    "decode_rows8": Workload("decode_rows8", 2, 8, 5000, 4990, 64, 4, 128, 128, 128, 16, "bf16", 2),
+    "decode_g2": Workload("decode_g2", 4, 1, 1500, 1499, 16, 2, 128, 128, 128, 4, "bf16", 1),
     "top1": Workload("top1", 1, 700, 700, 0, 32, 2, 128, 128, 128, 1, "bf16", 1),
     "d64_g4": Workload("d64_g4", 2, 700, 700, 0, 16, 4, 64, 64, 128, 5, "bf16", 1),
     "f32_d128_g8": Workload("f32_d128_g8", 1, 600, 600, 0, 16, 2, 128, 128, 128, 4, "f32", 0),
@@ -127,14 +132,16 @@ def test_select_block_scores(name):
                     w.top_k)
 
 
-def test_attend_flags_invalid_entries_and_skips_them():
-    w = SMALL["batch_offset"]
+@pytest.mark.parametrize("name", ["batch_offset", "decode_small"])
+def test_attend_flags_invalid_entries_and_skips_them(name):
+    w = SMALL[name]
     cpu, gpu = _inputs(w)
     oq2k = O.select(cpu["q_idx"], cpu["k_idx"], w.q_pos0, w.block_size, w.top_k)
     bad = oq2k.copy()
+    r1, r2 = min(5, w.rows - 1), min(7, w.rows - 2)
     # a block after the local one (not visible) and an id below -1
-    bad[0, 5, -1] = (w.q_pos0 + 5) // w.block_size + 1
-    bad[1, 7, 0] = -5
+    bad[0, r1, -1] = (w.q_pos0 + r1 % w.q_len) // w.block_size + 1
+    bad[1, r2, 0] = -5
     q2k = torch.from_numpy(bad.astype(np.int32)).cuda()
     with pytest.raises(msa.MsaError) as ei:
         msa.attend(gpu["q"], gpu["k"], gpu["v"], q2k, q_pos0=w.q_pos0, block_size=w.block_size,
@@ -142,8 +149,8 @@ def test_attend_flags_invalid_entries_and_skips_them():
     assert ei.value.code == 5
     out = msa.attend(gpu["q"], gpu["k"], gpu["v"], q2k, q_pos0=w.q_pos0, block_size=w.block_size)
     skip = bad.copy()
-    skip[0, 5, -1] = -1
-    skip[1, 7, 0] = -1
+    skip[0, r1, -1] = -1
+    skip[1, r2, 0] = -1
     oo, _ = O.attend(cpu["q"], cpu["k"], cpu["v"], skip, w.q_pos0, w.block_size)
     assert_close_out(to_np(out), oo, w.dtype)
 
