@@ -421,6 +421,13 @@ def weak_value(rows_per_rank: int, ms_local: float, world: int) -> tuple:
     return world * rows_per_rank / (ms * 1e-3), ms
 
 
+def workload_config(w: Workload, world: int) -> dict:
+    return {"workload": w.name, "batch": w.batch, "q_len": w.q_len, "kv_len": w.kv_len,
+            "q_pos0": w.q_pos0, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "index_dim": w.index_dim, "block_size": w.block_size,
+            "top_k": w.top_k, "parallelism": f"replicas x{world} (independent problems)"}
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -476,8 +483,7 @@ def main():
                 "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic",
-                "config": {"workload": w.name, "batch": w.batch, "q_len": w.q_len,
-                           "kv_len": w.kv_len, "q_pos0": w.q_pos0, "top_k": w.top_k},
+                "config": workload_config(w, world),
                 "cpu_baseline": cb,
                 "e2e": {"value": v, "unit": "query-tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0},
@@ -499,14 +505,9 @@ def main():
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1/d) inputs with planted needle blocks)",
-        "config": {"workload": w.name, "batch": w.batch, "q_len": w.q_len, "kv_len": w.kv_len,
-                   "q_pos0": w.q_pos0, "num_q_heads": w.num_q_heads,
-                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
-                   "index_dim": w.index_dim, "block_size": w.block_size, "top_k": w.top_k,
-                   "parallelism": f"replicas x{world} (independent problems)",
-                   "kernel_path": main_res["path"],
-                   "l2": "inputs larger than L2 (q alone is %.2f GB per step)" %
-                         (main_res["x"]["q"].numel() * 2 / 1e9)},
+        "config": dict(workload_config(w, world), kernel_path=main_res["path"],
+                       l2="inputs larger than L2 (q alone is %.2f GB per step)" %
+                          (main_res["x"]["q"].numel() * 2 / 1e9)),
         "clocks": main_res["clocks"],
         "gpu_launches": main_res["launches"],
         "stage_ms": {k: round(v, 4) for k, v in main_res["stage"].items()},

@@ -21,8 +21,8 @@
 //   * warps 2-5 (one TMEM lane quarter each) read their keys' N scores, mask
 //     the keys a row cannot see, reduce each column with a warp redux over
 //     orderable keys and combine the four warps' maxima through shared memory.
-// Persistent CTAs take contiguous ranges of items, so consecutive items mostly
-// share one sequence.
+// Persistent CTAs (two per SM for the 16-wide form) take contiguous ranges of
+// items, so consecutive items mostly share one sequence.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -42,7 +42,10 @@ constexpr int kMaxRG = 32;              // (rows per sequence) x groups handled
 
 template <int N>
 struct Cfg {
-  static constexpr int kStages = N <= 16 ? 6 : 5;
+  // 16-wide tiles: two CTAs of three stages per SM (two TMA streams per SM
+  // move more bytes than one); 32-wide tiles need more shared memory per stage
+  static constexpr int kStages = N <= 16 ? 3 : 5;
+  static constexpr int kCtasPerSm = N <= 16 ? 2 : 1;
   static constexpr int kQHalf = N * 128;                 // 64 dims x N padded queries
   static constexpr int kStageBytes = kKBytes + 2 * kQHalf;
   static constexpr uint32_t kTmemCols = kSlots * N < 32 ? 32 : kSlots * N;
@@ -83,7 +86,7 @@ __device__ __forceinline__ bool epi_any(bool v) {
 }
 
 template <int N>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
                     const __nv_bfloat16* __restrict__ q_idx, float* __restrict__ bmax,
                     int* __restrict__ status, int nvis) {
@@ -327,8 +330,9 @@ cudaError_t launch_index_decode(const Problem& P, const void* q_idx, const void*
     return cudaErrorInvalidValue;
   const int nvis = int((P.q_pos0 + P.Sq - 1) / P.Bk) + 1;
   const long long items = (long long)P.B * nvis;
-  const int grid = int(std::min<long long>(sm_count(), items));
   const int rg = P.Sq * P.Hkv;
+  const int per_sm = rg <= 16 ? Cfg<16>::kCtasPerSm : Cfg<32>::kCtasPerSm;
+  const int grid = int(std::min<long long>((long long)sm_count() * per_sm, items));
   return rg <= 16 ? launch_n<16>(map, P, q_idx, bmax, status, nvis, grid, s)
                   : launch_n<32>(map, P, q_idx, bmax, status, nvis, grid, s);
 }
