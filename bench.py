@@ -299,6 +299,8 @@ def run_e2e(msa, w, xh, out_h, steps, warmup):
 # the entry no longer applies and the bench reports traffic as null.
 NCU_TRAFFIC = {
     # stage: (workload, source file, git blob id, bytes per launch)
+    "attn": ("prefill_128k", "block_sparse_gqa_04_b200/csrc/attn_tc.cu",
+             "0de5df29cbd87c2c6db149d53ee96dba5c7fd1a8", 12784880128 + 34592174592),
 }
 
 
