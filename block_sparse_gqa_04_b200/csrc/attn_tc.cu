@@ -11,8 +11,10 @@
 // One persistent CTA per SM takes a contiguous share of the tiles.  Per tile:
 //   * TMA loads the block's K and V (128 keys x 128 dims each, 128-byte swizzle)
 //     into one of two buffers, once per list, and gathers the 8 queries' Q rows
-//     (16 heads x 128 dims, contiguous in memory) with two boxes per query,
-//     issued by sixteen lanes at once;
+//     (16 heads x 128 dims, 4 KB contiguous in memory) with one box per query
+//     through a 4D view of Q that lands the two 8-row groups with their two
+//     64-dim halves side by side (8-row groups 2 KB apart in the operand),
+//     issued by eight lanes at once;
 //   * S = Q K^T (both K-major in shared memory) lands in TMEM, one row per lane;
 //   * the softmax warps read their row, apply the scale and the causal cut of
 //     the local block, and write P (bf16) back over S in TMEM;
@@ -263,15 +265,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
           good = good && tc::mbar_wait(&bars->q_empty[q_stage], q_phase ^ 1, abort);
           if (good) tc::mbar_arrive_expect_tx(&bars->q_full[q_stage], uint32_t(tn) * 2 * kGroup * 128);
         }
-        // the Q boxes of the tile, issued together: lane 2e + h copies half h
-        // of query e (one copy per lane instead of sixteen from one lane)
-        if (__shfl_sync(MSA_FULL_MASK, good, 0) && lane < 2 * tn) {
-          const int e = lane >> 1, h = lane & 1;
+        // the Q boxes of the tile, issued together: lane e copies query e
+        if (__shfl_sync(MSA_FULL_MASK, good, 0) && lane < tn) {
+          const int e = lane;
           int qr = trow[0];
 #pragma unroll
           for (int x = 1; x < kQPerTile; ++x) qr = e == x ? trow[x] : qr;
-          tc::tma_load_2d_hint(qbuf + q_stage * kQBytes + h * kQHalf + e * (kGroup * 128), &tmap_q,
-                               &bars->q_full[q_stage], 64 * h, qr * P.Hq + tg * kGroup, q_policy);
+          // one box: the query's 16 heads as two 8-row groups, each group's two
+          // 64-dim halves adjacent (1 KB each, 128-byte swizzle)
+          tc::tma_load_4d_hint(qbuf + q_stage * kQBytes + e * (kGroup * 256), &tmap_q,
+                               &bars->q_full[q_stage], 0, 0, 0, (qr * P.Hq + tg * kGroup) >> 3,
+                               q_policy);
         }
         if (lane == 0) {
           const int d = jt % kDesc;
@@ -331,7 +335,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off = (kk >> 2) * kQHalf + (kk & 3) * 32;
-                tc::mma_ss(dt, tc::sdesc_sw128(qa + off, 16, 1024),
+                // Q: 8-row groups 2 KB apart, the 64-dim halves 1 KB apart inside
+                const uint32_t qoff = (kk >> 2) * 1024 + (kk & 3) * 32;
+                tc::mma_ss(dt, tc::sdesc_sw128(qa + qoff, 16, 2048),
                            tc::sdesc_sw128(ka + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
               }
               tc::mma_commit(&bars->s_full[buf]);
@@ -536,11 +542,12 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap mq, mk, mv, mo32, mo16;
   {
-    cuuint64_t dims[2] = {128, cuuint64_t(P.T) * P.Hq};
-    cuuint64_t strides[1] = {128 * 2};
-    cuuint32_t box[2] = {64, kGroup};
-    cuuint32_t estr[2] = {1, 1};
-    if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box,
+    // Q rows (token, head) of 128 dims viewed as (64 dims, 8 rows, 2 halves, row groups)
+    cuuint64_t dims[4] = {64, 8, 2, cuuint64_t(P.T) * P.Hq / 8};
+    cuuint64_t strides[3] = {128 * 2, 64 * 2, 8 * 128 * 2};
+    cuuint32_t box[4] = {64, 8, 2, kGroup / 8};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
