@@ -64,26 +64,43 @@ __host__ __device__ inline long long pairs_per_seq(const Problem& P) {
   return pairs_before(P, M - 1) + tile_blocks(P, M - 1);
 }
 
+// Query tiles are walked in the order 0, M-1, 1, M-2, ... so that every CTA's
+// contiguous share of pairs mixes short (early) and long (late) tiles: the
+// number of tile switches, each of which reloads the index queries into TMEM,
+// is then about the same on every CTA.
+__host__ __device__ inline int tile_at(const Problem& P, int u) {
+  return (u & 1) ? mtiles(P) - 1 - (u >> 1) : (u >> 1);
+}
+
+// Pairs of one sequence before position u of that order: the first (u+1)/2
+// tiles plus the last u/2 tiles.
+__host__ __device__ inline long long pairs_before_at(const Problem& P, int u, long long per_seq) {
+  const int ne = (u + 1) >> 1, no = u >> 1;
+  return pairs_before(P, ne) + (no > 0 ? per_seq - pairs_before(P, mtiles(P) - no) : 0);
+}
+
 // Walks (b, m, c) over a contiguous range of the linear pair index.
 struct Walk {
-  int b, m, c, nc;
+  int b, u, m, c, nc;
   __device__ void start(const Problem& P, long long L, long long per_seq) {
     b = int(L / per_seq);
     long long l = L % per_seq;
     int lo = 0, hi = mtiles(P) - 1;
     while (lo < hi) {
       int mid = (lo + hi + 1) >> 1;
-      if (pairs_before(P, mid) <= l) lo = mid; else hi = mid - 1;
+      if (pairs_before_at(P, mid, per_seq) <= l) lo = mid; else hi = mid - 1;
     }
-    m = lo;
-    c = int(l - pairs_before(P, m));
+    u = lo;
+    m = tile_at(P, u);
+    c = int(l - pairs_before_at(P, u, per_seq));
     nc = tile_blocks(P, m);
   }
   // advances; returns true when the next pair starts a new query tile
   __device__ bool next(const Problem& P) {
     if (++c < nc) return false;
     c = 0;
-    if (++m == mtiles(P)) { m = 0; ++b; }
+    if (++u == mtiles(P)) { u = 0; ++b; }
+    m = tile_at(P, u);
     nc = tile_blocks(P, m);
     return true;
   }
@@ -166,15 +183,15 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       bool seg_start = true;
       for (long long L = L0; L < L1 && !failed; ++L) {
         if (seg_start) {
-          if (!tc::mbar_wait(&bars->a_full, a_phase, abort)) { failed = true; break; }
+          if (!tc::mbar_spin(&bars->a_full, a_phase, abort)) { failed = true; break; }
           a_phase ^= 1;
           tc::tc_fence_after();
         }
-        if (!tc::mbar_wait(&bars->full[stage], phase, abort)) { failed = true; break; }
+        if (!tc::mbar_spin(&bars->full[stage], phase, abort)) { failed = true; break; }
         tc::tc_fence_after();
         const uint32_t sbase = tc::smem_addr(stages + stage * kStageBytes);
         for (int g = 0; g < P.Hkv; ++g) {
-          if (!tc::mbar_wait(&bars->acc_empty[slot], acc_phase ^ 1, abort)) {
+          if (!tc::mbar_spin(&bars->acc_empty[slot], acc_phase ^ 1, abort)) {
             failed = true;
             break;
           }
