@@ -313,44 +313,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       uint32_t kv_phase[2] = {0, 0};
       int ns = 0, np = 0;
       uint32_t idle = 0;
+      uint32_t sgot = 0;  // barriers of tile ns already seen complete (each is polled until then)
       while (tile_of(np) < total) {
         bool progress = false;
-        if (ns < np + 2 && tile_of(ns) < total) {
-          const int d = ns % kDesc, buf = ns & 1, qs = ns % kQStages;
-          if (tc::mbar_poll(&bars->d_full[d], (ns / kDesc) & 1)) {
-            const int flags = bars->desc[d].flags;
-            const int kvs = flags >> 2;
-            // S overwrites only the S|P columns of its buffer, which are free
-            // once the P V product of the buffer's previous tile has completed;
-            // the O columns may still be draining in the epilogue
-            const bool ready =
-                (!(flags & 1) || tc::mbar_poll(&bars->kv_full[kvs], kv_phase[kvs])) &&
-                tc::mbar_poll(&bars->q_full[qs], (ns / kQStages) & 1) &&
-                tc::mbar_poll(&bars->o_full[buf], ((ns >> 1) & 1) ^ 1);
-            if (ready) {
-              tc::tc_fence_after();
-              const uint32_t qa = tc::smem_addr(qbuf + qs * kQBytes);
-              const uint32_t ka = tc::smem_addr(kvbuf + kvs * kKVBytes);
-              const uint32_t dt = tmem + buf * 256;
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * kQHalf + (kk & 3) * 32;
-                // Q: 8-row groups 2 KB apart, the 64-dim halves 1 KB apart inside
-                const uint32_t qoff = (kk >> 2) * 1024 + (kk & 3) * 32;
-                tc::mma_ss(dt, tc::sdesc_sw128(qa + qoff, 16, 2048),
-                           tc::sdesc_sw128(ka + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-              }
-              tc::mma_commit(&bars->s_full[buf]);
-              if (flags & 1) kv_phase[kvs] ^= 1;
-              ++ns;
-              progress = true;
-            }
-          }
-        }
-        // O = P V needs its P and the O columns drained by the epilogue of the
-        // buffer's previous tile
-        if (np < ns && tc::mbar_poll(&bars->p_full[np & 1], (np >> 1) & 1) &&
-            tc::mbar_poll(&bars->buf_empty[np & 1], ((np >> 1) & 1) ^ 1)) {
+        // O = P V first (it is on its warpgroup's path).  Its P implies that the
+        // O columns are drained: the same four warps read the buffer's previous O
+        // before they wrote this P.
+        if (np < ns && tc::mbar_poll(&bars->p_full[np & 1], (np >> 1) & 1)) {
           tc::tc_fence_after();
           const int buf = np & 1, d = np % kDesc;
           const int flags = bars->desc[d].flags;
@@ -367,6 +336,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
           tc::mbar_arrive(&bars->d_empty[d]);
           ++np;
           progress = true;
+        }
+        if (ns < np + 2 && tile_of(ns) < total) {
+          const int d = ns % kDesc, buf = ns & 1, qs = ns % kQStages;
+          if (!(sgot & 1) && tc::mbar_poll(&bars->d_full[d], (ns / kDesc) & 1)) sgot |= 1;
+          if (sgot & 1) {
+            const int flags = bars->desc[d].flags;
+            const int kvs = flags >> 2;
+            // S overwrites only the S|P columns of its buffer, which are free
+            // once the P V product of the buffer's previous tile has completed
+            if (!(sgot & 2) && (!(flags & 1) || tc::mbar_poll(&bars->kv_full[kvs], kv_phase[kvs])))
+              sgot |= 2;
+            if (!(sgot & 4) && tc::mbar_poll(&bars->q_full[qs], (ns / kQStages) & 1)) sgot |= 4;
+            if (!(sgot & 8) && tc::mbar_poll(&bars->o_full[buf], ((ns >> 1) & 1) ^ 1)) sgot |= 8;
+            if (sgot == 15) {
+              tc::tc_fence_after();
+              const uint32_t qa = tc::smem_addr(qbuf + qs * kQBytes);
+              const uint32_t ka = tc::smem_addr(kvbuf + kvs * kKVBytes);
+              const uint32_t dt = tmem + buf * 256;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * kQHalf + (kk & 3) * 32;
+                // Q: 8-row groups 2 KB apart, the 64-dim halves 1 KB apart inside
+                const uint32_t qoff = (kk >> 2) * 1024 + (kk & 3) * 32;
+                tc::mma_ss(dt, tc::sdesc_sw128(qa + qoff, 16, 2048),
+                           tc::sdesc_sw128(ka + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+              }
+              tc::mma_commit(&bars->s_full[buf]);
+              if (flags & 1) kv_phase[kvs] ^= 1;
+              sgot = 0;
+              ++ns;
+              progress = true;
+            }
+          }
         }
         if (progress) {
           idle = 0;
