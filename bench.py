@@ -300,7 +300,7 @@ def run_e2e(msa, w, xh, out_h, steps, warmup):
 NCU_TRAFFIC = {
     # stage: (workload, source file, git blob id, bytes per launch)
     "attn": ("prefill_128k", "block_sparse_gqa_04_b200/csrc/attn_tc.cu",
-             "0de5df29cbd87c2c6db149d53ee96dba5c7fd1a8", 12784880128 + 34592174592),
+             "bcf6c0a9947c62b858e686af6f4ba095906b6513", 13299131136 + 34592495360),
 }
 
 
