@@ -56,7 +56,7 @@ def counts(w: Workload) -> dict:
     index_flops = 2.0 * w.index_dim * w.num_kv_heads * vis_keys
     main_flops = 4.0 * w.head_dim * w.num_q_heads * w.block_size * sel_blocks
     esz = 4 if w.dtype == "f32" else 2
-    kidx_bytes = float(B * w.kv_len * w.index_dim * esz)
+    kidx_bytes = float(B * w.kv_len * w.index_dim * (1 if w.index_dtype == "fp8" else esz))
     bmax_read = float(B * w.num_kv_heads * np.sum(c_t) * 4)
     partial_bytes = float(w.num_q_heads * sel_blocks * (w.head_dim * esz + 4))
     out_bytes = float(w.rows * w.num_q_heads * w.head_dim * esz)
@@ -424,7 +424,8 @@ def weak_value(rows_per_rank: int, ms_local: float, world: int) -> tuple:
 
 
 def workload_config(w: Workload, world: int) -> dict:
-    return {"workload": w.name, "batch": w.batch, "q_len": w.q_len, "kv_len": w.kv_len,
+    return {"workload": w.name, "index_dtype": w.index_dtype or w.dtype,
+            "batch": w.batch, "q_len": w.q_len, "kv_len": w.kv_len,
             "q_pos0": w.q_pos0, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "index_dim": w.index_dim, "block_size": w.block_size,
             "top_k": w.top_k, "parallelism": f"replicas x{world} (independent problems)"}
@@ -450,6 +451,8 @@ def main():
     ap.add_argument("--seq", type=int, default=0,
                     help="prefill length override (a smaller case of the same structure, "
                          "e.g. for profiling); needles scale with the length")
+    ap.add_argument("--index-dtype", default="", choices=["", "fp8"],
+                    help="fp8: q_idx and k_idx in fp8 e4m3 (bf16 workloads)")
     ap.add_argument("--batch", type=int, default=0,
                     help="batch override (a smaller case of the same structure, e.g. for "
                          "profiling); needles per sequence are kept")
@@ -463,6 +466,8 @@ def main():
             raise SystemExit("--seq applies to the prefill workloads")
         w = w.with_(name=f"{w.name}@{a.seq}", q_len=a.seq, kv_len=a.seq,
                     needles=max(1, w.needles * a.seq // w.q_len))
+    if a.index_dtype:
+        w = w.with_(name=f"{w.name}+idx_{a.index_dtype}", index_dtype=a.index_dtype)
     if a.batch:
         w = w.with_(name=f"{w.name}@b{a.batch}", batch=a.batch)
     peaks, peak_src = load_peaks()
@@ -528,7 +533,7 @@ def main():
                        "ms_per_step": e_ms}
     x_main = main_res.pop("x")
     if not a.no_decode:
-        wd = WORKLOADS["decode_128k"]
+        wd = WORKLOADS["decode_128k"].with_(index_dtype=a.index_dtype)
         del x_main
         torch.cuda.empty_cache()
         dres = measure_workload(msa, wd, dev, a.steps, a.warmup, peaks, False)

@@ -34,41 +34,50 @@
 namespace msa {
 namespace {
 
-constexpr int kKBytes = 128 * 128 * 2;  // one block of k_idx
-constexpr int kKHalf = kKBytes / 2;     // 64 dims (128 B) x 128 keys
+constexpr int kKHalf = 128 * 128;      // 128-byte rows x 128 keys (one swizzle span)
 constexpr int kThreads = 192;
 constexpr int kSlots = 4;               // TMEM accumulators
 constexpr int kMaxRG = 32;              // (rows per sequence) x groups handled
 
-template <int N>
+// N: padded query width (16 or 32); FP8: fp8 e4m3 index tensors (one 128-byte
+// half per row, kind::f8f6f4) instead of bf16 (two halves, kind::f16).
+template <int N, bool FP8>
 struct Cfg {
-  // 16-wide tiles: two CTAs of three stages per SM (two TMA streams per SM
-  // move more bytes than one); 32-wide tiles need more shared memory per stage
-  static constexpr int kStages = N <= 16 ? 3 : 5;
-  static constexpr int kCtasPerSm = N <= 16 ? 2 : 1;
-  static constexpr int kQHalf = N * 128;                 // 64 dims x N padded queries
-  static constexpr int kStageBytes = kKBytes + 2 * kQHalf;
+  static constexpr int kHalves = FP8 ? 1 : 2;            // 128-byte halves of a row
+  static constexpr int kRowChunks = 8 * kHalves;          // 16-byte chunks of a row
+  static constexpr int kKBytes = kHalves * kKHalf;        // one block of k_idx
+  static constexpr int kSteps = FP8 ? 4 : 8;              // K steps of 32 bytes
+  // 16-wide bf16 tiles and all fp8 tiles: two CTAs per SM (two TMA streams per
+  // SM move more bytes than one); 32-wide bf16 tiles need more shared memory
+  static constexpr int kStages = FP8 ? 5 : (N <= 16 ? 3 : 5);
+  static constexpr int kCtasPerSm = (FP8 || N <= 16) ? 2 : 1;
+  static constexpr int kQHalf = N * 128;                  // 128-byte rows of N padded queries
+  static constexpr int kStageBytes = kKBytes + kHalves * kQHalf;
   static constexpr uint32_t kTmemCols = kSlots * N < 32 ? 32 : kSlots * N;
-  static constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, N, 0, 0);
+  static constexpr uint32_t kIdesc =
+      FP8 ? tc::idesc_e4m3_f32(128, N) : tc::idesc_bf16_f32(128, N, 0, 0);
   static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
 };
 
-template <int N>
+template <int N, bool FP8>
 struct Shared {
-  uint64_t full[Cfg<N>::kStages], empty[Cfg<N>::kStages];
+  uint64_t full[Cfg<N, FP8>::kStages], empty[Cfg<N, FP8>::kStages];
   uint64_t acc_full[kSlots], acc_empty[kSlots];
   uint32_t red[kSlots][4][N];   // per accumulator: the four warps' column maxima
-  int qseq[Cfg<N>::kStages];    // sequence whose queries each stage holds (-1: none)
+  int qseq[Cfg<N, FP8>::kStages];  // sequence whose queries each stage holds (-1: none)
   uint32_t tmem_base;
   int abort;
 };
 
-template <int N>
+template <int N, bool FP8>
 constexpr size_t smem_bytes() {
-  return 1024 + Cfg<N>::kStages * Cfg<N>::kStageBytes + sizeof(Shared<N>) + 64;
+  return 1024 + Cfg<N, FP8>::kStages * Cfg<N, FP8>::kStageBytes + sizeof(Shared<N, FP8>) + 64;
 }
-static_assert(smem_bytes<16>() <= 232448, "more dynamic shared memory than a B200 CTA can have");
-static_assert(smem_bytes<32>() <= 232448, "more dynamic shared memory than a B200 CTA can have");
+// two CTAs per SM must fit in the SM's 228 KB where kCtasPerSm is 2
+static_assert(smem_bytes<16, false>() <= 116736, "two CTAs per SM");
+static_assert(smem_bytes<32, false>() <= 232448, "one CTA per SM");
+static_assert(smem_bytes<16, true>() <= 116736, "two CTAs per SM");
+static_assert(smem_bytes<32, true>() <= 116736, "two CTAs per SM");
 
 // Barrier of the four epilogue warps that also returns whether any of their
 // threads passed `v` (so that they leave together on a failed wait).
@@ -85,28 +94,28 @@ __device__ __forceinline__ bool epi_any(bool v) {
   return r != 0;
 }
 
-template <int N>
+template <int N, bool FP8>
 __global__ void __launch_bounds__(kThreads, 2)
 index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
-                    const __nv_bfloat16* __restrict__ q_idx, float* __restrict__ bmax,
+                    const uint8_t* __restrict__ q_idx, float* __restrict__ bmax,
                     int* __restrict__ status, int nvis) {
-  using C = Cfg<N>;
+  using C = Cfg<N, FP8>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  Shared<N>* sh = reinterpret_cast<Shared<N>*>(smem + S * C::kStageBytes);
+  Shared<N, FP8>* sh = reinterpret_cast<Shared<N, FP8>*>(smem + S * C::kStageBytes);
   volatile int* abort = &sh->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int RG = P.Sq * P.Hkv;
 
   // zero the padded query rows RG..N-1 of every stage once; only rows < RG are
   // rewritten later
-  for (int e = threadIdx.x; e < S * 2 * (N - RG) * 8; e += kThreads) {
-    const int st = e / (2 * (N - RG) * 8), rem = e % (2 * (N - RG) * 8);
+  for (int e = threadIdx.x; e < S * C::kHalves * (N - RG) * 8; e += kThreads) {
+    const int st = e / (C::kHalves * (N - RG) * 8), rem = e % (C::kHalves * (N - RG) * 8);
     const int h = rem / ((N - RG) * 8), x = rem % ((N - RG) * 8);
-    *reinterpret_cast<uint4*>(stages + st * C::kStageBytes + kKBytes + h * C::kQHalf +
+    *reinterpret_cast<uint4*>(stages + st * C::kStageBytes + C::kKBytes + h * C::kQHalf +
                               RG * 128 + x * 16) = make_uint4(0, 0, 0, 0);
   }
   tc::fence_async_smem();
@@ -137,7 +146,7 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
 
   if (warp == 0) {
     // ---------------- producer: k_idx by TMA, queries from registers ----------------
-    constexpr int kQv = N / 2;          // 16-byte query chunks per lane (RG * 16 / 32 at most)
+    constexpr int kQv = N * C::kRowChunks / 32;  // 16-byte query chunks per lane, at most
     uint4 qv[kQv];
     int qb = -1;
     int k = 0;
@@ -146,11 +155,12 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       const uint32_t ph = (k / S) & 1;
       const int b = int(it / nvis), c = int(it % nvis);
       if (b != qb) {
-        const uint4* src = reinterpret_cast<const uint4*>(q_idx + (long long)b * RG * 128);
+        const uint4* src =
+            reinterpret_cast<const uint4*>(q_idx + (long long)b * RG * C::kRowChunks * 16);
 #pragma unroll
         for (int x = 0; x < kQv; ++x) {
           const int e = lane + 32 * x;
-          qv[x] = e < RG * 16 ? __ldg(src + e) : make_uint4(0, 0, 0, 0);
+          qv[x] = e < RG * C::kRowChunks ? __ldg(src + e) : make_uint4(0, 0, 0, 0);
         }
         qb = b;
       }
@@ -159,10 +169,10 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       if (!__shfl_sync(MSA_FULL_MASK, ok, 0)) { failed = true; break; }
       uint8_t* st = stages + s * C::kStageBytes;
       if (lane == 0) {
-        tc::mbar_arrive_expect_tx(&sh->full[s], kKBytes);
+        tc::mbar_arrive_expect_tx(&sh->full[s], C::kKBytes);
         const int row = b * P.Skv + c * 128;
         tc::tma_load_2d(st, &tmap_k, &sh->full[s], 0, row);
-        tc::tma_load_2d(st + kKHalf, &tmap_k, &sh->full[s], 64, row);
+        if (!FP8) tc::tma_load_2d(st + kKHalf, &tmap_k, &sh->full[s], 64, row);
       }
       // query chunk e = (row n, 16-byte chunk j of its 256 B): K-major, 128-byte
       // swizzle, the layout TMA gives the key block.  A stage that already
@@ -172,9 +182,9 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
 #pragma unroll
         for (int x = 0; x < kQv; ++x) {
           const int e = lane + 32 * x;
-          if (e < RG * 16) {
-            const int n = e >> 4, j = e & 15;
-            *reinterpret_cast<uint4*>(st + kKBytes + (j >> 3) * C::kQHalf + n * 128 +
+          if (e < RG * C::kRowChunks) {
+            const int n = e / C::kRowChunks, j = e % C::kRowChunks;
+            *reinterpret_cast<uint4*>(st + C::kKBytes + (j >> 3) * C::kQHalf + n * 128 +
                                       (((j & 7) ^ (n & 7)) << 4)) = qv[x];
           }
         }
@@ -199,13 +209,16 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
         }
         tc::tc_fence_after();
         const uint32_t kb = tc::smem_addr(stages + s * C::kStageBytes);
-        const uint32_t qbase = kb + kKBytes;
+        const uint32_t qbase = kb + C::kKBytes;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < C::kSteps; ++kk) {
           const uint64_t ad = tc::sdesc_sw128(kb + (kk >> 2) * kKHalf + (kk & 3) * 32, 16, 1024);
           const uint64_t bd =
               tc::sdesc_sw128(qbase + (kk >> 2) * C::kQHalf + (kk & 3) * 32, 16, 1024);
-          tc::mma_ss(tmem + slot * N, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
+          if (FP8)
+            tc::mma_ss_f8(tmem + slot * N, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
+          else
+            tc::mma_ss(tmem + slot * N, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&sh->acc_full[slot]);
         tc::mma_commit(&sh->empty[s]);
@@ -302,15 +315,18 @@ bool index_decode_supported(const Problem& P) {
          (long long)P.B * P.Skv < (1LL << 31);
 }
 
-template <int N>
+template <int N, bool FP8>
 static cudaError_t launch_n(const CUtensorMap& map, const Problem& P, const void* q_idx,
-                            float* bmax, int32_t* status, int nvis, int grid, cudaStream_t s) {
-  constexpr size_t smem = smem_bytes<N>();
-  cudaError_t e = cudaFuncSetAttribute(index_decode_kernel<N>,
+                            float* bmax, int32_t* status, int nvis, long long items,
+                            cudaStream_t s) {
+  constexpr size_t smem = smem_bytes<N, FP8>();
+  const int grid =
+      int(std::min<long long>((long long)sm_count() * Cfg<N, FP8>::kCtasPerSm, items));
+  cudaError_t e = cudaFuncSetAttribute(index_decode_kernel<N, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  index_decode_kernel<N><<<grid, kThreads, smem, s>>>(
-      map, P, static_cast<const __nv_bfloat16*>(q_idx), bmax, status, nvis);
+  index_decode_kernel<N, FP8><<<grid, kThreads, smem, s>>>(
+      map, P, static_cast<const uint8_t*>(q_idx), bmax, status, nvis);
   return cudaGetLastError();
 }
 
@@ -319,22 +335,25 @@ cudaError_t launch_index_decode(const Problem& P, const void* q_idx, const void*
   if (!index_decode_supported(P)) return cudaErrorNotSupported;
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
+  // k_idx rows of 128 dims as 128-byte-wide boxes of 128 keys (128-byte swizzle)
   CUtensorMap map;
   cuuint64_t dims[2] = {128, cuuint64_t(P.B) * P.Skv};
-  cuuint64_t strides[1] = {128 * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint64_t strides[1] = {P.idx8 ? 128u : 256u};
+  cuuint32_t box[2] = {P.idx8 ? 128u : 64u, 128};
   cuuint32_t estr[2] = {1, 1};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_idx), dims, strides, box,
-          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  if (enc(&map, P.idx8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+          const_cast<void*>(k_idx), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   const int nvis = int((P.q_pos0 + P.Sq - 1) / P.Bk) + 1;
   const long long items = (long long)P.B * nvis;
   const int rg = P.Sq * P.Hkv;
-  const int per_sm = rg <= 16 ? Cfg<16>::kCtasPerSm : Cfg<32>::kCtasPerSm;
-  const int grid = int(std::min<long long>((long long)sm_count() * per_sm, items));
-  return rg <= 16 ? launch_n<16>(map, P, q_idx, bmax, status, nvis, grid, s)
-                  : launch_n<32>(map, P, q_idx, bmax, status, nvis, grid, s);
+  if (P.idx8)
+    return rg <= 16 ? launch_n<16, true>(map, P, q_idx, bmax, status, nvis, items, s)
+                    : launch_n<32, true>(map, P, q_idx, bmax, status, nvis, items, s);
+  return rg <= 16 ? launch_n<16, false>(map, P, q_idx, bmax, status, nvis, items, s)
+                  : launch_n<32, false>(map, P, q_idx, bmax, status, nvis, items, s);
 }
 
 }  // namespace msa

@@ -35,14 +35,24 @@ namespace msa {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kStageBytes = 128 * 128 * 2;  // one k_idx block, bf16
-constexpr int kHalfBytes = kStageBytes / 2; // 64 dims (128 B) x 128 keys
 constexpr int kThreads = 320;               // TMA, MMA, two epilogue warpgroups
 constexpr int kMaxGroups = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 256;           // accumulators follow the A region
-constexpr uint32_t kIdesc = tc::idesc_bf16_f32(128, 128, 0, 0);
-constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + 256;
+
+// Element type of the index tensors: bf16 (kind::f16, two 64-dim halves per key
+// row) or fp8 e4m3 (kind::f8f6f4, one 128-byte half, half the bytes).
+template <bool FP8>
+struct Idx {
+  static constexpr int kRowBytes = FP8 ? 128 : 256;            // one key / query row
+  static constexpr int kStageBytes = 128 * kRowBytes;          // one k_idx block
+  static constexpr int kHalfBytes = 128 * 128;                 // 128-byte rows x 128 keys
+  static constexpr int kSteps = FP8 ? 4 : 8;                   // K steps of 32 bytes
+  static constexpr uint32_t kGroupCols = FP8 ? 32 : 64;        // TMEM columns per group
+  static constexpr uint32_t kIdesc =
+      FP8 ? tc::idesc_e4m3_f32(128, 128) : tc::idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + 256;
+};
 
 // Blocks query tile m (128 rows) of a sequence can see.
 __host__ __device__ inline int tile_blocks(const Problem& P, int m) {
@@ -117,15 +127,17 @@ struct Bars {
   int abort;
 };
 
+template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
 index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
-                const __nv_bfloat16* __restrict__ q_idx, float* __restrict__ bmax,
+                const uint8_t* __restrict__ q_idx, float* __restrict__ bmax,
                 int* __restrict__ status, long long per_seq) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+  using X = Idx<FP8>;
+  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * X::kStageBytes);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -164,11 +176,11 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       uint32_t phase = 0;
       for (long long L = L0; L < L1; ++L) {
         if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort)) { failed = true; break; }
-        tc::mbar_arrive_expect_tx(&bars->full[stage], kStageBytes);
+        tc::mbar_arrive_expect_tx(&bars->full[stage], X::kStageBytes);
         const int row = w.b * P.Skv + w.c * P.Bk;
-        uint8_t* dst = stages + stage * kStageBytes;
+        uint8_t* dst = stages + stage * X::kStageBytes;
         tc::tma_load_2d(dst, &tmap_k, &bars->full[stage], 0, row);
-        tc::tma_load_2d(dst + kHalfBytes, &tmap_k, &bars->full[stage], 64, row);
+        if (!FP8) tc::tma_load_2d(dst + X::kHalfBytes, &tmap_k, &bars->full[stage], 64, row);
         if (++stage == kStages) { stage = 0; phase ^= 1; }
         w.next(P);
       }
@@ -189,7 +201,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
         }
         if (!tc::mbar_spin(&bars->full[stage], phase, abort)) { failed = true; break; }
         tc::tc_fence_after();
-        const uint32_t sbase = tc::smem_addr(stages + stage * kStageBytes);
+        const uint32_t sbase = tc::smem_addr(stages + stage * X::kStageBytes);
         for (int g = 0; g < P.Hkv; ++g) {
           if (!tc::mbar_spin(&bars->acc_empty[slot], acc_phase ^ 1, abort)) {
             failed = true;
@@ -198,10 +210,14 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
           tc::tc_fence_after();
           const uint32_t d = tmem + kAccCol + slot * 128;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t bd = tc::sdesc_sw128(sbase + (kk >> 2) * kHalfBytes + (kk & 3) * 32,
+          for (int kk = 0; kk < X::kSteps; ++kk) {
+            // 32 bytes of K per step: 16 bf16 or 32 fp8, 8 TMEM columns of A
+            const uint64_t bd = tc::sdesc_sw128(sbase + (kk >> 2) * X::kHalfBytes + (kk & 3) * 32,
                                                 16, 1024);
-            tc::mma_ts(d, tmem + g * 64 + kk * 8, bd, kIdesc, kk > 0 ? 1u : 0u);
+            if (FP8)
+              tc::mma_ts_f8(d, tmem + g * X::kGroupCols + kk * 8, bd, X::kIdesc, kk > 0 ? 1u : 0u);
+            else
+              tc::mma_ts(d, tmem + g * X::kGroupCols + kk * 8, bd, X::kIdesc, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&bars->acc_full[slot]);
           slot ^= 1;
@@ -241,20 +257,21 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
           }
           first = false;
           // each warpgroup writes the index queries of every other group
-          const uint4* src = reinterpret_cast<const uint4*>(q_idx + r * P.Hkv * 128);
+          const uint4* src = reinterpret_cast<const uint4*>(q_idx + r * P.Hkv * X::kRowBytes);
           for (int g = ewg; g < P.Hkv; g += 2) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < X::kRowBytes / 128; ++h) {
               uint32_t v[32];
 #pragma unroll
               for (int x = 0; x < 8; ++x) {
-                uint4 u = valid ? __ldg(src + g * 16 + h * 8 + x) : make_uint4(0, 0, 0, 0);
+                uint4 u = valid ? __ldg(src + g * (X::kRowBytes / 16) + h * 8 + x)
+                                : make_uint4(0, 0, 0, 0);
                 v[4 * x + 0] = u.x;
                 v[4 * x + 1] = u.y;
                 v[4 * x + 2] = u.z;
                 v[4 * x + 3] = u.w;
               }
-              tc::tmem_st32(tmem + lane_addr + g * 64 + h * 32, v);
+              tc::tmem_st32(tmem + lane_addr + g * X::kGroupCols + h * 32, v);
             }
           }
           tc::tmem_st_wait();
@@ -345,29 +362,39 @@ bool index_tc_supported(const Problem& P) {
          (long long)P.B * P.Skv < (1LL << 31);
 }
 
-cudaError_t launch_index_tc(const Problem& P, const void* q_idx, const void* k_idx,
-                            float* bmax, int32_t* status, cudaStream_t s) {
+template <bool FP8>
+static cudaError_t launch_t(const Problem& P, const void* q_idx, const void* k_idx, float* bmax,
+                           int32_t* status, cudaStream_t s) {
+  using X = Idx<FP8>;
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
+  // k_idx rows of 128 dims, copied as 128-byte-wide boxes of 128 keys (128-byte swizzle)
   CUtensorMap map;
-  cuuint64_t dims[2] = {128, cuuint64_t(P.B) * P.Skv};
-  cuuint64_t strides[1] = {128 * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint64_t dims[2] = {FP8 ? 128u : 128u, cuuint64_t(P.B) * P.Skv};
+  cuuint64_t strides[1] = {cuuint64_t(X::kRowBytes)};
+  cuuint32_t box[2] = {FP8 ? 128u : 64u, 128};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_idx), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = enc(&map, FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(k_idx), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   const long long per_seq = pairs_per_seq(P);
   const long long total = per_seq * P.B;
   const int grid = int(std::min<long long>(sm_count(), total));
-  cudaError_t e = cudaFuncSetAttribute(index_tc_kernel,
+  cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(kSmemBytes));
+                                       int(X::kSmemBytes));
   if (e != cudaSuccess) return e;
-  index_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(
-      map, P, static_cast<const __nv_bfloat16*>(q_idx), bmax, status, per_seq);
+  index_tc_kernel<FP8><<<grid, kThreads, X::kSmemBytes, s>>>(
+      map, P, static_cast<const uint8_t*>(q_idx), bmax, status, per_seq);
   return cudaGetLastError();
+}
+
+cudaError_t launch_index_tc(const Problem& P, const void* q_idx, const void* k_idx,
+                            float* bmax, int32_t* status, cudaStream_t s) {
+  return P.idx8 ? launch_t<true>(P, q_idx, k_idx, bmax, status, s)
+                : launch_t<false>(P, q_idx, k_idx, bmax, status, s);
 }
 
 }  // namespace msa

@@ -18,7 +18,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
-MSA_BF16, MSA_F32 = 0, 1
+MSA_BF16, MSA_F32, MSA_FP8_E4M3 = 0, 1, 2
 OP_SELECT, OP_ATTEND, OP_FORWARD = 0, 1, 2
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
@@ -44,7 +44,7 @@ class Problem(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("index_dim", ctypes.c_int32),
         ("block_size", ctypes.c_int32), ("top_k", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("q_pos0", ctypes.c_int64), ("softmax_scale", ctypes.c_float),
-        ("reserved", ctypes.c_int32),
+        ("index_dtype", ctypes.c_int32),
     ]
 
 
@@ -87,17 +87,21 @@ def load() -> ctypes.CDLL:
 
 def make_problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
                  block_size=128, top_k=16, dtype=torch.bfloat16, q_pos0=0,
-                 softmax_scale=0.0) -> Problem:
+                 softmax_scale=0.0, index_dtype=None) -> Problem:
+    """dtype: torch dtype of q/k/v (fp32 or bf16); index_dtype: torch dtype of
+    q_idx/k_idx when it differs (torch.float8_e4m3fn for fp8 index tensors)."""
+    fp8 = torch.float8_e4m3fn
+    main = MSA_F32 if dtype == torch.float32 else MSA_BF16
+    idx = MSA_FP8_E4M3 if (index_dtype == fp8 or dtype == fp8) else 0
     return Problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
-                   block_size, top_k, MSA_F32 if dtype == torch.float32 else MSA_BF16,
-                   q_pos0, softmax_scale, 0)
+                   block_size, top_k, main, q_pos0, softmax_scale, idx)
 
 
 def problem_of(w, softmax_scale: float = 0.0) -> Problem:
     """Problem of a :class:`~block_sparse_gqa_04_b200.workload.Workload`."""
     return make_problem(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
                         w.head_dim, w.index_dim, w.block_size, w.top_k, w.torch_dtype,
-                        w.q_pos0, softmax_scale)
+                        w.q_pos0, softmax_scale, index_dtype=w.torch_index_dtype)
 
 
 def workspace_size(p: Problem, op: int = OP_FORWARD) -> int:
@@ -176,7 +180,8 @@ def select(q_idx: torch.Tensor, k_idx: torch.Tensor, *, q_pos0: int = 0, block_s
     _require_cuda(q_idx, k_idx)
     B, Sq, Hkv, di = q_idx.shape
     Skv = k_idx.shape[1]
-    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, top_k, q_idx.dtype, q_pos0)
+    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, top_k, q_idx.dtype, q_pos0,
+                     index_dtype=q_idx.dtype)
     dev = q_idx.device
     q2k = torch.empty((Hkv, B * Sq, top_k), dtype=torch.int32, device=dev)
     nblk = -(-Skv // block_size)
@@ -204,7 +209,8 @@ def select_static(q_idx: torch.Tensor, k_idx: torch.Tensor, q2k: torch.Tensor, *
         raise ValueError("q2k must be int32 [Hkv, B*Sq, top_k]")
     if device_status is not None and device_status.dtype != torch.int32:
         raise ValueError("device_status must be an int32 tensor")
-    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, q2k.shape[2], q_idx.dtype, q_pos0)
+    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, q2k.shape[2], q_idx.dtype, q_pos0,
+                     index_dtype=q_idx.dtype)
     _check(load().msa_select_static(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(q2k),
                                     _ptr(device_status), _stream(q_idx.device)),
            "msa_select_static")
@@ -253,7 +259,7 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
     _require_cuda(q, k, v, q_idx, k_idx)
     B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx)
     p = make_problem(B, Sq, Skv, Hq, Hkv, D, di, block_size, top_k, q.dtype, q_pos0,
-                     softmax_scale)
+                     softmax_scale, index_dtype=q_idx.dtype)
     dev = q.device
     o = out if (out is not None and not host) else torch.empty_like(q)
     lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=dev) if return_lse else None

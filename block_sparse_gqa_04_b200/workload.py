@@ -11,7 +11,8 @@ Recipe (the same for every workload):
     two devices' streams differ; each is fixed by the seed);
   * each tensor is multiplied by 1 (``fp32`` workloads) or by 1/sqrt(d)
     (``bf16`` workloads, d = head_dim for Q/K/V and index_dim for the index
-    tensors) and rounded once to the workload's dtype (round to nearest even);
+    tensors) and rounded once to the workload's dtype (round to nearest even; q_idx and
+    k_idx to fp8 e4m3 instead when index_dtype is "fp8");
   * needles: for every sequence b and group g, ``needles`` distinct "past"
     blocks are drawn uniformly (``torch.randperm`` from the same generator, in
     (b, g) order) from blocks ``0 .. upper-1`` where ``upper`` is the block of
@@ -44,6 +45,7 @@ class Workload:
     top_k: int
     dtype: str          # "f32" or "bf16"
     needles: int        # planted needle blocks per (sequence, group)
+    index_dtype: str = ""  # "" (same as dtype) or "fp8" (q_idx, k_idx in fp8 e4m3)
 
     @property
     def rows(self) -> int:
@@ -56,6 +58,10 @@ class Workload:
     @property
     def torch_dtype(self) -> torch.dtype:
         return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def torch_index_dtype(self) -> torch.dtype:
+        return torch.float8_e4m3fn if self.index_dtype == "fp8" else self.torch_dtype
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -107,7 +113,7 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu") -> Dict[str, torch.Ten
     q = _draw(gen, (B * Sq, w.num_q_heads, w.head_dim), s_main, dt)
     k = _draw(gen, (B * Skv, w.num_kv_heads, w.head_dim), s_main, dt)
     v = _draw(gen, (B * Skv, w.num_kv_heads, w.head_dim), s_main, dt)
-    q_idx = _draw(gen, (B * Sq, w.num_kv_heads, w.index_dim), s_idx, dt)
+    q_idx = _draw(gen, (B * Sq, w.num_kv_heads, w.index_dim), s_idx, w.torch_index_dtype)
     # k_idx stays fp32 until the needles are in, then is rounded once.
     k_idx32 = _draw(gen, (B * Skv, w.index_dim), s_idx, torch.float32)
     needle_ids = torch.full((B, w.num_kv_heads, max(w.needles, 0)), -1, dtype=torch.int64,
@@ -127,7 +133,7 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu") -> Dict[str, torch.Ten
                     lo = c * w.block_size
                     hi = min(lo + w.block_size, Skv)
                     kv[b, lo:hi] += shift
-    k_idx = k_idx32.to(dt)
+    k_idx = k_idx32.to(w.torch_index_dtype)
     return {
         "q": q.view(B, Sq, w.num_q_heads, w.head_dim),
         "k": k.view(B, Skv, w.num_kv_heads, w.head_dim),

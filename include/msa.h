@@ -62,7 +62,10 @@ typedef enum {
   MSA_ERR_TOO_LARGE = 6      /* problem exceeds msa_select_static's scratch   */
 } msa_status_t;
 
-typedef enum { MSA_BF16 = 0, MSA_F32 = 1 } msa_dtype_t;
+/* MSA_FP8_E4M3 is an index_dtype only: fp8 e4m3 index queries and keys of a bf16
+ * problem ("MiniMax új eljárása ..." (aiforradalom.online), section
+ * "Elérhetőség": the MSA inference kernels come in BF16, FP8, NVFP4 and FP4). */
+typedef enum { MSA_BF16 = 0, MSA_F32 = 1, MSA_FP8_E4M3 = 2 } msa_dtype_t;
 
 typedef enum { MSA_OP_SELECT = 0, MSA_OP_ATTEND = 1, MSA_OP_FORWARD = 2 } msa_op_t;
 
@@ -83,7 +86,8 @@ typedef struct {
   int32_t dtype;          /* msa_dtype_t of q, k, v, q_idx, k_idx and out      */
   int64_t q_pos0;         /* absolute position of query row 0 of every sequence */
   float softmax_scale;    /* main-branch logit scale; 0 selects 1/sqrt(head_dim) */
-  int32_t reserved;       /* must be 0                                         */
+  int32_t index_dtype;    /* 0: q_idx and k_idx have `dtype`; MSA_FP8_E4M3: they are
+                             fp8 e4m3 (bf16 problems); other values are invalid  */
 } msa_problem_t;
 
 /* Bytes of workspace that `op` needs for problem `p` (0 if p is invalid).

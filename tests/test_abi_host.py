@@ -45,13 +45,13 @@ def test_problem_struct_layout_matches_header(tmp_path):
         '#include <stdio.h>\n#include <stddef.h>\n#include "msa.h"\n'
         "int main(void){printf(\"%zu %zu %zu %zu\\n\", sizeof(msa_problem_t),"
         " offsetof(msa_problem_t,q_pos0), offsetof(msa_problem_t,softmax_scale),"
-        " offsetof(msa_problem_t,reserved));return 0;}\n")
+        " offsetof(msa_problem_t,index_dtype));return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
                    check=True)
     got = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     P = msa.Problem
-    want = [ctypes.sizeof(P), P.q_pos0.offset, P.softmax_scale.offset, P.reserved.offset]
+    want = [ctypes.sizeof(P), P.q_pos0.offset, P.softmax_scale.offset, P.index_dtype.offset]
     assert [int(x) for x in got] == want
 
 
@@ -76,7 +76,8 @@ def test_workspace_sizes(lib):
     ("index_dim", 48, 2),
     ("q_pos0", 131072, 1),           # q_pos0 + q_len > kv_len
     ("batch", 0, 1),
-    ("reserved", 1, 1),
+    ("index_dtype", 1, 1),           # only fp8 e4m3 may differ from dtype
+    ("index_dtype", 5, 1),
     ("dtype", 7, 1),
 ])
 def test_invalid_problems_are_rejected_on_the_host(lib, field, value, code):
@@ -87,6 +88,19 @@ def test_invalid_problems_are_rejected_on_the_host(lib, field, value, code):
     st = lib.msa_forward(ctypes.byref(p), fake, fake, fake, fake, fake, fake, None, None, fake,
                          1 << 40, None)
     assert st == code
+
+
+def test_index_dtype_values(lib):
+    """fp8 e4m3 index tensors are valid for bf16 problems only."""
+    p = msa.problem_of(workload.WORKLOADS["prefill_32k"])
+    p.index_dtype = msa.MSA_FP8_E4M3
+    assert msa.workspace_size(p, msa.OP_FORWARD) > 0
+    t = msa.problem_of(workload.WORKLOADS["tiny"])       # an fp32 problem
+    assert msa.workspace_size(t, msa.OP_FORWARD) > 0
+    t.index_dtype = msa.MSA_FP8_E4M3
+    assert msa.workspace_size(t, msa.OP_FORWARD) == 0
+    w8 = workload.WORKLOADS["prefill_32k"].with_(index_dtype="fp8")
+    assert msa.problem_of(w8).index_dtype == msa.MSA_FP8_E4M3
 
 
 def test_null_misaligned_and_small_workspace(lib):

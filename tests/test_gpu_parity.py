@@ -31,6 +31,15 @@ SMALL = {
     "decode_rows4": Workload("decode_rows4", 3, 4, 3000, 2942, 32, 4, 128, 128, 128, 8, "bf16", 2),
     "decode_rows8": Workload("decode_rows8", 2, 8, 5000, 4990, 64, 4, 128, 128, 128, 16, "bf16", 2),
     "decode_g2": Workload("decode_g2", 4, 1, 1500, 1499, 16, 2, 128, 128, 128, 4, "bf16", 1),
+    # fp8 (e4m3) index tensors: tensor-core prefill index, decode index at both
+    # query widths, and the SIMT index kernel (index_dim 64)
+    "fp8_prefill": Workload("fp8_prefill", 1, 2125, 2125, 0, 64, 4, 128, 128, 128, 16, "bf16", 2,
+                            "fp8"),
+    "fp8_decode": Workload("fp8_decode", 5, 1, 3000, 2999, 64, 4, 128, 128, 128, 16, "bf16", 3,
+                           "fp8"),
+    "fp8_decode_rows8": Workload("fp8_decode_rows8", 2, 8, 5000, 4990, 64, 4, 128, 128, 128, 16,
+                                 "bf16", 2, "fp8"),
+    "fp8_di64": Workload("fp8_di64", 1, 700, 700, 0, 16, 4, 64, 64, 128, 5, "bf16", 1, "fp8"),
     "top1": Workload("top1", 1, 700, 700, 0, 32, 2, 128, 128, 128, 1, "bf16", 1),
     "d64_g4": Workload("d64_g4", 2, 700, 700, 0, 16, 4, 64, 64, 128, 5, "bf16", 1),
     "f32_d128_g8": Workload("f32_d128_g8", 1, 600, 600, 0, 16, 2, 128, 128, 128, 4, "f32", 0),
@@ -116,7 +125,7 @@ def test_attend_with_oracle_selection(name):
 
 
 @pytest.mark.parametrize("name", ["tiny", "bf16_ragged", "chunk_unaligned", "decode_small",
-                                  "g32_di32"])
+                                  "g32_di32", "fp8_prefill", "fp8_decode", "fp8_di64"])
 def test_select_block_scores(name):
     w = SMALL[name]
     cpu, gpu = _inputs(w)
