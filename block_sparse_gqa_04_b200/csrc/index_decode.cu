@@ -47,10 +47,11 @@ struct Cfg {
   static constexpr int kRowChunks = 8 * kHalves;          // 16-byte chunks of a row
   static constexpr int kKBytes = kHalves * kKHalf;        // one block of k_idx
   static constexpr int kSteps = FP8 ? 4 : 8;              // K steps of 32 bytes
-  // 16-wide bf16 tiles and all fp8 tiles: two CTAs per SM (two TMA streams per
-  // SM move more bytes than one); 32-wide bf16 tiles need more shared memory
-  static constexpr int kStages = FP8 ? 5 : (N <= 16 ? 3 : 5);
-  static constexpr int kCtasPerSm = (FP8 || N <= 16) ? 2 : 1;
+  // Several CTAs per SM, each with its own TMA stream (more streams per SM move
+  // more bytes): 16-wide bf16 tiles two, fp8 tiles (18-20 KB stages) three;
+  // 32-wide bf16 tiles need more shared memory per stage and run one
+  static constexpr int kStages = FP8 ? 3 : (N <= 16 ? 3 : 5);
+  static constexpr int kCtasPerSm = FP8 ? 3 : (N <= 16 ? 2 : 1);
   static constexpr int kQHalf = N * 128;                  // 128-byte rows of N padded queries
   static constexpr int kStageBytes = kKBytes + kHalves * kQHalf;
   static constexpr uint32_t kTmemCols = kSlots * N < 32 ? 32 : kSlots * N;
@@ -76,8 +77,8 @@ constexpr size_t smem_bytes() {
 // two CTAs per SM must fit in the SM's 228 KB where kCtasPerSm is 2
 static_assert(smem_bytes<16, false>() <= 116736, "two CTAs per SM");
 static_assert(smem_bytes<32, false>() <= 232448, "one CTA per SM");
-static_assert(smem_bytes<16, true>() <= 116736, "two CTAs per SM");
-static_assert(smem_bytes<32, true>() <= 116736, "two CTAs per SM");
+static_assert(smem_bytes<16, true>() <= 77824, "three CTAs per SM");
+static_assert(smem_bytes<32, true>() <= 77824, "three CTAs per SM");
 
 // Barrier of the four epilogue warps that also returns whether any of their
 // threads passed `v` (so that they leave together on a failed wait).

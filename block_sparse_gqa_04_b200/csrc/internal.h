@@ -105,7 +105,7 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
                            const Lists& L, const Partials& part, int32_t* status,
                            cudaStream_t s);
 cudaError_t launch_combine(const Problem& P, const int32_t* pos, const Partials& part,
-                           void* out, float* lse, cudaStream_t s);
+                           void* out, float* lse, int32_t* status, cudaStream_t s);
 
 // Device status bits (workspace status word): 1 = invalid q2k entry given to
 // attend, 2 = a bounded wait inside a tensor-core kernel gave up.

@@ -162,7 +162,7 @@ msa_status_t run_attend(const Problem& P, const void* q, const void* k, const vo
     stage_mark(s);
   }
   if (e == cudaSuccess) {
-    e = msa::launch_combine(P, lists.pos, part, out, lse, s);
+    e = msa::launch_combine(P, lists.pos, part, out, lse, at<int32_t>(ws, L.status), s);
     stage_mark(s);
   }
   return cuda_status(e);
