@@ -13,11 +13,15 @@
 // strided share of the row and finds the `need`-th largest of those 32 lane
 // maxima, tau: the lanes holding the top `need` maxima give `need` distinct keys
 // >= tau, so the true top-`need` keys are all >= tau.  The keys >= tau (a few
-// dozen on typical rows) are compacted into shared memory.  Phase 2 picks the
-// top keys among them, one warp-wide maximum at a time, each pass restricted to
-// keys below the previous pick; keys are unique (they carry the block id), so
-// every pass takes exactly one key.  Rows with more candidates than fit in
-// shared memory rescan the row in phase 2 instead.
+// dozen on typical rows) are compacted into shared memory.  Phase 2 keeps the
+// `need` largest of them.  Keys are unique (they carry the block id), so a key's
+// rank (how many keys are larger) decides both steps: each lane counts the
+// larger keys among the 32 it sees through shuffles, which are independent of
+// one another, instead of running `need` dependent warp-wide maxima.  Rows with
+// more than 32 candidates pick them one warp-wide maximum at a time (each pass
+// takes the largest key below the previous pick), and rows with more than fit in
+// shared memory rescan the row for each pass.  Only the set matters: the kept
+// ids are written in ascending order.
 #include "common.cuh"
 #include "internal.h"
 
@@ -25,6 +29,19 @@ namespace msa {
 
 constexpr int kTopkWarps = 8;
 constexpr int kCandCap = 128;  // candidates >= tau kept in shared memory per warp
+
+// Number of lanes among 0 .. n-1 whose key is larger than this lane's.
+__device__ __forceinline__ int warp_rank_u64(uint64_t v, int n) {
+  const uint32_t hi = uint32_t(v >> 32), lo = uint32_t(v);
+  int r = 0;
+#pragma unroll 8
+  for (int i = 0; i < n; ++i) {
+    const uint32_t oh = __shfl_sync(MSA_FULL_MASK, hi, i);
+    const uint32_t ol = __shfl_sync(MSA_FULL_MASK, lo, i);
+    r += (oh > hi) || (oh == hi && ol > lo);
+  }
+  return r;
+}
 
 __global__ void __launch_bounds__(256) topk_kernel(Problem P, const float* __restrict__ bmax,
                                                    int32_t* __restrict__ q2k) {
@@ -40,7 +57,7 @@ __global__ void __launch_bounds__(256) topk_kernel(Problem P, const float* __res
   const int c_t = int(t / P.Bk);
   const int ksel = min(P.K, c_t + 1);
   const int need = ksel - 1;  // earlier blocks to pick
-  int mine = INT_MAX;         // lane s < need holds the s-th pick
+  int mine = INT_MAX;         // lanes 0 .. need-1 hold the picks
   if (need == c_t) {
     // every visible block is selected
     if (lane < c_t) mine = lane;
@@ -52,11 +69,12 @@ __global__ void __launch_bounds__(256) topk_kernel(Problem P, const float* __res
       uint64_t key = block_key(row[c], c);
       lmax = key > lmax ? key : lmax;
     }
-    uint64_t prev = ~0ull, tau = 0;
-    for (int s = 0; s < need; ++s) {
-      tau = warp_max_u64(lmax < prev ? lmax : 0);
-      prev = tau;
-    }
+    // lanes without a block hold 0 and rank below every real key; since
+    // need < c_t, the lane of rank need - 1 holds a real key
+    const int r1 = warp_rank_u64(lmax, 32);
+    const int src = __ffs(__ballot_sync(MSA_FULL_MASK, r1 == need - 1)) - 1;
+    const uint64_t tau = (uint64_t(__shfl_sync(MSA_FULL_MASK, uint32_t(lmax >> 32), src)) << 32) |
+                         __shfl_sync(MSA_FULL_MASK, uint32_t(lmax), src);
     // compact the keys >= tau
     int count = 0;
     for (int base = 0; base < c_t; base += 32) {
@@ -69,24 +87,35 @@ __global__ void __launch_bounds__(256) topk_kernel(Problem P, const float* __res
       count += __popc(m);
     }
     __syncwarp();
-    // phase 2: `need` passes, each taking the largest key below the last pick
-    prev = ~0ull;
-    for (int s = 0; s < need; ++s) {
-      uint64_t best = 0;
-      if (count <= kCandCap) {
-        for (int e = lane; e < count; e += 32) {
-          const uint64_t key = cand[e];
-          if (key < prev && key > best) best = key;
+    if (count <= 32) {
+      // phase 2 by rank: keep the candidates with fewer than `need` larger
+      // ones, placed in lanes 0 .. need-1 by their rank
+      const uint64_t key = lane < count ? cand[lane] : 0;
+      const int r2 = warp_rank_u64(key, count);
+      __syncwarp();
+      if (lane < count && r2 < need) cand[r2] = key;
+      __syncwarp();
+      if (lane < need) mine = key_block(cand[lane]);
+    } else {
+      // phase 2: `need` passes, each taking the largest key below the last pick
+      uint64_t prev = ~0ull;
+      for (int s = 0; s < need; ++s) {
+        uint64_t best = 0;
+        if (count <= kCandCap) {
+          for (int e = lane; e < count; e += 32) {
+            const uint64_t key = cand[e];
+            if (key < prev && key > best) best = key;
+          }
+        } else {
+          for (int c = lane; c < c_t; c += 32) {
+            const uint64_t key = block_key(row[c], c);
+            if (key >= tau && key < prev && key > best) best = key;
+          }
         }
-      } else {
-        for (int c = lane; c < c_t; c += 32) {
-          const uint64_t key = block_key(row[c], c);
-          if (key >= tau && key < prev && key > best) best = key;
-        }
+        best = warp_max_u64(best);
+        if (lane == s) mine = key_block(best);
+        prev = best;
       }
-      best = warp_max_u64(best);
-      if (lane == s) mine = key_block(best);
-      prev = best;
     }
   }
   if (lane == need) mine = c_t;
