@@ -54,13 +54,14 @@ def counts(w: Workload) -> dict:
     vis_keys = float(B * np.sum(t + 1))
     sel_blocks = float(B * np.sum(ksel))           # per group
     index_flops = 2.0 * w.index_dim * w.num_kv_heads * vis_keys
-    main_flops = 4.0 * w.head_dim * w.num_q_heads * w.block_size * sel_blocks
+    main_flops = 4.0 * w.head_dim * w.num_q_heads * w.block_size * sel_blocks  # S and P V
     esz = 4 if w.dtype == "f32" else 2
     kidx_bytes = float(B * w.kv_len * w.index_dim * (1 if w.index_dtype == "fp8" else esz))
     bmax_read = float(B * w.num_kv_heads * np.sum(c_t) * 4)
     partial_bytes = float(w.num_q_heads * sel_blocks * (w.head_dim * esz + 4))
     out_bytes = float(w.rows * w.num_q_heads * w.head_dim * esz)
     return {"index_flops": index_flops, "main_flops": main_flops, "kidx_bytes": kidx_bytes,
+            "index_fp8": w.index_dtype == "fp8", "qk_fp8": w.qk_dtype == "fp8",
             "bmax_read_bytes": bmax_read, "partial_bytes": partial_bytes,
             "out_bytes": out_bytes, "sel_blocks_per_group": sel_blocks,
             "q2k_bytes": float(w.num_kv_heads * w.rows * w.top_k * 4)}
@@ -75,7 +76,7 @@ def selected_kv_bytes(w: Workload, q2k: torch.Tensor) -> float:
     key = key[q2k >= 0]
     n = int(torch.unique(key).numel())
     esz = 4 if w.dtype == "f32" else 2
-    return float(n) * w.block_size * w.head_dim * esz * 2
+    return float(n) * w.block_size * w.head_dim * ((1 if w.qk_dtype == "fp8" else esz) + esz)
 
 
 def load_peaks() -> tuple:
@@ -320,21 +321,37 @@ def measured_traffic(stage: str, workload: str):
     return ent[3]
 
 
+FP8_RATIO = 2.0  # nominal dense fp8 : bf16 tensor throughput (4.5 : 2.25 PFLOP/s)
+
+
+def tensor_seconds(cnt, bf16_tflops):
+    """Time of the step's contractions at the tensor peak of each one's dtype:
+    the index GEMM, S = Q K^T (half of the main FLOPs) and P V (bf16)."""
+    r_idx = FP8_RATIO if cnt["index_fp8"] else 1.0
+    r_qk = FP8_RATIO if cnt["qk_fp8"] else 1.0
+    half = cnt["main_flops"] / 2
+    return {"index": cnt["index_flops"] / (bf16_tflops * r_idx * 1e12),
+            "attn": half / (bf16_tflops * r_qk * 1e12) + half / (bf16_tflops * 1e12)}
+
+
 def kernel_roofline(w, cnt, stage_ms, path, peaks, kv_sel_bytes, sustained=True):
-    """Roofline entry of the slowest stage of the step."""
+    """Roofline entry of the slowest stage of the step.  A contraction's peak is
+    its dtype's: the measured bf16 peak, times the nominal fp8 ratio for fp8
+    operands (the attention mixes an fp8 S with a bf16 P V when q/k are fp8)."""
     name = max(stage_ms, key=stage_ms.get)
     ms = stage_ms[name]
     tflops_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    t_peak = tensor_seconds(cnt, tflops_peak)
     alu_peak = SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
     if name == "index":
         tc = "index:tc" in path
         bound, unit, work = ("tensor" if tc else "alu"), "TFLOP/s", cnt["index_flops"]
-        peak = tflops_peak if tc else alu_peak
+        peak = work / t_peak["index"] / 1e12 if tc else alu_peak
         achieved = work / (ms * 1e-3) / 1e12
     elif name == "attn":
         tc = "attn:tc" in path
         bound, unit, work = ("tensor" if tc else "alu"), "TFLOP/s", cnt["main_flops"]
-        peak = tflops_peak if tc else alu_peak
+        peak = work / t_peak["attn"] / 1e12 if tc else alu_peak
         achieved = work / (ms * 1e-3) / 1e12
     else:
         bound, unit = "hbm", "GB/s"
@@ -343,11 +360,13 @@ def kernel_roofline(w, cnt, stage_ms, path, peaks, kv_sel_bytes, sustained=True)
                 "combine": cnt["partial_bytes"] + cnt["out_bytes"] + cnt["q2k_bytes"]}[name]
         peak = peaks["hbm_gbs"]
         achieved = work / (ms * 1e-3) / 1e9
-    return {"kernel": name, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+    return {"kernel": name, "bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 2),
             "unit": unit, "frac": round(achieved / peak, 4),
             "traffic": measured_traffic(name, w.name),
             "ms": round(ms, 4), "algorithmic_per_launch": work,
-            "peak_kind": "sustained" if (bound == "tensor" and sustained) else
+            "peak_kind": ("sustained" + (" bf16 x 2 for fp8 operands" if
+                                         (cnt["index_fp8"] or cnt["qk_fp8"]) else ""))
+                         if (bound == "tensor" and sustained) else
                          ("derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock" if bound == "alu"
                           else "measured")}
 
@@ -355,14 +374,15 @@ def kernel_roofline(w, cnt, stage_ms, path, peaks, kv_sel_bytes, sustained=True)
 def path_roofline(cnt, kv_sel_bytes, ms, peaks):
     F = cnt["index_flops"] + cnt["main_flops"]
     Bytes = cnt["kidx_bytes"] + kv_sel_bytes
-    t_tensor = F / (peaks["bf16_tflops"] * 1e12)
+    t_tensor = sum(tensor_seconds(cnt, peaks["bf16_tflops"]).values())
     t_hbm = Bytes / (peaks["hbm_gbs"] * 1e9)
     t_roof = max(t_tensor, t_hbm)
     return {"flops": F, "bytes": Bytes, "bound": "tensor" if t_tensor >= t_hbm else "hbm",
             "t_roofline_ms": round(t_roof * 1e3, 4), "t_measured_ms": round(ms, 4),
             "frac": round(t_roof * 1e3 / ms, 4),
-            "note": "roofline = max(index+main FLOPs / bf16 burst peak, (k_idx + distinct "
-                    "selected K/V bytes) / HBM peak)"}
+            "note": "roofline = max(index+main FLOPs at the burst tensor peak of their "
+                    "dtype (bf16 measured, fp8 = 2 x bf16), (k_idx + distinct selected K/V "
+                    "bytes) / HBM peak)"}
 
 
 def measure_workload(msa, w, dev, steps, warmup, peaks, with_e2e):
@@ -371,7 +391,7 @@ def measure_workload(msa, w, dev, steps, warmup, peaks, with_e2e):
     p = msa.problem_of(w)
     path = msa.kernel_path(p)
     ws = msa.new_workspace(p, msa.OP_FORWARD, dev)
-    out = torch.empty_like(x["q"])
+    out = torch.empty(x["q"].shape, dtype=x["v"].dtype, device=dev)  # out has v's dtype
     _, q2k = msa.forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], q_pos0=w.q_pos0,
                          block_size=w.block_size, top_k=w.top_k, workspace=ws, return_q2k=True)
     kv_sel = selected_kv_bytes(w, q2k)
@@ -386,7 +406,7 @@ def measure_workload(msa, w, dev, steps, warmup, peaks, with_e2e):
         xh = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "q_idx", "k_idx")}
         del ws
         torch.cuda.empty_cache()
-        out_h = torch.empty(x["q"].shape, dtype=x["q"].dtype).pin_memory()
+        out_h = torch.empty(x["q"].shape, dtype=x["v"].dtype).pin_memory()
         e_ms, h2d, d2h = run_e2e(msa, w, xh, out_h, max(1, steps // 2), 1)
         res["e2e"] = (e_ms, h2d, d2h)
     return res
@@ -425,6 +445,7 @@ def weak_value(rows_per_rank: int, ms_local: float, world: int) -> tuple:
 
 def workload_config(w: Workload, world: int) -> dict:
     return {"workload": w.name, "index_dtype": w.index_dtype or w.dtype,
+            "qk_dtype": w.qk_dtype or w.dtype,
             "batch": w.batch, "q_len": w.q_len, "kv_len": w.kv_len,
             "q_pos0": w.q_pos0, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "index_dim": w.index_dim, "block_size": w.block_size,
@@ -453,6 +474,8 @@ def main():
                          "e.g. for profiling); needles scale with the length")
     ap.add_argument("--index-dtype", default="", choices=["", "fp8"],
                     help="fp8: q_idx and k_idx in fp8 e4m3 (bf16 workloads)")
+    ap.add_argument("--qk-dtype", default="", choices=["", "fp8"],
+                    help="fp8: the main branch's q and k in fp8 e4m3, v bf16 (bf16 workloads)")
     ap.add_argument("--batch", type=int, default=0,
                     help="batch override (a smaller case of the same structure, e.g. for "
                          "profiling); needles per sequence are kept")
@@ -466,8 +489,9 @@ def main():
             raise SystemExit("--seq applies to the prefill workloads")
         w = w.with_(name=f"{w.name}@{a.seq}", q_len=a.seq, kv_len=a.seq,
                     needles=max(1, w.needles * a.seq // w.q_len))
-    if a.index_dtype:
-        w = w.with_(name=f"{w.name}+idx_{a.index_dtype}", index_dtype=a.index_dtype)
+    suffix = (f"+idx_{a.index_dtype}" if a.index_dtype else "") + \
+        (f"+qk_{a.qk_dtype}" if a.qk_dtype else "")
+    w = w.with_(name=w.name + suffix, index_dtype=a.index_dtype, qk_dtype=a.qk_dtype)
     if a.batch:
         w = w.with_(name=f"{w.name}@b{a.batch}", batch=a.batch)
     peaks, peak_src = load_peaks()
@@ -533,7 +557,8 @@ def main():
                        "ms_per_step": e_ms}
     x_main = main_res.pop("x")
     if not a.no_decode:
-        wd = WORKLOADS["decode_128k"].with_(index_dtype=a.index_dtype)
+        wd = WORKLOADS["decode_128k"]
+        wd = wd.with_(name=wd.name + suffix, index_dtype=a.index_dtype, qk_dtype=a.qk_dtype)
         del x_main
         torch.cuda.empty_cache()
         dres = measure_workload(msa, wd, dev, a.steps, a.warmup, peaks, False)

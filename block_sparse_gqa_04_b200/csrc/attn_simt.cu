@@ -5,7 +5,8 @@
 // the softmax over that block's visible tokens is complete inside the tile, so
 // the kernel writes the normalised partial output and its base-2 log-normaliser
 // and the combine kernel merges the slots.  Used for fp32 problems and for the
-// shapes the tensor-core kernel does not cover.
+// shapes the tensor-core kernel does not cover.  With fp8 (e4m3) q and k the
+// scores are formed from those values (widened exactly to fp32); v stays bf16.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,17 +23,18 @@ __device__ __forceinline__ long long find_list(const int32_t* __restrict__ tile_
   return lo;
 }
 
-template <typename T, typename PT, int D>
-__global__ void __launch_bounds__(128) attn_simt_kernel(Problem P, const T* __restrict__ q,
-                                                        const T* __restrict__ k,
-                                                        const T* __restrict__ v, Lists L,
+// TQ: element type of q and k (the scores q . k), TV: of v.
+template <typename TQ, typename TV, typename PT, int D>
+__global__ void __launch_bounds__(128) attn_simt_kernel(Problem P, const TQ* __restrict__ q,
+                                                        const TQ* __restrict__ k,
+                                                        const TV* __restrict__ v, Lists L,
                                                         PT* __restrict__ part_o,
                                                         float* __restrict__ part_lse) {
   constexpr int EPL = D / 32;  // elements per lane
   extern __shared__ unsigned char smem_raw[];
-  T* ks = reinterpret_cast<T*>(smem_raw);          // [Bk][D]
-  T* vs = ks + 128 * D;                            // [Bk][D]
-  float* sc = reinterpret_cast<float*>(vs + 128 * D);  // [4 warps][Bk]
+  TQ* ks = reinterpret_cast<TQ*>(smem_raw);                        // [Bk][D]
+  TV* vs = reinterpret_cast<TV*>(smem_raw + 128 * D * sizeof(TQ));  // [Bk][D]
+  float* sc = reinterpret_cast<float*>(vs + 128 * D);              // [4 warps][Bk]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int total_tiles = L.tile_off[P.nlists];
   const float scale_log2 = P.scale * 1.4426950408889634f;
@@ -63,11 +65,11 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(Problem P, const T* __re
       const long long t = P.q_pos0 + r % P.Sq;
       const int jn = (int)min((long long)nkeys, t - j0 + 1);
       float qv[EPL];
-      load_vec<T, EPL>(q + ((long long)r * P.Hq + h) * D + lane * EPL, qv);
+      load_vec<TQ, EPL>(q + ((long long)r * P.Hq + h) * D + lane * EPL, qv);
       float m = -INFINITY;
       for (int j = 0; j < jn; ++j) {
         float kv[EPL];
-        load_vec<T, EPL>(ks + j * D + lane * EPL, kv);
+        load_vec<TQ, EPL>(ks + j * D + lane * EPL, kv);
         float acc = 0.f;
 #pragma unroll
         for (int x = 0; x < EPL; ++x) acc = fmaf(qv[x], kv[x], acc);
@@ -84,7 +86,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(Problem P, const T* __re
         const float p = exp2f(s[j] - m);
         l += p;
         float vv[EPL];
-        load_vec<T, EPL>(vs + j * D + lane * EPL, vv);
+        load_vec<TV, EPL>(vs + j * D + lane * EPL, vv);
 #pragma unroll
         for (int x = 0; x < EPL; ++x) o[x] = fmaf(p, vv[x], o[x]);
       }
@@ -99,27 +101,33 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(Problem P, const T* __re
   }
 }
 
-template <typename T, typename PT, int D>
+template <typename TQ, typename TV, typename PT, int D>
 static cudaError_t launch_t(const Problem& P, const void* q, const void* k, const void* v,
                             const Lists& L, const Partials& part, cudaStream_t s) {
-  size_t smem = 2 * 128 * D * sizeof(T) + 4 * 128 * sizeof(float);
-  auto kern = attn_simt_kernel<T, PT, D>;
+  size_t smem = 128 * D * (sizeof(TQ) + sizeof(TV)) + 4 * 128 * sizeof(float);
+  auto kern = attn_simt_kernel<TQ, TV, PT, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<148 * 4, 128, smem, s>>>(P, (const T*)q, (const T*)k, (const T*)v, L,
+  kern<<<148 * 4, 128, smem, s>>>(P, (const TQ*)q, (const TQ*)k, (const TV*)v, L,
                                   (PT*)part.o, part.lse2);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_simt(const Problem& P, const void* q, const void* k, const void* v,
                              const Lists& L, const Partials& part, cudaStream_t s) {
+  using bf16 = __nv_bfloat16;
+  using fp8 = __nv_fp8_e4m3;
   if (P.f32) {
-    return P.D == 64 ? launch_t<float, float, 64>(P, q, k, v, L, part, s)
-                     : launch_t<float, float, 128>(P, q, k, v, L, part, s);
+    return P.D == 64 ? launch_t<float, float, float, 64>(P, q, k, v, L, part, s)
+                     : launch_t<float, float, float, 128>(P, q, k, v, L, part, s);
   }
-  return P.D == 64 ? launch_t<__nv_bfloat16, __nv_bfloat16, 64>(P, q, k, v, L, part, s)
-                   : launch_t<__nv_bfloat16, __nv_bfloat16, 128>(P, q, k, v, L, part, s);
+  if (P.qk8) {
+    return P.D == 64 ? launch_t<fp8, bf16, bf16, 64>(P, q, k, v, L, part, s)
+                     : launch_t<fp8, bf16, bf16, 128>(P, q, k, v, L, part, s);
+  }
+  return P.D == 64 ? launch_t<bf16, bf16, bf16, 64>(P, q, k, v, L, part, s)
+                   : launch_t<bf16, bf16, bf16, 128>(P, q, k, v, L, part, s);
 }
 
 }  // namespace msa

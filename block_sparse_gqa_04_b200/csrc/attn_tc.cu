@@ -29,6 +29,14 @@
 // issued as soon as its previous P V has completed, so it overlaps the
 // previous tile's epilogue.  Each softmax thread holds its whole S row (and
 // later its O row) in registers, so a tile costs one TMEM round trip each.
+//
+// With fp8 (e4m3) q and k (aiforradalom.online "Elérhetőség": the inference
+// kernels come in BF16 and FP8 among others) the score product S = Q K^T runs as
+// kind::f8f6f4 MMAs on 128-byte rows (K = 32 per instruction) and P V stays
+// bf16.  A query's Q rows are then 2 KB (one 2D box of 16 rows), a Q stage 16 KB,
+// so four stages fit, and each stage is released as soon as its S product has
+// completed; the output rows are staged in a separate 32 KB area per softmax
+// warpgroup instead of the tile's Q stage.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -42,15 +50,26 @@ namespace {
 
 constexpr int kThreads = 320;                 // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
 constexpr int kRows = 128;
-constexpr int kQBytes = kRows * 128 * 2;      // 32 KB: 128 rows x 128 dims
-constexpr int kQHalf = kQBytes / 2;           // one 64-dim half
-constexpr int kKVBytes = 2 * kQBytes;         // K then V
-constexpr int kQStages = 3;
+constexpr int kTileBytes = kRows * 128 * 2;   // 32 KB: 128 rows x 128 dims of bf16
+constexpr int kHalf = kTileBytes / 2;         // one 64-dim half of a bf16 tile
+constexpr int kMaxQStages = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kIdescS = tc::idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t kIdescO = tc::idesc_bf16_f32(128, 128, 0, 1);  // V is MN-major
 constexpr int kGroup = 16;                    // query heads per group
 constexpr int kQPerTile = kRows / kGroup;     // 8 gathered queries
+
+// Buffer plan by the element type of q and k (v is bf16 either way).
+template <bool QK8>
+struct Cfg {
+  static constexpr int kQBox = QK8 ? 2048 : 4096;          // one query's 16 head rows
+  static constexpr int kQStageBytes = kQPerTile * kQBox;   // 16 or 32 KB
+  static constexpr int kQStages = QK8 ? 4 : 3;
+  static constexpr int kKBytes = QK8 ? 16384 : kTileBytes; // 128 keys x 128 dims
+  static constexpr int kKVBytes = kKBytes + kTileBytes;    // K then V
+  static constexpr int kOStageBytes = QK8 ? kTileBytes : 0;  // per warpgroup (else the Q stage)
+  static constexpr uint32_t kIdescS =
+      QK8 ? tc::idesc_e4m3_f32(128, 128) : tc::idesc_bf16_f32(128, 128, 0, 0);
+};
 
 // Tiles are dealt to CTAs block-cyclically in chunks of kChunk consecutive
 // tiles: chunk k goes to CTA k % grid.  Consecutive tiles of a list stay on
@@ -68,7 +87,7 @@ struct TileDesc {
 
 struct Bars {
   uint64_t kv_full[2], kv_empty[2];
-  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t q_full[kMaxQStages], q_empty[kMaxQStages];
   uint64_t s_full[2], p_full[2], o_full[2], buf_empty[2];
   uint64_t d_full[kDesc], d_empty[kDesc];
   TileDesc desc[kDesc];
@@ -76,7 +95,14 @@ struct Bars {
   int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 + kQStages * kQBytes + 2 * kKVBytes + sizeof(Bars) + 64;
+template <bool QK8>
+constexpr size_t smem_bytes() {
+  using C = Cfg<QK8>;
+  return 1024 + C::kQStages * C::kQStageBytes + 2 * C::kKVBytes + 2 * C::kOStageBytes +
+         sizeof(Bars) + 64;
+}
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448,
+              "shared memory of one CTA");
 
 // The j-th tile of this CTA.
 __device__ __forceinline__ long long tile_of(int j) {
@@ -151,6 +177,7 @@ __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t p) {
   return (uint64_t(p & 0xffff0000u) << 32) | uint64_t(p << 16);
 }
 
+template <bool QK8>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                const __grid_constant__ CUtensorMap tmap_k,
@@ -158,19 +185,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                const __grid_constant__ CUtensorMap tmap_o32,
                const __grid_constant__ CUtensorMap tmap_o16, Problem P, Lists L,
                float* __restrict__ part_lse, int* __restrict__ status) {
+  using C = Cfg<QK8>;
+  constexpr int kQStages = C::kQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qbuf = smem;                          // [3][32 KB]: Q, then output staging
-  uint8_t* kvbuf = qbuf + kQStages * kQBytes;    // [2][K 32 KB | V 32 KB]
-  Bars* bars = reinterpret_cast<Bars*>(kvbuf + 2 * kKVBytes);
+  uint8_t* qbuf = smem;                                  // [stages]: Q (bf16: then output staging)
+  uint8_t* kvbuf = qbuf + kQStages * C::kQStageBytes;    // [2][K | V 32 KB]
+  uint8_t* obuf = kvbuf + 2 * C::kKVBytes;               // fp8 q/k: [2][32 KB] output staging
+  Bars* bars = reinterpret_cast<Bars*>(obuf + 2 * C::kOStageBytes);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
       tc::mbar_init(&bars->q_full[s], 1);
-      tc::mbar_init(&bars->q_empty[s], 4);  // the four warps that stored the tile
+      // bf16: the four warps that stored the tile from it; fp8: the S MMAs' commit
+      tc::mbar_init(&bars->q_empty[s], QK8 ? 1 : 4);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->kv_full[s], 1);
@@ -253,17 +284,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             good = tc::mbar_wait(&bars->kv_empty[kv_stage], kv_phase ^ 1, abort);
             if (good) {
               uint64_t* fb = &bars->kv_full[kv_stage];
-              tc::mbar_arrive_expect_tx(fb, kKVBytes);
-              uint8_t* dst = kvbuf + kv_stage * kKVBytes;
+              tc::mbar_arrive_expect_tx(fb, C::kKVBytes);
+              uint8_t* dst = kvbuf + kv_stage * C::kKVBytes;
               const int key0 = tb * P.Skv + tc_ * P.Bk;
-              tc::tma_load_3d(dst, &tmap_k, fb, 0, tg, key0);
-              tc::tma_load_3d(dst + kQHalf, &tmap_k, fb, 64, tg, key0);
-              tc::tma_load_3d(dst + kQBytes, &tmap_v, fb, 0, tg, key0);
-              tc::tma_load_3d(dst + kQBytes + kQHalf, &tmap_v, fb, 64, tg, key0);
+              tc::tma_load_3d(dst, &tmap_k, fb, 0, tg, key0);  // fp8: all 128 dims
+              if (!QK8) tc::tma_load_3d(dst + kHalf, &tmap_k, fb, 64, tg, key0);
+              tc::tma_load_3d(dst + C::kKBytes, &tmap_v, fb, 0, tg, key0);
+              tc::tma_load_3d(dst + C::kKBytes + kHalf, &tmap_v, fb, 64, tg, key0);
             }
           }
           good = good && tc::mbar_wait(&bars->q_empty[q_stage], q_phase ^ 1, abort);
-          if (good) tc::mbar_arrive_expect_tx(&bars->q_full[q_stage], uint32_t(tn) * 2 * kGroup * 128);
+          if (good) tc::mbar_arrive_expect_tx(&bars->q_full[q_stage], uint32_t(tn) * C::kQBox);
         }
         // the Q boxes of the tile, issued together: lane e copies query e
         if (__shfl_sync(MSA_FULL_MASK, good, 0) && lane < tn) {
@@ -271,11 +302,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
           int qr = trow[0];
 #pragma unroll
           for (int x = 1; x < kQPerTile; ++x) qr = e == x ? trow[x] : qr;
-          // one box: the query's 16 heads as two 8-row groups, each group's two
-          // 64-dim halves adjacent (1 KB each, 128-byte swizzle)
-          tc::tma_load_4d_hint(qbuf + q_stage * kQBytes + e * (kGroup * 256), &tmap_q,
-                               &bars->q_full[q_stage], 0, 0, 0, (qr * P.Hq + tg * kGroup) >> 3,
-                               q_policy);
+          if (QK8) {
+            // one box: the query's 16 heads as 16 rows of 128 fp8 dims (2 KB)
+            tc::tma_load_2d_hint(qbuf + q_stage * C::kQStageBytes + e * C::kQBox, &tmap_q,
+                                 &bars->q_full[q_stage], 0, qr * P.Hq + tg * kGroup, q_policy);
+          } else {
+            // one box: the query's 16 heads as two 8-row groups, each group's two
+            // 64-dim halves adjacent (1 KB each, 128-byte swizzle)
+            tc::tma_load_4d_hint(qbuf + q_stage * C::kQStageBytes + e * C::kQBox, &tmap_q,
+                                 &bars->q_full[q_stage], 0, 0, 0,
+                                 (qr * P.Hq + tg * kGroup) >> 3, q_policy);
+          }
         }
         if (lane == 0) {
           const int d = jt % kDesc;
@@ -324,11 +361,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
           const int buf = np & 1, d = np % kDesc;
           const int flags = bars->desc[d].flags;
           const int kvs = flags >> 2;
-          const uint32_t va = tc::smem_addr(kvbuf + kvs * kKVBytes + kQBytes);
+          const uint32_t va = tc::smem_addr(kvbuf + kvs * C::kKVBytes + C::kKBytes);
           const uint32_t o = tmem + buf * 256 + 128;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            tc::mma_ts(o, tmem + buf * 256 + kk * 8, tc::sdesc_sw128(va + kk * 2048, kQHalf, 1024),
+            tc::mma_ts(o, tmem + buf * 256 + kk * 8, tc::sdesc_sw128(va + kk * 2048, kHalf, 1024),
                        kIdescO, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&bars->o_full[buf]);
@@ -351,18 +388,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             if (!(sgot & 8) && tc::mbar_poll(&bars->o_full[buf], ((ns >> 1) & 1) ^ 1)) sgot |= 8;
             if (sgot == 15) {
               tc::tc_fence_after();
-              const uint32_t qa = tc::smem_addr(qbuf + qs * kQBytes);
-              const uint32_t ka = tc::smem_addr(kvbuf + kvs * kKVBytes);
+              const uint32_t qa = tc::smem_addr(qbuf + qs * C::kQStageBytes);
+              const uint32_t ka = tc::smem_addr(kvbuf + kvs * C::kKVBytes);
               const uint32_t dt = tmem + buf * 256;
+              if (QK8) {
+                // fp8: 128-byte rows of 128 dims, K = 32 per MMA
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * kQHalf + (kk & 3) * 32;
-                // Q: 8-row groups 2 KB apart, the 64-dim halves 1 KB apart inside
-                const uint32_t qoff = (kk >> 2) * 1024 + (kk & 3) * 32;
-                tc::mma_ss(dt, tc::sdesc_sw128(qa + qoff, 16, 2048),
-                           tc::sdesc_sw128(ka + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk)
+                  tc::mma_ss_f8(dt, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
+                                tc::sdesc_sw128(ka + kk * 32, 16, 1024), C::kIdescS,
+                                kk > 0 ? 1u : 0u);
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                  // Q: 8-row groups 2 KB apart, the 64-dim halves 1 KB apart inside
+                  const uint32_t qoff = (kk >> 2) * 1024 + (kk & 3) * 32;
+                  tc::mma_ss(dt, tc::sdesc_sw128(qa + qoff, 16, 2048),
+                             tc::sdesc_sw128(ka + off, 16, 1024), C::kIdescS, kk > 0 ? 1u : 0u);
+                }
               }
               tc::mma_commit(&bars->s_full[buf]);
+              if (QK8) tc::mma_commit(&bars->q_empty[qs]);  // the Q stage is read
               if (flags & 1) kv_phase[kvs] ^= 1;
               sgot = 0;
               ++ns;
@@ -442,12 +489,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       if (lane == 0) tc::mbar_arrive(&bars->p_full[wg]);
       if (!warp_wait(&bars->o_full[wg], par, abort)) { failed = true; break; }
       tc::tc_fence_after();
-      // Stage the normalised bf16 O row in this tile's Q buffer (S is done with
-      // it).  Each warp owns 32 consecutive rows (two gathered queries,
-      // contiguous in the entry-ordered partial states) and stores them itself
-      // with TMA.  The staging uses the 128-byte swizzle (16-byte chunk k of a
-      // row goes to chunk k ^ (row % 8)), which the TMA store undoes.
-      uint8_t* wst = qbuf + qs * kQBytes + quarter * 8192;
+      // Stage the normalised bf16 O row in this tile's Q buffer (bf16 q/k: S is
+      // done with it) or in the warpgroup's staging area (fp8 q/k).  Each warp
+      // owns 32 consecutive rows (two gathered queries, contiguous in the
+      // entry-ordered partial states) and stores them itself with TMA.  The
+      // staging uses the 128-byte swizzle (16-byte chunk k of a row goes to
+      // chunk k ^ (row % 8)), which the TMA store undoes.
+      uint8_t* wst = QK8 ? obuf + wg * C::kOStageBytes + quarter * 8192
+                         : qbuf + qs * C::kQStageBytes + quarter * 8192;
+      if (QK8) {
+        // this warp's previous store from the area must have read it
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        __syncwarp();
+      }
       const float inv = 1.f / l;
       const uint64_t invx2 = f2(inv, inv);
       uint32_t o[4][32];
@@ -485,10 +539,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
           for (int h = 0; h < 2; ++h) tc::tma_store_2d_hint(map, wst + h * 4096, 64 * h, grow, o_policy);
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          if (!QK8) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
-        // the Q buffer may be refilled once the store has read it
-        tc::mbar_arrive(&bars->q_empty[qs]);
+        // bf16: the Q buffer may be refilled once the store has read it
+        if (!QK8) tc::mbar_arrive(&bars->q_empty[qs]);
         tc::mbar_arrive(&bars->d_empty[d]);
       }
     }
@@ -543,27 +597,43 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap mq, mk, mv, mo32, mo16;
-  {
+  const CUtensorMapDataType qk_type =
+      P.qk8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint64_t qk_row = P.qk8 ? 128 : 256;  // bytes of one 128-dim row of q or k
+  if (P.qk8) {
+    // Q rows (token, head) of 128 fp8 dims: one 16-row box per gathered query
+    cuuint64_t dims[2] = {128, cuuint64_t(P.T) * P.Hq};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {128, kGroup};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&mq, qk_type, 2, const_cast<void*>(q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
     // Q rows (token, head) of 128 dims viewed as (64 dims, 8 rows, 2 halves, row groups)
     cuuint64_t dims[4] = {64, 8, 2, cuuint64_t(P.T) * P.Hq / 8};
     cuuint64_t strides[3] = {128 * 2, 64 * 2, 8 * 128 * 2};
     cuuint32_t box[4] = {64, 8, 2, kGroup / 8};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    if (enc(&mq, qk_type, 4, const_cast<void*>(q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   {
+    // K (fp8: one 128-byte box row per key) and V (bf16: two 64-dim halves)
     cuuint64_t dims[3] = {128, cuuint64_t(P.Hkv), cuuint64_t(P.B) * P.Skv};
-    cuuint64_t strides[2] = {128 * 2, cuuint64_t(P.Hkv) * 128 * 2};
-    cuuint32_t box[3] = {64, 1, 128};
+    cuuint64_t kstr[2] = {qk_row, cuuint64_t(P.Hkv) * qk_row};
+    cuuint64_t vstr[2] = {128 * 2, cuuint64_t(P.Hkv) * 128 * 2};
+    cuuint32_t kbox[3] = {P.qk8 ? 128u : 64u, 1, 128};
+    cuuint32_t vbox[3] = {64, 1, 128};
     cuuint32_t estr[3] = {1, 1, 1};
-    if (enc(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    if (enc(&mk, qk_type, 3, const_cast<void*>(k), dims, kstr, kbox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
-    if (enc(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(v), dims, strides, box,
+    if (enc(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(v), dims, vstr, vbox,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
@@ -583,12 +653,12 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(kSmemBytes));
+  auto kern = P.qk8 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  const size_t smem = P.qk8 ? smem_bytes<true>() : smem_bytes<false>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<sm_count(), kThreads, kSmemBytes, s>>>(
-      mq, mk, mv, mo32, mo16, P, L, part.lse2, status);
+  kern<<<sm_count(), kThreads, smem, s>>>(mq, mk, mv, mo32, mo16, P, L, part.lse2, status);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,7 @@ struct Problem {
   float scale;      // main-branch logit scale
   bool f32;         // fp32 tensors (else bf16)
   bool idx8;        // q_idx and k_idx are fp8 e4m3 (bf16 problems)
+  bool qk8;         // q and k are fp8 e4m3, v bf16 (bf16 problems)
   long long nlists; // B * Hkv * nqc * nblk
 };
 

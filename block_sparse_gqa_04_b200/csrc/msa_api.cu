@@ -23,6 +23,8 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
   if (!p) return MSA_ERR_INVALID_ARG;
   if (p->index_dtype != 0 && !(p->index_dtype == MSA_FP8_E4M3 && p->dtype == MSA_BF16))
     return MSA_ERR_INVALID_ARG;
+  if (p->qk_dtype != 0 && !(p->qk_dtype == MSA_FP8_E4M3 && p->dtype == MSA_BF16))
+    return MSA_ERR_INVALID_ARG;
   if (p->batch < 1 || p->q_len < 0 || p->kv_len < 1 || p->q_pos0 < 0) return MSA_ERR_INVALID_ARG;
   if (p->q_pos0 + p->q_len > p->kv_len) return MSA_ERR_INVALID_ARG;
   if (p->num_kv_heads < 1 || p->num_q_heads < 1 || p->num_q_heads % p->num_kv_heads != 0)
@@ -60,6 +62,7 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
   P->scale = p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / sqrtf((float)p->head_dim);
   P->f32 = p->dtype == MSA_F32;
   P->idx8 = p->index_dtype == MSA_FP8_E4M3;
+  P->qk8 = p->qk_dtype == MSA_FP8_E4M3;
   P->nlists = (long long)P->B * P->Hkv * P->nqc * P->nblk;
   if (P->nlists + 1 >= (1LL << 31)) return MSA_ERR_UNSUPPORTED;
   return MSA_OK;

@@ -44,7 +44,7 @@ class Problem(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("index_dim", ctypes.c_int32),
         ("block_size", ctypes.c_int32), ("top_k", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("q_pos0", ctypes.c_int64), ("softmax_scale", ctypes.c_float),
-        ("index_dtype", ctypes.c_int32),
+        ("index_dtype", ctypes.c_int32), ("qk_dtype", ctypes.c_int32),
     ]
 
 
@@ -87,21 +87,24 @@ def load() -> ctypes.CDLL:
 
 def make_problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
                  block_size=128, top_k=16, dtype=torch.bfloat16, q_pos0=0,
-                 softmax_scale=0.0, index_dtype=None) -> Problem:
-    """dtype: torch dtype of q/k/v (fp32 or bf16); index_dtype: torch dtype of
-    q_idx/k_idx when it differs (torch.float8_e4m3fn for fp8 index tensors)."""
+                 softmax_scale=0.0, index_dtype=None, qk_dtype=None) -> Problem:
+    """dtype: torch dtype of v and out (and of every other tensor unless stated:
+    fp32 or bf16); index_dtype / qk_dtype: torch dtype of q_idx/k_idx / of q/k
+    when it differs (torch.float8_e4m3fn for fp8 tensors)."""
     fp8 = torch.float8_e4m3fn
     main = MSA_F32 if dtype == torch.float32 else MSA_BF16
     idx = MSA_FP8_E4M3 if (index_dtype == fp8 or dtype == fp8) else 0
+    qk = MSA_FP8_E4M3 if qk_dtype == fp8 else 0
     return Problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
-                   block_size, top_k, main, q_pos0, softmax_scale, idx)
+                   block_size, top_k, main, q_pos0, softmax_scale, idx, qk)
 
 
 def problem_of(w, softmax_scale: float = 0.0) -> Problem:
     """Problem of a :class:`~block_sparse_gqa_04_b200.workload.Workload`."""
     return make_problem(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
                         w.head_dim, w.index_dim, w.block_size, w.top_k, w.torch_dtype,
-                        w.q_pos0, softmax_scale, index_dtype=w.torch_index_dtype)
+                        w.q_pos0, softmax_scale, index_dtype=w.torch_index_dtype,
+                        qk_dtype=w.torch_qk_dtype)
 
 
 def workspace_size(p: Problem, op: int = OP_FORWARD) -> int:
@@ -166,10 +169,17 @@ def _require_cuda(*ts):
             raise ValueError("libmsa takes contiguous tensors")
 
 
-def _dims(q, k, q_idx=None):
+def _dims(q, k, q_idx=None, v=None, k_idx=None):
+    """Sizes from q [B, Sq, Hq, D], k [B, Skv, Hkv, D] (and q_idx [B, Sq, Hkv, d]);
+    v, k_idx and the rest must agree, or nothing is launched."""
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
     di = q_idx.shape[3] if q_idx is not None else 32
+    want = {"k": (k, (B, Skv, Hkv, D)), "v": (v, (B, Skv, Hkv, D)),
+            "q_idx": (q_idx, (B, Sq, Hkv, di)), "k_idx": (k_idx, (B, Skv, di))}
+    for name, (t, shape) in want.items():
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
     return B, Sq, Hq, D, Skv, Hkv, di
 
 
@@ -217,17 +227,28 @@ def select_static(q_idx: torch.Tensor, k_idx: torch.Tensor, q2k: torch.Tensor, *
     return q2k
 
 
+def _check_qkv_dtypes(q, k, v):
+    """q and k share one dtype; it is v's, or fp8 e4m3 with bf16 v."""
+    if k.dtype != q.dtype:
+        raise ValueError(f"q and k dtypes differ: {q.dtype} vs {k.dtype}")
+    if q.dtype != v.dtype and not (q.dtype == torch.float8_e4m3fn and v.dtype == torch.bfloat16):
+        raise ValueError(f"q/k dtype {q.dtype} with v dtype {v.dtype} is not supported")
+
+
 def attend(q, k, v, q2k, *, q_pos0: int = 0, block_size: int = 128,
            softmax_scale: float = 0.0, return_lse: bool = False,
            workspace: Optional[torch.Tensor] = None, check_device_status: bool = False):
     """Main branch over a given selection q2k [Hkv, B*Sq, top_k] (int32)."""
     _require_cuda(q, k, v, q2k)
-    B, Sq, Hq, D, Skv, Hkv, _ = _dims(q, k)
+    B, Sq, Hq, D, Skv, Hkv, _ = _dims(q, k, v=v)
     top_k = q2k.shape[2]
-    p = make_problem(B, Sq, Skv, Hq, Hkv, D, 32, block_size, top_k, q.dtype, q_pos0,
-                     softmax_scale)
+    if q2k.dtype != torch.int32 or tuple(q2k.shape[:2]) != (Hkv, B * Sq):
+        raise ValueError("q2k must be int32 [Hkv, B*Sq, top_k]")
+    _check_qkv_dtypes(q, k, v)
+    p = make_problem(B, Sq, Skv, Hq, Hkv, D, 32, block_size, top_k, v.dtype, q_pos0,
+                     softmax_scale, qk_dtype=q.dtype)
     dev = q.device
-    out = torch.empty_like(q)
+    out = torch.empty(q.shape, dtype=v.dtype, device=dev)
     lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=dev) if return_lse else None
     ws = workspace if workspace is not None else new_workspace(p, OP_ATTEND, dev)
     wp, wn = _ws_view(ws)
@@ -257,11 +278,16 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
         nb = q.is_pinned()
         q, k, v, q_idx, k_idx = (t.to(dev, non_blocking=nb) for t in (q, k, v, q_idx, k_idx))
     _require_cuda(q, k, v, q_idx, k_idx)
-    B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx)
-    p = make_problem(B, Sq, Skv, Hq, Hkv, D, di, block_size, top_k, q.dtype, q_pos0,
-                     softmax_scale, index_dtype=q_idx.dtype)
+    B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx, v=v, k_idx=k_idx)
+    _check_qkv_dtypes(q, k, v)
+    if out is not None and (out.dtype != v.dtype or tuple(out.shape) != tuple(q.shape)
+                            or not out.is_contiguous()):
+        raise ValueError(f"out must be a contiguous {tuple(q.shape)} tensor of v's dtype "
+                         f"{v.dtype}, got {tuple(out.shape)} {out.dtype}")
+    p = make_problem(B, Sq, Skv, Hq, Hkv, D, di, block_size, top_k, v.dtype, q_pos0,
+                     softmax_scale, index_dtype=q_idx.dtype, qk_dtype=q.dtype)
     dev = q.device
-    o = out if (out is not None and not host) else torch.empty_like(q)
+    o = out if (out is not None and not host) else torch.empty(q.shape, dtype=v.dtype, device=dev)
     lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=dev) if return_lse else None
     q2k = (torch.empty((Hkv, B * Sq, top_k), dtype=torch.int32, device=dev)
            if return_q2k else None)

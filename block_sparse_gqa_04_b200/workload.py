@@ -12,7 +12,9 @@ Recipe (the same for every workload):
   * each tensor is multiplied by 1 (``fp32`` workloads) or by 1/sqrt(d)
     (``bf16`` workloads, d = head_dim for Q/K/V and index_dim for the index
     tensors) and rounded once to the workload's dtype (round to nearest even; q_idx and
-    k_idx to fp8 e4m3 instead when index_dtype is "fp8");
+    k_idx to fp8 e4m3 instead when index_dtype is "fp8", Q and K when qk_dtype
+    is "fp8": the same draws, so an fp8 workload's inputs are its bf16 twin's
+    rounded to e4m3);
   * needles: for every sequence b and group g, ``needles`` distinct "past"
     blocks are drawn uniformly (``torch.randperm`` from the same generator, in
     (b, g) order) from blocks ``0 .. upper-1`` where ``upper`` is the block of
@@ -46,6 +48,7 @@ class Workload:
     dtype: str          # "f32" or "bf16"
     needles: int        # planted needle blocks per (sequence, group)
     index_dtype: str = ""  # "" (same as dtype) or "fp8" (q_idx, k_idx in fp8 e4m3)
+    qk_dtype: str = ""     # "" (same as dtype) or "fp8" (q, k in fp8 e4m3; v stays bf16)
 
     @property
     def rows(self) -> int:
@@ -62,6 +65,10 @@ class Workload:
     @property
     def torch_index_dtype(self) -> torch.dtype:
         return torch.float8_e4m3fn if self.index_dtype == "fp8" else self.torch_dtype
+
+    @property
+    def torch_qk_dtype(self) -> torch.dtype:
+        return torch.float8_e4m3fn if self.qk_dtype == "fp8" else self.torch_dtype
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -110,8 +117,8 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu") -> Dict[str, torch.Ten
     s_main = 1.0 if w.dtype == "f32" else 1.0 / math.sqrt(w.head_dim)
     s_idx = 1.0 if w.dtype == "f32" else 1.0 / math.sqrt(w.index_dim)
     B, Sq, Skv = w.batch, w.q_len, w.kv_len
-    q = _draw(gen, (B * Sq, w.num_q_heads, w.head_dim), s_main, dt)
-    k = _draw(gen, (B * Skv, w.num_kv_heads, w.head_dim), s_main, dt)
+    q = _draw(gen, (B * Sq, w.num_q_heads, w.head_dim), s_main, w.torch_qk_dtype)
+    k = _draw(gen, (B * Skv, w.num_kv_heads, w.head_dim), s_main, w.torch_qk_dtype)
     v = _draw(gen, (B * Skv, w.num_kv_heads, w.head_dim), s_main, dt)
     q_idx = _draw(gen, (B * Sq, w.num_kv_heads, w.index_dim), s_idx, w.torch_index_dtype)
     # k_idx stays fp32 until the needles are in, then is rounded once.

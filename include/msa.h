@@ -62,9 +62,10 @@ typedef enum {
   MSA_ERR_TOO_LARGE = 6      /* problem exceeds msa_select_static's scratch   */
 } msa_status_t;
 
-/* MSA_FP8_E4M3 is an index_dtype only: fp8 e4m3 index queries and keys of a bf16
- * problem ("MiniMax új eljárása ..." (aiforradalom.online), section
- * "Elérhetőség": the MSA inference kernels come in BF16, FP8, NVFP4 and FP4). */
+/* MSA_FP8_E4M3 is an index_dtype or qk_dtype only: fp8 e4m3 index queries and
+ * keys, or main-branch queries and keys, of a bf16 problem ("MiniMax új
+ * eljárása ..." (aiforradalom.online), section "Elérhetőség": the MSA inference
+ * kernels come in BF16, FP8, NVFP4 and FP4). */
 typedef enum { MSA_BF16 = 0, MSA_F32 = 1, MSA_FP8_E4M3 = 2 } msa_dtype_t;
 
 typedef enum { MSA_OP_SELECT = 0, MSA_OP_ATTEND = 1, MSA_OP_FORWARD = 2 } msa_op_t;
@@ -83,11 +84,16 @@ typedef struct {
   int32_t index_dim;      /* d of q_idx, k_idx                                 */
   int32_t block_size;     /* Bk, tokens per KV block (128)                     */
   int32_t top_k;          /* blocks kept per (query, group), local one included */
-  int32_t dtype;          /* msa_dtype_t of q, k, v, q_idx, k_idx and out      */
+  int32_t dtype;          /* msa_dtype_t of q, k, v, q_idx, k_idx and out (see
+                             index_dtype and qk_dtype for fp8 inputs)          */
   int64_t q_pos0;         /* absolute position of query row 0 of every sequence */
   float softmax_scale;    /* main-branch logit scale; 0 selects 1/sqrt(head_dim) */
   int32_t index_dtype;    /* 0: q_idx and k_idx have `dtype`; MSA_FP8_E4M3: they are
                              fp8 e4m3 (bf16 problems); other values are invalid  */
+  int32_t qk_dtype;       /* 0: q and k have `dtype`; MSA_FP8_E4M3: q and k are fp8
+                             e4m3 and the main-branch scores q . k are formed from
+                             them (bf16 problems; v, out and the partial states stay
+                             bf16); other values are invalid                      */
 } msa_problem_t;
 
 /* Bytes of workspace that `op` needs for problem `p` (0 if p is invalid).
@@ -113,7 +119,7 @@ msa_status_t msa_select(const msa_problem_t* p, const void* q_idx, const void* k
  * be visible blocks, 0 <= c <= floor(t/Bk)).  Every query head of group g
  * attends over the visible tokens of the blocks q2k[g, r, :] with softmax
  * scale p->softmax_scale (snilld.dk "Hvad er MSA i praksis": scaled
- * dot-product softmax over exactly those tokens).  Writes out (dtype of q) and,
+ * dot-product softmax over exactly those tokens).  Writes out (`dtype`) and,
  * if lse_opt is not NULL, the natural-log softmax normaliser per (row, head);
  * a row with no valid block gets zeros and -inf. */
 msa_status_t msa_attend(const msa_problem_t* p, const void* q, const void* k, const void* v,

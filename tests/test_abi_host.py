@@ -8,6 +8,7 @@ import subprocess
 import tempfile
 
 import pytest
+import torch
 
 from block_sparse_gqa_04_b200 import msa, workload
 
@@ -43,15 +44,16 @@ def test_problem_struct_layout_matches_header(tmp_path):
     src = tmp_path / "layout.c"
     src.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "msa.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu\\n\", sizeof(msa_problem_t),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu\\n\", sizeof(msa_problem_t),"
         " offsetof(msa_problem_t,q_pos0), offsetof(msa_problem_t,softmax_scale),"
-        " offsetof(msa_problem_t,index_dtype));return 0;}\n")
+        " offsetof(msa_problem_t,index_dtype), offsetof(msa_problem_t,qk_dtype));return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
                    check=True)
     got = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     P = msa.Problem
-    want = [ctypes.sizeof(P), P.q_pos0.offset, P.softmax_scale.offset, P.index_dtype.offset]
+    want = [ctypes.sizeof(P), P.q_pos0.offset, P.softmax_scale.offset, P.index_dtype.offset,
+            P.qk_dtype.offset]
     assert [int(x) for x in got] == want
 
 
@@ -78,6 +80,8 @@ def test_workspace_sizes(lib):
     ("batch", 0, 1),
     ("index_dtype", 1, 1),           # only fp8 e4m3 may differ from dtype
     ("index_dtype", 5, 1),
+    ("qk_dtype", 1, 1),              # only fp8 e4m3 may differ from dtype
+    ("qk_dtype", -2, 1),
     ("dtype", 7, 1),
 ])
 def test_invalid_problems_are_rejected_on_the_host(lib, field, value, code):
@@ -101,6 +105,34 @@ def test_index_dtype_values(lib):
     assert msa.workspace_size(t, msa.OP_FORWARD) == 0
     w8 = workload.WORKLOADS["prefill_32k"].with_(index_dtype="fp8")
     assert msa.problem_of(w8).index_dtype == msa.MSA_FP8_E4M3
+
+
+def test_qk_dtype_values(lib):
+    """fp8 e4m3 q and k are valid for bf16 problems only; v and out stay bf16."""
+    p = msa.problem_of(workload.WORKLOADS["prefill_32k"])
+    p.qk_dtype = msa.MSA_FP8_E4M3
+    fwd = msa.workspace_size(p, msa.OP_FORWARD)
+    assert fwd == msa.workspace_size(msa.problem_of(workload.WORKLOADS["prefill_32k"]),
+                                     msa.OP_FORWARD)  # bf16 partial states either way
+    t = msa.problem_of(workload.WORKLOADS["tiny"])       # an fp32 problem
+    t.qk_dtype = msa.MSA_FP8_E4M3
+    assert msa.workspace_size(t, msa.OP_FORWARD) == 0
+    w8 = workload.WORKLOADS["prefill_32k"].with_(qk_dtype="fp8")
+    assert msa.problem_of(w8).qk_dtype == msa.MSA_FP8_E4M3
+    assert msa.problem_of(w8).dtype == msa.MSA_BF16
+
+
+def test_qkv_dtype_combinations_are_checked_in_python():
+    q = torch.zeros((1, 4, 16, 128), dtype=torch.float8_e4m3fn)
+    k = torch.zeros((1, 4, 1, 128), dtype=torch.float8_e4m3fn)
+    v = torch.zeros((1, 4, 1, 128), dtype=torch.bfloat16)
+    msa._check_qkv_dtypes(q, k, v)                           # fp8 q/k with bf16 v
+    with pytest.raises(ValueError):
+        msa._check_qkv_dtypes(q, k.to(torch.bfloat16), v)    # q and k differ
+    with pytest.raises(ValueError):
+        msa._check_qkv_dtypes(q, k, v.float())               # fp8 q/k need bf16 v
+    with pytest.raises(ValueError):
+        msa._check_qkv_dtypes(q.float(), k.float(), v)       # fp32 q/k with bf16 v
 
 
 def test_null_misaligned_and_small_workspace(lib):

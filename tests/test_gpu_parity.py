@@ -40,6 +40,20 @@ SMALL = {
     "fp8_decode_rows8": Workload("fp8_decode_rows8", 2, 8, 5000, 4990, 64, 4, 128, 128, 128, 16,
                                  "bf16", 2, "fp8"),
     "fp8_di64": Workload("fp8_di64", 1, 700, 700, 0, 16, 4, 64, 64, 128, 5, "bf16", 1, "fp8"),
+    # fp8 (e4m3) q and k in the main branch (v bf16): tensor-core attention in
+    # prefill, an unaligned chunk and decode, the SIMT attention for groups of 8
+    # and head_dim 64, and fp8 index tensors together with fp8 q/k
+    "qk8_prefill": Workload("qk8_prefill", 1, 2125, 2125, 0, 64, 4, 128, 128, 128, 16, "bf16",
+                            2, "", "fp8"),
+    "qk8_chunk": Workload("qk8_chunk", 1, 300, 2000, 1700, 64, 4, 128, 128, 128, 16, "bf16", 2,
+                          "", "fp8"),
+    "qk8_decode": Workload("qk8_decode", 5, 1, 3000, 2999, 64, 4, 128, 128, 128, 16, "bf16", 3,
+                           "", "fp8"),
+    "qk8_batch_g8": Workload("qk8_batch_g8", 3, 200, 777, 577, 16, 2, 128, 128, 128, 6, "bf16",
+                             1, "", "fp8"),
+    "qk8_d64": Workload("qk8_d64", 2, 700, 700, 0, 16, 4, 64, 64, 128, 5, "bf16", 1, "", "fp8"),
+    "fp8_all": Workload("fp8_all", 2, 1100, 1100, 0, 64, 4, 128, 128, 128, 16, "bf16", 2, "fp8",
+                        "fp8"),
     "top1": Workload("top1", 1, 700, 700, 0, 32, 2, 128, 128, 128, 1, "bf16", 1),
     "d64_g4": Workload("d64_g4", 2, 700, 700, 0, 16, 4, 64, 64, 128, 5, "bf16", 1),
     "f32_d128_g8": Workload("f32_d128_g8", 1, 600, 600, 0, 16, 2, 128, 128, 128, 4, "f32", 0),
@@ -55,8 +69,11 @@ _cache = {}
 
 def _host(t: torch.Tensor):
     """Host copy for the oracle: a NumPy fp32 array when small, else the torch
-    tensor itself (the oracle then gathers only the rows it needs)."""
+    tensor itself (the oracle then gathers only the rows it needs).  fp8 e4m3
+    tensors are widened to bf16 first, which holds every e4m3 value exactly."""
     t = t.cpu()
+    if t.dtype == torch.float8_e4m3fn:
+        t = t.to(torch.bfloat16)
     return t.float().numpy() if t.numel() <= (1 << 27) else t
 
 
@@ -111,7 +128,8 @@ def test_forward_matches_oracle_sampled(name):
     _forward_parity(w, sample_rows(w, n))
 
 
-@pytest.mark.parametrize("name", ["tiny", "bf16_ragged", "batch_offset", "d64_g4"])
+@pytest.mark.parametrize("name", ["tiny", "bf16_ragged", "batch_offset", "d64_g4", "qk8_prefill",
+                                  "qk8_batch_g8"])
 def test_attend_with_oracle_selection(name):
     w = SMALL[name]
     cpu, gpu = _inputs(w)
@@ -199,11 +217,18 @@ def test_host_buffers_round_trip():
 
 FULL_SAMPLES = {"tiny": None, "prefill_32k": 48, "prefill_128k": 32, "decode_128k": None,
                 "chunk_1m": 24}
+# the 128K workloads with fp8 (e4m3) index tensors and fp8 q/k, as the bench
+# runs them with --index-dtype fp8 --qk-dtype fp8
+for _n, _r in (("prefill_128k", 16), ("decode_128k", None)):
+    FULL_SAMPLES[_n + "+fp8"] = _r
 
 
 @pytest.mark.parametrize("name", list(FULL_SAMPLES))
 def test_named_workload_full_size(name):
-    w = WORKLOADS[name]
+    base, _, fp8 = name.partition("+")
+    w = WORKLOADS[base]
+    if fp8:
+        w = w.with_(name=f"{base}_fp8", index_dtype="fp8", qk_dtype="fp8")
     n = FULL_SAMPLES[name]
     rows = None if n is None else sample_rows(w, n)
     dec, agree, und = _forward_parity(w, rows)
