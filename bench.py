@@ -534,11 +534,12 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": ("f32" if w.dtype == "f32" else
+                  "e4m3+bf16" if (w.index_dtype == "fp8" or w.qk_dtype == "fp8") else "bf16"),
         "data": "synthetic (seeded N(0,1/d) inputs with planted needle blocks)",
         "config": dict(workload_config(w, world), kernel_path=main_res["path"],
                        l2="inputs larger than L2 (q alone is %.2f GB per step)" %
-                          (main_res["x"]["q"].numel() * 2 / 1e9)),
+                          (main_res["x"]["q"].numel() * main_res["x"]["q"].element_size() / 1e9)),
         "clocks": main_res["clocks"],
         "gpu_launches": main_res["launches"],
         "stage_ms": {k: round(v, 4) for k, v in main_res["stage"].items()},
