@@ -44,6 +44,23 @@ design notes of the repository):
   R5  a row that sees fewer than top_k blocks selects all of them.
   R6  the selected ids are returned in ascending order, -1 padded.
   R7  main-branch scale is 1/sqrt(head_dim) ([DK] "scaled dot-product").
+  R17 the index branch's distribution for the KL-alignment loss is the
+      softmax of the raw token-level index scores over the same causally
+      visible tokens of the selected blocks that the main branch attends.
+  R18 the loss is KL(teacher || index) per (query row, group), the teacher
+      being the mean over the group's query heads of the main-branch softmax
+      over those tokens; the loss is the mean over all (row, group) pairs.
+  R19 gradient detach: the teacher and the selection are constants; the
+      gradients flow into q_idx and k_idx only.
+
+Additional source for the KL-alignment loss:
+  [DK]  section "Træning og stabilisering": Top-k is not differentiable, so an
+        extra KL-alignment loss trains the index projections, the index branch
+        matching the main branch's attention pattern, whose teacher is the
+        group-averaged main distribution over the selected tokens, with
+        gradient detach.
+  [HU]  section "A betanítás és a kernel-optimalizáció": a KL-divergence loss
+        aligns the Index Branch distribution to the Main Branch pattern.
 """
 from __future__ import annotations
 
@@ -248,6 +265,83 @@ def forward(q, k, v, q_idx, k_idx, q_pos0: int, block_size: int, top_k: int,
     q2k = select(q_idx, k_idx, q_pos0, block_size, top_k, rows)
     out, lse = attend(q, k, v, q2k, q_pos0, block_size, scale, rows)
     return out, lse, q2k
+
+
+# ---------------------------------------------------------------------------
+# KL-alignment loss of the index branch (training side)
+# ---------------------------------------------------------------------------
+
+def selected_tokens(blocks, t: int, block_size: int) -> np.ndarray:
+    """The causally visible tokens 0..t of the selected blocks, ascending."""
+    keys = []
+    for c in blocks:
+        if c < 0:
+            continue
+        keys.extend(range(c * block_size, min((c + 1) * block_size, t + 1)))
+    return np.array(sorted(keys), dtype=np.int64)
+
+
+def index_kl_row(q_heads, k_seq_g, q_idx_vec, k_idx_seq, blocks, t: int, block_size: int,
+                 scale: float):
+    """KL-alignment term of one (query row, group) and its score gradient.
+
+    [DK] "Træning og stabilisering": the index branch is trained to match the
+    main branch; the teacher is the group-averaged main distribution over the
+    selected tokens (readings R17-R19).  Over the tokens J of the selected
+    blocks (visible ones only):
+      index  p_I = softmax_j(q_idx . k_idx[j])                 (raw scores, R1)
+      teacher p_T = mean over the group's heads h of softmax_j(scale * q_h . k[j])
+      kl = sum_j p_T[j] * (ln p_T[j] - ln p_I[j])
+    and d kl / d s_j = p_I[j] - p_T[j].  Returns (kl, J, p_I - p_T).
+    """
+    J = selected_tokens(blocks, t, block_size)
+    s = _take(k_idx_seq, J) @ _f64(q_idx_vec)            # [n]
+    lse_i = s.max() + math.log(np.exp(s - s.max()).sum())
+    log_pi = s - lse_i
+    z = scale * (_f64(q_heads) @ _take(k_seq_g, J).T)    # [G, n]
+    a = np.exp(z - z.max(axis=1, keepdims=True))
+    a /= a.sum(axis=1, keepdims=True)
+    p_t = a.mean(axis=0)
+    pos = p_t > 0
+    kl = float(np.sum(p_t[pos] * (np.log(p_t[pos]) - log_pi[pos])))
+    return kl, J, np.exp(log_pi) - p_t
+
+
+def index_kl(q, k, q_idx, k_idx, q2k, q_pos0: int, block_size: int,
+             scale: Optional[float] = None):
+    """Mean KL-alignment loss over all (row, group) pairs and its gradients.
+
+    Returns (loss, dq_idx [B, Sq, Hkv, di], dk_idx [B, Skv, di], kl [Hkv, B*Sq]).
+    With N = B*Sq*Hkv pairs, d loss / d s = (p_I - p_T) / N for each pair's
+    tokens, so dq_idx[row, g] = sum_j ds_j k_idx[j] and dk_idx[j] collects
+    ds_j q_idx[row, g] over every (row, group) whose selection holds token j
+    (k_idx is the one index-key head shared by all groups).  q, k and the
+    selection q2k are constants (R19).  ``scale`` defaults to 1/sqrt(D) (R7).
+    """
+    B, Sq, Hq, D = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    di = q_idx.shape[3]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    sel = np.asarray(q2k)
+    N = B * Sq * Hkv
+    kl = np.zeros((Hkv, B * Sq))
+    dq = np.zeros((B, Sq, Hkv, di))
+    dk = np.zeros((B, k_idx.shape[1], di))
+    for b in range(B):
+        kis = _f64(k_idx[b])
+        for i in range(Sq):
+            r = b * Sq + i
+            t = q_pos0 + i
+            for g in range(Hkv):
+                qi = _f64(q_idx[b, i, g])
+                kl[g, r], J, ds = index_kl_row(q[b, i, g * G:(g + 1) * G], k[b, :, g], qi,
+                                               kis, sel[g, r], t, block_size, scale)
+                ds = ds / N
+                dq[b, i, g] = ds @ kis[J]
+                dk[b, J] += np.outer(ds, qi)
+    return float(kl.sum() / N), dq, dk, kl
 
 
 # ---------------------------------------------------------------------------
