@@ -301,7 +301,7 @@ def run_e2e(msa, w, xh, out_h, steps, warmup):
 NCU_TRAFFIC = {
     # stage: (workload, source file, git blob id, bytes per launch)
     "attn": ("prefill_128k", "block_sparse_gqa_04_b200/csrc/attn_tc.cu",
-             "bcf6c0a9947c62b858e686af6f4ba095906b6513", 13299131136 + 34592495360),
+             "94f2370ab0df85d8092da83eea7b8bb2f8a264f2", 14249309696 + 34591866112),
 }
 
 
@@ -458,6 +458,69 @@ def barrier(world: int):
         dist.barrier()
 
 
+def index_kl_flops(w: Workload, q2k: torch.Tensor) -> float:
+    """Algorithmic FLOPs of one msa_index_kl: per (row, group) and selected
+    visible token, the teacher's logits (G heads x D MACs), the index score and
+    its dq_idx term (2 x di MACs), and its dk_idx term (di MACs)."""
+    Hkv, T, K = q2k.shape
+    pos = (w.q_pos0 + torch.arange(T, device=q2k.device) % w.q_len).view(1, T, 1)
+    c = q2k.to(torch.int64)
+    vis = torch.clamp(pos - c * w.block_size + 1, 0, w.block_size) * (c >= 0)
+    tokens = float(vis.sum().item())
+    G = w.num_q_heads // w.num_kv_heads
+    return 2.0 * tokens * (G * w.head_dim + 3 * w.index_dim)
+
+
+def bench_index_kl(a, w, world, rank, local, peaks):
+    """Times msa_index_kl on the workload's inputs and its own selection (made
+    once, untimed): exactly a.steps calls after a.warmup, CUDA events on the
+    launching stream, max over ranks."""
+    from block_sparse_gqa_04_b200 import msa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    x = make_inputs(w, seed=rank, device=dev)
+    x.pop("needles")
+    q2k = msa.select(x["q_idx"], x["k_idx"], q_pos0=w.q_pos0, block_size=w.block_size,
+                     top_k=w.top_k)
+    p = msa.problem_of(w)
+    ws = msa.new_workspace(p, msa.OP_INDEX_KL, dev)
+    kw = dict(q_pos0=w.q_pos0, block_size=w.block_size, workspace=ws)
+    for _ in range(a.warmup):
+        msa.index_kl(x["q"], x["k"], x["q_idx"], x["k_idx"], q2k, **kw)
+    start, end = _events(2)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        start.record()
+        for _ in range(a.steps):
+            msa.index_kl(x["q"], x["k"], x["q_idx"], x["k_idx"], q2k, **kw)
+        end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end) / a.steps, world)
+    flops = index_kl_flops(w, q2k)
+    alu_peak = SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    if rank == 0:
+        line = {"metric": "index KL-alignment loss + q_idx/k_idx gradients (training side), "
+                          "query-tokens/s", "value": world * w.rows / (ms * 1e-3),
+                "unit": "query-tokens/s", "n_gpus": world, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32" if w.dtype == "f32" else "f32 (bf16/e4m3 inputs)",
+                "data": "synthetic (seeded N(0,1/d) inputs with planted needle blocks)",
+                "config": dict(workload_config(w, world),
+                               kernel_path=msa.kernel_path(p, msa.OP_INDEX_KL)),
+                "clocks": clk.summary(),
+                "gpu_launches": a.steps * msa.launch_count(p, msa.OP_INDEX_KL),
+                "roofline": {"kernel": "index_kl", "bound": "alu", "achieved": round(achieved, 2),
+                             "peak": round(alu_peak, 2), "unit": "TFLOP/s",
+                             "frac": round(achieved / alu_peak, 4), "traffic": None,
+                             "algorithmic_per_launch": flops,
+                             "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock"}}
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -476,6 +539,9 @@ def main():
                     help="fp8: q_idx and k_idx in fp8 e4m3 (bf16 workloads)")
     ap.add_argument("--qk-dtype", default="", choices=["", "fp8"],
                     help="fp8: the main branch's q and k in fp8 e4m3, v bf16 (bf16 workloads)")
+    ap.add_argument("--index-kl", action="store_true",
+                    help="time the KL-alignment loss and its index-branch gradients "
+                         "(training side, msa_index_kl) instead of the forward")
     ap.add_argument("--batch", type=int, default=0,
                     help="batch override (a smaller case of the same structure, e.g. for "
                          "profiling); needles per sequence are kept")
@@ -495,6 +561,9 @@ def main():
     if a.batch:
         w = w.with_(name=f"{w.name}@b{a.batch}", batch=a.batch)
     peaks, peak_src = load_peaks()
+
+    if a.index_kl and a.impl != "reference":
+        return bench_index_kl(a, w, world, rank, local, peaks)
 
     if a.impl == "reference":
         # the reference arm is the fp64 oracle on the host cores, rank 0 only

@@ -108,6 +108,14 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
 cudaError_t launch_combine(const Problem& P, const int32_t* pos, const Partials& part,
                            void* out, float* lse, int32_t* status, cudaStream_t s);
 
+// --- KL-alignment loss of the index branch (training side) --------------------
+bool index_kl_supported(const Problem& P);
+// kl_rows [Hkv*T] and ds_buf [Hkv*T*K*Bk] are workspace; dk_idx is overwritten.
+cudaError_t launch_index_kl(const Problem& P, const void* q, const void* k, const void* q_idx,
+                            const void* k_idx, const int32_t* q2k, const Lists& L,
+                            float* kl_rows, float* ds_buf, float* loss, float* dq_idx,
+                            float* dk_idx, int32_t* status, cudaStream_t s);
+
 // Device status bits (workspace status word): 1 = invalid q2k entry given to
 // attend, 2 = a bounded wait inside a tensor-core kernel gave up.
 constexpr int kStatusBadEntry = 1;

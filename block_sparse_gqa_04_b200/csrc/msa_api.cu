@@ -71,7 +71,7 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
 // Workspace layout (each region 256-byte aligned, in this order).
 struct Layout {
   size_t status, bmax, q2k, counts, cursor, list_off, tile_off, entries, pos, tiles, seg_sums,
-      part_o, part_lse, total;
+      part_o, part_lse, kl_rows, kl_ds, total;
 };
 
 Layout layout(const Problem& P, int op) {
@@ -83,17 +83,24 @@ Layout layout(const Problem& P, int op) {
   L.status = take(sizeof(int32_t));
   const bool sel = op == MSA_OP_SELECT || op == MSA_OP_FORWARD;
   const bool att = op == MSA_OP_ATTEND || op == MSA_OP_FORWARD;
+  const bool kl = op == MSA_OP_INDEX_KL;
   L.bmax = sel ? take(size_t(P.Hkv) * T * P.nblk * sizeof(float)) : 0;
   L.q2k = op == MSA_OP_FORWARD ? take(size_t(P.Hkv) * T * P.K * sizeof(int32_t)) : 0;
-  if (att) {
+  if (att || kl) {
     L.counts = take(size_t(P.nlists) * 4);
     L.cursor = take(size_t(P.nlists) * 4);
     L.list_off = take(size_t(P.nlists + 1) * 4);
     L.tile_off = take(size_t(P.nlists + 1) * 4);
     L.entries = take(size_t(P.Hkv) * T * P.K * 4);
     L.pos = take(size_t(P.Hkv) * T * P.K * 4);
-    L.tiles = take(size_t(msa::max_tiles(P)) * sizeof(msa::TileRec));
     L.seg_sums = take(size_t((P.nlists + 2047) / 2048) * 8);
+  }
+  if (kl) {
+    L.kl_rows = take(size_t(P.Hkv) * T * sizeof(float));
+    L.kl_ds = take(size_t(P.Hkv) * T * P.K * P.Bk * sizeof(float));
+  }
+  if (att) {
+    L.tiles = take(size_t(msa::max_tiles(P)) * sizeof(msa::TileRec));
     // one partial state per (entry, head of the group): Hkv*T*K*G = T*Hq*K rows
     L.part_o = take(T * P.Hq * P.K * size_t(P.D) * esz);
     L.part_lse = take(T * P.Hq * P.K * sizeof(float));
@@ -181,7 +188,7 @@ extern "C" {
 
 size_t msa_workspace_size(const msa_problem_t* p, int32_t op) {
   Problem P;
-  if (resolve(p, &P) != MSA_OK || op < MSA_OP_SELECT || op > MSA_OP_FORWARD) return 0;
+  if (resolve(p, &P) != MSA_OK || op < MSA_OP_SELECT || op > MSA_OP_INDEX_KL) return 0;
   return layout(P, op).total;
 }
 
@@ -247,6 +254,37 @@ msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, c
   return run_attend(P, q, k, v, q2k, out, lse_opt, ws, L, s);
 }
 
+msa_status_t msa_index_kl(const msa_problem_t* p, const void* q, const void* k,
+                          const void* q_idx, const void* k_idx, const int32_t* q2k,
+                          float* loss, float* dq_idx, float* dk_idx, void* ws, size_t ws_bytes,
+                          void* stream) {
+  Problem P;
+  msa_status_t st = resolve(p, &P);
+  if (st != MSA_OK) return st;
+  if (P.T == 0) return MSA_OK;  // no (row, group) pair: nothing to average
+  if (!msa::index_kl_supported(P)) return MSA_ERR_UNSUPPORTED;
+  if (!q || !k || !q_idx || !k_idx || !q2k || !loss || !dq_idx || !dk_idx)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_idx) || !aligned16(k_idx) ||
+      !aligned16(q2k) || !aligned16(dq_idx) || !aligned16(dk_idx) ||
+      (reinterpret_cast<uintptr_t>(loss) & 3u) != 0)
+    return MSA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, MSA_OP_INDEX_KL, ws, ws_bytes)) != MSA_OK) return st;
+  const Layout L = layout(P, MSA_OP_INDEX_KL);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  msa::Lists lists{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.cursor),
+                   at<int32_t>(ws, L.list_off), at<int32_t>(ws, L.tile_off),
+                   at<int32_t>(ws, L.entries), at<int32_t>(ws, L.pos), nullptr,
+                   at<int32_t>(ws, L.seg_sums)};
+  int32_t* status = at<int32_t>(ws, L.status);
+  cudaError_t e = msa::launch_invert(P, q2k, lists, status, s);
+  if (e == cudaSuccess)
+    e = msa::launch_index_kl(P, q, k, q_idx, k_idx, q2k, lists, at<float>(ws, L.kl_rows),
+                             at<float>(ws, L.kl_ds), loss, dq_idx, dk_idx, status, s);
+  return cuda_status(e);
+}
+
 msa_status_t msa_device_status(const void* ws, int32_t* code, void* stream) {
   if (!ws || !code) return MSA_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
@@ -277,6 +315,7 @@ int32_t msa_launch_count(const msa_problem_t* p, int32_t op) {
     case MSA_OP_SELECT: return sel;
     case MSA_OP_ATTEND: return att;
     case MSA_OP_FORWARD: return sel + att;
+    case MSA_OP_INDEX_KL: return msa::kLaunchesInvert + 3;  // lists, rows, dk, sum
   }
   return 0;
 }
@@ -294,6 +333,7 @@ const char* msa_kernel_path(const msa_problem_t* p, int32_t op) {
     case MSA_OP_SELECT: return sel[ik];
     case MSA_OP_ATTEND: return atc ? "attn:tc" : "attn:simt";
     case MSA_OP_FORWARD: return fwd[ik][atc ? 1 : 0];
+    case MSA_OP_INDEX_KL: return "kl:simt";
   }
   return "invalid";
 }

@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
 MSA_BF16, MSA_F32, MSA_FP8_E4M3 = 0, 1, 2
-OP_SELECT, OP_ATTEND, OP_FORWARD = 0, 1, 2
+OP_SELECT, OP_ATTEND, OP_FORWARD, OP_INDEX_KL = 0, 1, 2, 3
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
           3: "MSA_ERR_WORKSPACE", 4: "MSA_ERR_CUDA", 5: "MSA_ERR_DEVICE",
@@ -27,7 +27,7 @@ STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 
 EXPORTED = ("msa_workspace_size", "msa_select", "msa_attend", "msa_forward",
             "msa_device_status", "msa_set_stage_events", "msa_launch_count", "msa_kernel_path",
-            "msa_status_string", "msa_select_static")
+            "msa_status_string", "msa_select_static", "msa_index_kl")
 STAGES = ("index", "topk", "lists", "attn", "combine")
 
 
@@ -81,6 +81,8 @@ def load() -> ctypes.CDLL:
         lib.msa_status_string.restype = ctypes.c_char_p
         lib.msa_select_static.argtypes = [pp, vp, vp, vp, vp, vp]
         lib.msa_select_static.restype = i32
+        lib.msa_index_kl.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.msa_index_kl.restype = i32
         _lib = lib
     return _lib
 
@@ -259,6 +261,41 @@ def attend(q, k, v, q2k, *, q_pos0: int = 0, block_size: int = 128,
         _check(load().msa_device_status(ctypes.c_void_p(wp), ctypes.byref(code), _stream(dev)),
                "msa_attend (device status)")
     return (out, lse) if return_lse else out
+
+
+def index_kl(q, k, q_idx, k_idx, q2k, *, q_pos0: int = 0, block_size: int = 128,
+             softmax_scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+             check_device_status: bool = False):
+    """KL-alignment loss of the index branch and its gradients (training side).
+
+    The selection q2k [Hkv, B*Sq, top_k] (int32, as :func:`select` returns it)
+    and the teacher, from q and k, are constants.  Returns (loss, dq_idx, dk_idx):
+    the mean KL(teacher || index) over the (row, group) pairs as a 0-d fp32
+    tensor, and its fp32 gradients shaped like q_idx and k_idx.
+    """
+    _require_cuda(q, k, q_idx, k_idx, q2k)
+    B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx, k_idx=k_idx)
+    if q2k.dtype != torch.int32 or q2k.dim() != 3 or tuple(q2k.shape[:2]) != (Hkv, B * Sq):
+        raise ValueError("q2k must be int32 [Hkv, B*Sq, top_k]")
+    if k.dtype != q.dtype:
+        raise ValueError(f"q and k dtypes differ: {q.dtype} vs {k.dtype}")
+    main = torch.float32 if q.dtype == torch.float32 else torch.bfloat16
+    p = make_problem(B, Sq, Skv, Hq, Hkv, D, di, block_size, q2k.shape[2], main, q_pos0,
+                     softmax_scale, index_dtype=q_idx.dtype, qk_dtype=q.dtype)
+    dev = q.device
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    dq = torch.empty(q_idx.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k_idx.shape, dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else new_workspace(p, OP_INDEX_KL, dev)
+    wp, wn = _ws_view(ws)
+    _check(load().msa_index_kl(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(q_idx), _ptr(k_idx),
+                               _ptr(q2k), _ptr(loss), _ptr(dq), _ptr(dk), ctypes.c_void_p(wp),
+                               wn, _stream(dev)), "msa_index_kl")
+    if check_device_status:
+        code = ctypes.c_int32(0)
+        _check(load().msa_device_status(ctypes.c_void_p(wp), ctypes.byref(code), _stream(dev)),
+               "msa_index_kl (device status)")
+    return loss, dq, dk
 
 
 def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, top_k: int = 16,

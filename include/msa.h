@@ -68,7 +68,12 @@ typedef enum {
  * kernels come in BF16, FP8, NVFP4 and FP4). */
 typedef enum { MSA_BF16 = 0, MSA_F32 = 1, MSA_FP8_E4M3 = 2 } msa_dtype_t;
 
-typedef enum { MSA_OP_SELECT = 0, MSA_OP_ATTEND = 1, MSA_OP_FORWARD = 2 } msa_op_t;
+typedef enum {
+  MSA_OP_SELECT = 0,
+  MSA_OP_ATTEND = 1,
+  MSA_OP_FORWARD = 2,
+  MSA_OP_INDEX_KL = 3 /* msa_index_kl (training side) */
+} msa_op_t;
 
 /* One MSA problem.  Supported: block_size 128; top_k 1..32; head_dim 64 or
  * 128; index_dim 32, 64 or 128; num_q_heads a multiple of num_kv_heads with at
@@ -157,6 +162,31 @@ msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, c
  * Other arguments and errors as msa_select. */
 msa_status_t msa_select_static(const msa_problem_t* p, const void* q_idx, const void* k_idx,
                                int32_t* q2k, int32_t* device_status_opt, void* stream);
+
+/* KL-alignment loss of the index branch and its gradients (training side).
+ * snilld.dk "Træning og stabilisering": Top-k is not differentiable, so an
+ * extra KL-alignment loss trains the index projections, the index branch
+ * matching the main branch, whose group-averaged distribution over the selected
+ * tokens is the teacher, with gradient detach.  For every row r and group g,
+ * over the causally visible tokens J of the blocks q2k[g, r, :] (as msa_select
+ * writes them):
+ *   p_I = softmax_j(q_idx[r,g] . k_idx[j])                       (raw scores)
+ *   p_T = mean over the group's heads h of softmax_j(scale * q[r,h] . k[j,g])
+ *   kl  = sum_j p_T[j] (ln p_T[j] - ln p_I[j])
+ * Writes *loss (device, one float) = the mean of kl over the batch*q_len*
+ * num_kv_heads pairs, and the gradients of that mean with respect to q_idx
+ * (dq_idx, fp32, [batch, q_len, num_kv_heads, index_dim]) and k_idx (dk_idx,
+ * fp32, [batch, kv_len, index_dim], overwritten) with q, k and q2k held constant
+ * (no gradient reaches q or k).  q, k, q_idx, k_idx take the problem's dtypes
+ * (qk_dtype, index_dtype).  Workspace: msa_workspace_size(p, MSA_OP_INDEX_KL).
+ * q2k entries outside the row's visible blocks are skipped and flag the status
+ * word (1), as in msa_attend.  Runs on CUDA cores; MSA_ERR_UNSUPPORTED when the
+ * per-(row, group) working set (group heads x head_dim + 2 x top_k x 128
+ * floats) exceeds 200 KB of shared memory.  Other errors as msa_attend. */
+msa_status_t msa_index_kl(const msa_problem_t* p, const void* q, const void* k,
+                          const void* q_idx, const void* k_idx, const int32_t* q2k,
+                          float* loss, float* dq_idx, float* dk_idx, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* Reads the workspace status word written by the last call that used `ws`:
  * waits for `stream`, stores the device code (0 = fine) in *code and returns

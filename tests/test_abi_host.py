@@ -107,6 +107,27 @@ def test_index_dtype_values(lib):
     assert msa.problem_of(w8).index_dtype == msa.MSA_FP8_E4M3
 
 
+def test_index_kl_workspace_and_argument_checks(lib):
+    p = msa.problem_of(workload.WORKLOADS["prefill_32k"])
+    n = msa.workspace_size(p, msa.OP_INDEX_KL)
+    w = workload.WORKLOADS["prefill_32k"]
+    # the per-token score gradients dominate: Hkv * rows * top_k * 128 floats
+    assert n >= w.num_kv_heads * w.rows * w.top_k * w.block_size * 4
+    assert msa.workspace_size(p, 4) == 0
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected before any launch
+    st = lib.msa_index_kl(ctypes.byref(p), fake, fake, None, fake, fake, fake, fake, fake, fake,
+                          1 << 40, None)
+    assert st == 1                    # a null q_idx
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    st = lib.msa_index_kl(ctypes.byref(p), fake, fake, fake, fake, fake, fake, mis, fake, fake,
+                          1 << 40, None)
+    assert st == 1                    # a misaligned dq_idx
+    st = lib.msa_index_kl(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                          16, None)
+    assert st == 3                    # workspace too small
+    assert lib.msa_kernel_path(ctypes.byref(p), msa.OP_INDEX_KL) == b"kl:simt"
+
+
 def test_qk_dtype_values(lib):
     """fp8 e4m3 q and k are valid for bf16 problems only; v and out stay bf16."""
     p = msa.problem_of(workload.WORKLOADS["prefill_32k"])
