@@ -247,9 +247,10 @@ def _events(n):
     return ev
 
 
-def run_steps(msa, w, x, ws, out, steps, warmup, stage_timing=True):
+def run_steps(msa, w, x, ws, out, steps, warmup, stage_timing=True, extra=None):
     """Warm-up, then exactly ``steps`` timed forwards.  Returns (ms/step, stage ms)."""
     kw = dict(q_pos0=w.q_pos0, block_size=w.block_size, top_k=w.top_k, workspace=ws, out=out)
+    kw.update(extra or {})
     for _ in range(warmup):
         msa.forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], **kw)
     per = [(_events(1)[0], _events(5)) for _ in range(steps)] if stage_timing else []
@@ -385,24 +386,55 @@ def path_roofline(cnt, kv_sel_bytes, ms, peaks):
                     "bytes) / HBM peak)"}
 
 
-def measure_workload(msa, w, dev, steps, warmup, peaks, with_e2e):
+def page_inputs(x, w, dev, seed=0):
+    """Moves k, v and k_idx into a shuffled pool of 128-token pages (64 spare
+    pages, zero tails) and returns the forward's paging kwargs.  Untimed."""
+    B, nblk = w.batch, w.nblk
+    npages = B * nblk + 64
+    g = torch.Generator(device=dev).manual_seed(seed + 1)
+    perm = torch.randperm(npages, generator=g, device=dev)[: B * nblk]
+    for name in ("k", "v", "k_idx"):
+        t = x[name].view(torch.uint8)  # bytes: index_copy_ takes every dtype that way
+        tail = tuple(t.shape[2:])
+        pad = nblk * 128 - w.kv_len
+        if pad:
+            t = torch.cat([t, torch.zeros((B, pad) + tail, dtype=t.dtype, device=dev)], dim=1)
+        pool = torch.zeros((npages, 128) + tail, dtype=torch.uint8, device=dev)
+        pool.index_copy_(0, perm, t.reshape((B * nblk, 128) + tail))
+        x[name] = pool.view(x[name].dtype)
+        del t
+    table = perm.view(B, nblk).to(torch.int32).contiguous()
+    return {"block_table": table, "kv_len": w.kv_len}, npages
+
+
+def measure_workload(msa, w, dev, steps, warmup, peaks, with_e2e, paged=False):
     x = make_inputs(w, seed=0, device=dev)
     x.pop("needles")
     p = msa.problem_of(w)
+    extra = {}
+    if paged:
+        extra, npages = page_inputs(x, w, dev)
+        p = msa.make_problem(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
+                             w.head_dim, w.index_dim, w.block_size, w.top_k, w.torch_dtype,
+                             w.q_pos0, index_dtype=w.torch_index_dtype,
+                             qk_dtype=w.torch_qk_dtype, num_pages=npages,
+                             block_table=extra["block_table"])
+        torch.cuda.empty_cache()
     path = msa.kernel_path(p)
     ws = msa.new_workspace(p, msa.OP_FORWARD, dev)
     out = torch.empty(x["q"].shape, dtype=x["v"].dtype, device=dev)  # out has v's dtype
     _, q2k = msa.forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], q_pos0=w.q_pos0,
-                         block_size=w.block_size, top_k=w.top_k, workspace=ws, return_q2k=True)
+                         block_size=w.block_size, top_k=w.top_k, workspace=ws, return_q2k=True,
+                         **extra)
     kv_sel = selected_kv_bytes(w, q2k)
     del q2k
     cnt = counts(w)
     idx = dev.index if dev.index is not None else 0
     with ClockSampler(idx) as clk:
-        ms, stage = run_steps(msa, w, x, ws, out, steps, warmup)
+        ms, stage = run_steps(msa, w, x, ws, out, steps, warmup, extra=extra)
     res = {"w": w, "ms": ms, "stage": stage, "path": path, "cnt": cnt, "kv_sel": kv_sel,
            "clocks": clk.summary(), "launches": msa.launch_count(p) * steps, "x": x}
-    if with_e2e:
+    if with_e2e and not paged:
         xh = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "q_idx", "k_idx")}
         del ws
         torch.cuda.empty_cache()
@@ -539,6 +571,9 @@ def main():
                     help="fp8: q_idx and k_idx in fp8 e4m3 (bf16 workloads)")
     ap.add_argument("--qk-dtype", default="", choices=["", "fp8"],
                     help="fp8: the main branch's q and k in fp8 e4m3, v bf16 (bf16 workloads)")
+    ap.add_argument("--paged", action="store_true",
+                    help="k, v and k_idx in a shuffled pool of 128-token pages (paged KV "
+                         "cache, block table) instead of contiguous sequences")
     ap.add_argument("--index-kl", action="store_true",
                     help="time the KL-alignment loss and its index-branch gradients "
                          "(training side, msa_index_kl) instead of the forward")
@@ -556,7 +591,7 @@ def main():
         w = w.with_(name=f"{w.name}@{a.seq}", q_len=a.seq, kv_len=a.seq,
                     needles=max(1, w.needles * a.seq // w.q_len))
     suffix = (f"+idx_{a.index_dtype}" if a.index_dtype else "") + \
-        (f"+qk_{a.qk_dtype}" if a.qk_dtype else "")
+        (f"+qk_{a.qk_dtype}" if a.qk_dtype else "") + ("+paged" if a.paged else "")
     w = w.with_(name=w.name + suffix, index_dtype=a.index_dtype, qk_dtype=a.qk_dtype)
     if a.batch:
         w = w.with_(name=f"{w.name}@b{a.batch}", batch=a.batch)
@@ -597,7 +632,8 @@ def main():
     torch.cuda.set_device(dev)
     msa.load()
     barrier(world)
-    main_res = measure_workload(msa, w, dev, a.steps, a.warmup, peaks, not a.no_e2e)
+    main_res = measure_workload(msa, w, dev, a.steps, a.warmup, peaks, not a.no_e2e,
+                                paged=a.paged)
     value, ms = weak_value(w.rows, main_res["ms"], world)
     cnt = main_res["cnt"]
     line = {
@@ -631,7 +667,7 @@ def main():
         wd = wd.with_(name=wd.name + suffix, index_dtype=a.index_dtype, qk_dtype=a.qk_dtype)
         del x_main
         torch.cuda.empty_cache()
-        dres = measure_workload(msa, wd, dev, a.steps, a.warmup, peaks, False)
+        dres = measure_workload(msa, wd, dev, a.steps, a.warmup, peaks, False, paged=a.paged)
         dval, dms = weak_value(wd.rows, dres["ms"], world)
         dcnt = dres["cnt"]
         dbytes = dcnt["kidx_bytes"] + dres["kv_sel"]

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(Problem P, const TQ* __r
     __syncthreads();  // previous tile done with ks / vs
     for (int e = threadIdx.x; e < nkeys * D; e += blockDim.x) {
       const int j = e / D, d = e % D;
-      const long long src = (((long long)b * P.Skv + j0 + j) * P.Hkv + g) * D + d;
+      const long long src = ((block_row(P, b, c) + j) * P.Hkv + g) * D + d;
       ks[e] = k[src];
       vs[e] = v[src];
     }

@@ -286,7 +286,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
               uint64_t* fb = &bars->kv_full[kv_stage];
               tc::mbar_arrive_expect_tx(fb, C::kKVBytes);
               uint8_t* dst = kvbuf + kv_stage * C::kKVBytes;
-              const int key0 = tb * P.Skv + tc_ * P.Bk;
+              const int key0 = int(block_row(P, tb, tc_));
               tc::tma_load_3d(dst, &tmap_k, fb, 0, tg, key0);  // fp8: all 128 dims
               if (!QK8) tc::tma_load_3d(dst + kHalf, &tmap_k, fb, 64, tg, key0);
               tc::tma_load_3d(dst + C::kKBytes, &tmap_v, fb, 0, tg, key0);
@@ -588,7 +588,7 @@ int sm_count() {
 
 bool attn_tc_supported(const Problem& P) {
   return !P.f32 && P.D == 128 && P.G == kGroup && P.Bk == 128 &&
-         (long long)P.T * P.Hq < (1LL << 31) && (long long)P.B * P.Skv < (1LL << 31);
+         (long long)P.T * P.Hq < (1LL << 31) && P.kv_rows < (1LL << 31);
 }
 
 cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const void* v,
@@ -623,7 +623,7 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
   }
   {
     // K (fp8: one 128-byte box row per key) and V (bf16: two 64-dim halves)
-    cuuint64_t dims[3] = {128, cuuint64_t(P.Hkv), cuuint64_t(P.B) * P.Skv};
+    cuuint64_t dims[3] = {128, cuuint64_t(P.Hkv), cuuint64_t(P.kv_rows)};
     cuuint64_t kstr[2] = {qk_row, cuuint64_t(P.Hkv) * qk_row};
     cuuint64_t vstr[2] = {128 * 2, cuuint64_t(P.Hkv) * 128 * 2};
     cuuint32_t kbox[3] = {P.qk8 ? 128u : 64u, 1, 128};

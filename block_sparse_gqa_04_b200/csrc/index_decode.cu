@@ -171,7 +171,7 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       uint8_t* st = stages + s * C::kStageBytes;
       if (lane == 0) {
         tc::mbar_arrive_expect_tx(&sh->full[s], C::kKBytes);
-        const int row = b * P.Skv + c * 128;
+        const int row = int(block_row(P, b, c));
         tc::tma_load_2d(st, &tmap_k, &sh->full[s], 0, row);
         if (!FP8) tc::tma_load_2d(st + kKHalf, &tmap_k, &sh->full[s], 64, row);
       }
@@ -313,7 +313,7 @@ int sm_count() {
 bool index_decode_supported(const Problem& P) {
   const int rg = P.Sq * P.Hkv;
   return !P.f32 && P.DI == 128 && P.Bk == 128 && P.Sq <= 8 && rg >= 1 && rg <= kMaxRG &&
-         (long long)P.B * P.Skv < (1LL << 31);
+         P.kv_rows < (1LL << 31);
 }
 
 template <int N, bool FP8>
@@ -338,7 +338,7 @@ cudaError_t launch_index_decode(const Problem& P, const void* q_idx, const void*
   if (!enc) return cudaErrorNotSupported;
   // k_idx rows of 128 dims as 128-byte-wide boxes of 128 keys (128-byte swizzle)
   CUtensorMap map;
-  cuuint64_t dims[2] = {128, cuuint64_t(P.B) * P.Skv};
+  cuuint64_t dims[2] = {128, cuuint64_t(P.kv_rows)};
   cuuint64_t strides[1] = {P.idx8 ? 128u : 256u};
   cuuint32_t box[2] = {P.idx8 ? 128u : 64u, 128};
   cuuint32_t estr[2] = {1, 1};

@@ -113,7 +113,6 @@ __global__ void __launch_bounds__(kKlThreads) kl_rows_kernel(
     const long long j = (long long)c * Bk + m % Bk;
     return j <= t ? j : -1;
   };
-  const long long seq0 = (long long)b * P.Skv;
 
   // pass 1: per head, the maximum and the normaliser of the scaled logits
   for (int hb = 0; hb < G; hb += kHB) {
@@ -125,7 +124,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_rows_kernel(
       const long long j = token(m);
       if (j < 0) continue;
       float z[kHB];
-      head_logits<TQ>(qh, D, hb, nh, k + ((seq0 + j) * P.Hkv + g) * D, P.scale, z);
+      head_logits<TQ>(qh, D, hb, nh, k + (key_row(P, b, j) * P.Hkv + g) * D, P.scale, z);
 #pragma unroll
       for (int i = 0; i < kHB; ++i) {
         if (z[i] > mx[i]) { sm[i] = sm[i] * __expf(mx[i] - z[i]) + 1.f; mx[i] = z[i]; }
@@ -149,7 +148,8 @@ __global__ void __launch_bounds__(kKlThreads) kl_rows_kernel(
     const long long j = token(m);
     if (j < 0) { pt[m] = 0.f; sc[m] = -INFINITY; continue; }
     float p = 0.f;
-    const TQ* krow = k + ((seq0 + j) * P.Hkv + g) * D;
+    const long long row = key_row(P, b, j);
+    const TQ* krow = k + (row * P.Hkv + g) * D;
     for (int hb = 0; hb < G; hb += kHB) {
       const int nh = min(kHB, G - hb);
       float z[kHB];
@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_rows_kernel(
         if (i < nh) p += __expf(z[i] - hm[hb + i]) / hl[hb + i];
     }
     pt[m] = p / G;
-    const TI* irow = k_idx + (seq0 + j) * DI;
+    const TI* irow = k_idx + row * DI;
     float s = 0.f;
     for (int d0 = 0; d0 < DI; d0 += 8) {
       float kv[8];
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_rows_kernel(
     float acc = 0.f;
     for (int m = 0; m < n; ++m) {
       const long long j = token(m);
-      if (j >= 0) acc = fmaf(sc[m], to_f32(k_idx[(seq0 + j) * DI + d]), acc);
+      if (j >= 0) acc = fmaf(sc[m], to_f32(k_idx[key_row(P, b, j) * DI + d]), acc);
     }
     dq_idx[((long long)r * P.Hkv + g) * DI + d] = acc;
   }
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_dk_kernel(Problem P, const TI* 
         }
       }
       if (j < P.Skv) {
-        float* dst = dk_idx + ((long long)b * P.Skv + j) * DI + d0;
+        float* dst = dk_idx + (block_row(P, b, c) + off) * DI + d0;
 #pragma unroll
         for (int i = 0; i < kDkChunk; ++i) atomicAdd(dst + i, acc[i]);
       }
@@ -290,7 +290,7 @@ static cudaError_t launch_kl_t(const Problem& P, const void* q, const void* k, c
   rows<<<pairs, kKlThreads, smem, s>>>(P, (const TQ*)q, (const TQ*)k, (const TI*)q_idx,
                                        (const TI*)k_idx, q2k, kl_rows, dq_idx, ds_buf, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  e = cudaMemsetAsync(dk_idx, 0, sizeof(float) * size_t(P.B) * P.Skv * P.DI, s);
+  e = cudaMemsetAsync(dk_idx, 0, sizeof(float) * size_t(P.kv_rows) * P.DI, s);
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(std::min<long long>(P.nlists, 148LL * 16));
   kl_dk_kernel<TI><<<grid, kKlThreads, 0, s>>>(P, (const TI*)q_idx, ds_buf, L, dk_idx);

@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(128) index_rows_kernel(Problem P, const T* __r
   const long long j0 = (long long)c * P.Bk;
   if (j0 > t_last) return;  // no row of this tile sees block c
   const int nkeys = (int)min((long long)P.Bk, (long long)P.Skv - j0);
-  const T* kb = k_idx + ((long long)b * P.Skv + j0) * DI;
+  const T* kb = k_idx + block_row(P, b, c) * DI;
   for (int e = threadIdx.x; e < nkeys * DI; e += blockDim.x) ks[e] = to_f32(kb[e]);
   __syncthreads();
   if (i >= P.Sq) return;
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(128) index_keys_kernel(Problem P, const T* __r
   const bool in_seq = threadIdx.x < P.Bk && j < P.Skv;
   float kv[DI];
   if (in_seq) {
-    load_vec<T, DI>(k_idx + ((long long)b * P.Skv + j) * DI, kv);
+    load_vec<T, DI>(k_idx + key_row(P, b, j) * DI, kv);
   } else {
 #pragma unroll
     for (int d = 0; d < DI; ++d) kv[d] = 0.f;

@@ -177,7 +177,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       for (long long L = L0; L < L1; ++L) {
         if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort)) { failed = true; break; }
         tc::mbar_arrive_expect_tx(&bars->full[stage], X::kStageBytes);
-        const int row = w.b * P.Skv + w.c * P.Bk;
+        const int row = int(block_row(P, w.b, w.c));
         uint8_t* dst = stages + stage * X::kStageBytes;
         tc::tma_load_2d(dst, &tmap_k, &bars->full[stage], 0, row);
         if (!FP8) tc::tma_load_2d(dst + X::kHalfBytes, &tmap_k, &bars->full[stage], 64, row);
@@ -359,7 +359,7 @@ int sm_count() {
 
 bool index_tc_supported(const Problem& P) {
   return !P.f32 && P.DI == 128 && P.Bk == 128 && P.Hkv <= kMaxGroups && P.Sq > 8 &&
-         (long long)P.B * P.Skv < (1LL << 31);
+         P.kv_rows < (1LL << 31);
 }
 
 template <bool FP8>
@@ -370,7 +370,7 @@ static cudaError_t launch_t(const Problem& P, const void* q_idx, const void* k_i
   if (!enc) return cudaErrorNotSupported;
   // k_idx rows of 128 dims, copied as 128-byte-wide boxes of 128 keys (128-byte swizzle)
   CUtensorMap map;
-  cuuint64_t dims[2] = {FP8 ? 128u : 128u, cuuint64_t(P.B) * P.Skv};
+  cuuint64_t dims[2] = {FP8 ? 128u : 128u, cuuint64_t(P.kv_rows)};
   cuuint64_t strides[1] = {cuuint64_t(X::kRowBytes)};
   cuuint32_t box[2] = {FP8 ? 128u : 64u, 128};
   cuuint32_t estr[2] = {1, 1};

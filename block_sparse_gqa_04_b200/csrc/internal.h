@@ -28,6 +28,11 @@ struct Problem {
   bool f32;         // fp32 tensors (else bf16)
   bool idx8;        // q_idx and k_idx are fp8 e4m3 (bf16 problems)
   bool qk8;         // q and k are fp8 e4m3, v bf16 (bf16 problems)
+  // KV storage: contiguous per sequence (table == nullptr) or a pool of
+  // `pages` pages of Bk tokens named by table[b * nblk + c]
+  const int32_t* table;
+  int pages;
+  long long kv_rows;  // rows of k, v and k_idx in memory: B * Skv or pages * Bk
   long long nlists; // B * Hkv * nqc * nblk
 };
 
@@ -117,8 +122,26 @@ cudaError_t launch_index_kl(const Problem& P, const void* q, const void* k, cons
                             float* dk_idx, int32_t* status, cudaStream_t s);
 
 // Device status bits (workspace status word): 1 = invalid q2k entry given to
-// attend, 2 = a bounded wait inside a tensor-core kernel gave up.
+// attend, 2 = a bounded wait inside a tensor-core kernel gave up, 4 = a block
+// table page id outside [0, pages).
 constexpr int kStatusBadEntry = 1;
+constexpr int kStatusBadPage = 4;
+
+// First memory row of block c of sequence b in k, v and k_idx: contiguous
+// sequences, or the page the block table names (page 0 for an id outside
+// [0, pages), which launch_check_table flags).  Rows of a block are contiguous.
+__device__ __forceinline__ long long block_row(const Problem& P, int b, long long c) {
+  if (!P.table) return (long long)b * P.Skv + c * P.Bk;
+  const int pg = P.table[(long long)b * P.nblk + c];
+  return (pg >= 0 && pg < P.pages) ? (long long)pg * P.Bk : 0;
+}
+// Memory row of token j of sequence b.
+__device__ __forceinline__ long long key_row(const Problem& P, int b, long long j) {
+  return block_row(P, b, j / P.Bk) + j % P.Bk;
+}
+// Flags kStatusBadPage for every block table entry outside [0, pages) (paged
+// problems only; no launch otherwise).
+cudaError_t launch_check_table(const Problem& P, int32_t* status, cudaStream_t s);
 
 // Kernel launches made by each launcher (for msa_launch_count).
 constexpr int kLaunchesInvert = 5;

@@ -279,6 +279,21 @@ static unsigned grid_for(long long n, int threads) {
   return unsigned(b < 1 ? 1 : b);
 }
 
+__global__ void check_table_kernel(Problem P, int32_t* status) {
+  const long long n = (long long)P.B * P.nblk;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int pg = P.table[i];
+    if (pg < 0 || pg >= P.pages) atomicOr(status, kStatusBadPage);
+  }
+}
+
+cudaError_t launch_check_table(const Problem& P, int32_t* status, cudaStream_t s) {
+  if (!P.table) return cudaSuccess;
+  check_table_kernel<<<grid_for((long long)P.B * P.nblk, 256), 256, 0, s>>>(P, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_invert(const Problem& P, const int32_t* q2k, const Lists& L,
                           int32_t* status, cudaStream_t s) {
   const long long n = (long long)P.Hkv * P.T * P.K;

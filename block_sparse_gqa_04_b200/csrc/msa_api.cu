@@ -63,6 +63,11 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
   P->f32 = p->dtype == MSA_F32;
   P->idx8 = p->index_dtype == MSA_FP8_E4M3;
   P->qk8 = p->qk_dtype == MSA_FP8_E4M3;
+  if (p->num_pages < 0 || (p->num_pages > 0 && !p->block_table)) return MSA_ERR_INVALID_ARG;
+  P->table = p->num_pages > 0 ? p->block_table : nullptr;
+  P->pages = p->num_pages;
+  P->kv_rows = P->table ? (long long)P->pages * P->Bk : (long long)P->B * P->Skv;
+  if (P->kv_rows >= (1LL << 31)) return MSA_ERR_UNSUPPORTED;
   P->nlists = (long long)P->B * P->Hkv * P->nqc * P->nblk;
   if (P->nlists + 1 >= (1LL << 31)) return MSA_ERR_UNSUPPORTED;
   return MSA_OK;
@@ -133,8 +138,9 @@ msa_status_t run_select(const Problem& P, const void* q_idx, const void* k_idx, 
                         float* bscores, void* ws, cudaStream_t s) {
   const Layout L = layout(P, MSA_OP_SELECT);
   float* bmax = bscores ? bscores : at<float>(ws, L.bmax);
-  cudaError_t e = cudaSuccess;
-  if (bscores) e = msa::launch_fill(bscores, size_t(P.Hkv) * P.T * P.nblk, -INFINITY, s);
+  cudaError_t e = msa::launch_check_table(P, at<int32_t>(ws, L.status), s);
+  if (bscores && e == cudaSuccess)
+    e = msa::launch_fill(bscores, size_t(P.Hkv) * P.T * P.nblk, -INFINITY, s);
   if (e == cudaSuccess) {
     int32_t* status = at<int32_t>(ws, L.status);
     e = msa::index_tc_supported(P)       ? msa::launch_index_tc(P, q_idx, k_idx, bmax, status, s)
@@ -158,8 +164,9 @@ msa_status_t run_attend(const Problem& P, const void* q, const void* k, const vo
                    at<int32_t>(ws, L.tiles), at<int32_t>(ws, L.seg_sums)};
   msa::Partials part{at<void>(ws, L.part_o), at<float>(ws, L.part_lse)};
   const bool tc = msa::attn_tc_supported(P);
-  cudaError_t e;
-  if (msa::lists_direct(P)) {
+  cudaError_t e = msa::launch_check_table(P, at<int32_t>(ws, L.status), s);
+  if (e != cudaSuccess) {
+  } else if (msa::lists_direct(P)) {
     e = msa::launch_lists_direct(P, q2k, lists, at<int32_t>(ws, L.status), s);
   } else {
     e = msa::launch_invert(P, q2k, lists, at<int32_t>(ws, L.status), s);
@@ -278,7 +285,8 @@ msa_status_t msa_index_kl(const msa_problem_t* p, const void* q, const void* k,
                    at<int32_t>(ws, L.entries), at<int32_t>(ws, L.pos), nullptr,
                    at<int32_t>(ws, L.seg_sums)};
   int32_t* status = at<int32_t>(ws, L.status);
-  cudaError_t e = msa::launch_invert(P, q2k, lists, status, s);
+  cudaError_t e = msa::launch_check_table(P, status, s);
+  if (e == cudaSuccess) e = msa::launch_invert(P, q2k, lists, status, s);
   if (e == cudaSuccess)
     e = msa::launch_index_kl(P, q, k, q_idx, k_idx, q2k, lists, at<float>(ws, L.kl_rows),
                              at<float>(ws, L.kl_ds), loss, dq_idx, dk_idx, status, s);
@@ -306,16 +314,18 @@ int32_t msa_set_stage_events(void* const* events, int32_t n) {
 int32_t msa_launch_count(const msa_problem_t* p, int32_t op) {
   Problem P;
   if (resolve(p, &P) != MSA_OK || P.T == 0) return 0;
-  const int sel = 2;                               // index + top-k
+  const int chk = P.table ? 1 : 0;                  // block table check (paged)
+  const int sel = chk + 2;                         // index + top-k
   // lists (+ tile records on the tensor-core path) + attention + combine
-  const int att = (msa::lists_direct(P) ? 1
-                                         : msa::kLaunchesInvert + (msa::attn_tc_supported(P) ? 1 : 0)) +
+  const int att = chk +
+                  (msa::lists_direct(P) ? 1
+                                        : msa::kLaunchesInvert + (msa::attn_tc_supported(P) ? 1 : 0)) +
                   2;
   switch (op) {
     case MSA_OP_SELECT: return sel;
     case MSA_OP_ATTEND: return att;
     case MSA_OP_FORWARD: return sel + att;
-    case MSA_OP_INDEX_KL: return msa::kLaunchesInvert + 3;  // lists, rows, dk, sum
+    case MSA_OP_INDEX_KL: return chk + msa::kLaunchesInvert + 3;  // lists, rows, dk, sum
   }
   return 0;
 }

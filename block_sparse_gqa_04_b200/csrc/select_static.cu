@@ -76,6 +76,7 @@ extern "C" msa_status_t msa_select_static(const msa_problem_t* p, const void* q_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = msa::launch_check_table(P, status, s);
   if (e == cudaSuccess)
     e = msa::index_tc_supported(P)       ? msa::launch_index_tc(P, q_idx, k_idx, bmax, status, s)
         : msa::index_decode_supported(P) ? msa::launch_index_decode(P, q_idx, k_idx, bmax, status, s)

@@ -45,6 +45,7 @@ class Problem(ctypes.Structure):
         ("block_size", ctypes.c_int32), ("top_k", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("q_pos0", ctypes.c_int64), ("softmax_scale", ctypes.c_float),
         ("index_dtype", ctypes.c_int32), ("qk_dtype", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32), ("block_table", ctypes.c_void_p),
     ]
 
 
@@ -89,16 +90,21 @@ def load() -> ctypes.CDLL:
 
 def make_problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
                  block_size=128, top_k=16, dtype=torch.bfloat16, q_pos0=0,
-                 softmax_scale=0.0, index_dtype=None, qk_dtype=None) -> Problem:
+                 softmax_scale=0.0, index_dtype=None, qk_dtype=None, num_pages=0,
+                 block_table=None) -> Problem:
     """dtype: torch dtype of v and out (and of every other tensor unless stated:
     fp32 or bf16); index_dtype / qk_dtype: torch dtype of q_idx/k_idx / of q/k
-    when it differs (torch.float8_e4m3fn for fp8 tensors)."""
+    when it differs (torch.float8_e4m3fn for fp8 tensors).  num_pages > 0 with
+    block_table (an int32 CUDA tensor [batch, ceil(kv_len/128)]) describes a
+    paged KV cache: k, v [num_pages, 128, Hkv, D], k_idx [num_pages, 128, di]."""
     fp8 = torch.float8_e4m3fn
     main = MSA_F32 if dtype == torch.float32 else MSA_BF16
     idx = MSA_FP8_E4M3 if (index_dtype == fp8 or dtype == fp8) else 0
     qk = MSA_FP8_E4M3 if qk_dtype == fp8 else 0
+    table = block_table.data_ptr() if block_table is not None else None
     return Problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
-                   block_size, top_k, main, q_pos0, softmax_scale, idx, qk)
+                   block_size, top_k, main, q_pos0, softmax_scale, idx, qk,
+                   num_pages if block_table is not None else 0, table)
 
 
 def problem_of(w, softmax_scale: float = 0.0) -> Problem:
@@ -171,29 +177,56 @@ def _require_cuda(*ts):
             raise ValueError("libmsa takes contiguous tensors")
 
 
-def _dims(q, k, q_idx=None, v=None, k_idx=None):
+def _dims(q, k, q_idx=None, v=None, k_idx=None, kv_len=None):
     """Sizes from q [B, Sq, Hq, D], k [B, Skv, Hkv, D] (and q_idx [B, Sq, Hkv, d]);
-    v, k_idx and the rest must agree, or nothing is launched."""
+    v, k_idx and the rest must agree, or nothing is launched.  With a paged
+    cache (kv_len given) k, v are [pages, 128, Hkv, D] and k_idx [pages, 128, d]."""
     B, Sq, Hq, D = q.shape
-    Skv, Hkv = k.shape[1], k.shape[2]
+    Hkv = k.shape[2]
     di = q_idx.shape[3] if q_idx is not None else 32
-    want = {"k": (k, (B, Skv, Hkv, D)), "v": (v, (B, Skv, Hkv, D)),
-            "q_idx": (q_idx, (B, Sq, Hkv, di)), "k_idx": (k_idx, (B, Skv, di))}
+    if kv_len is None:
+        Skv = k.shape[1]
+        rows = (B, Skv)
+    else:
+        Skv = int(kv_len)
+        rows = (k.shape[0], 128)
+    want = {"k": (k, rows + (Hkv, D)), "v": (v, rows + (Hkv, D)),
+            "q_idx": (q_idx, (B, Sq, Hkv, di)), "k_idx": (k_idx, rows + (di,))}
     for name, (t, shape) in want.items():
         if t is not None and tuple(t.shape) != shape:
             raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
     return B, Sq, Hq, D, Skv, Hkv, di
 
 
+def _paged(block_table, kv_len, batch, num_pages, block_size):
+    """Checks a paged cache's block table; returns make_problem's paging kwargs."""
+    if block_table is None:
+        if kv_len is not None:
+            raise ValueError("kv_len is given only with a block_table")
+        return {}
+    if kv_len is None:
+        raise ValueError("a paged cache needs kv_len")
+    _require_cuda(block_table)
+    nblk = -(-int(kv_len) // 128)
+    if (block_table.dtype != torch.int32 or tuple(block_table.shape) != (batch, nblk)
+            or block_size != 128):
+        raise ValueError(f"block_table must be int32 [{batch}, {nblk}] with block_size 128")
+    return {"num_pages": int(num_pages), "block_table": block_table}
+
+
 def select(q_idx: torch.Tensor, k_idx: torch.Tensor, *, q_pos0: int = 0, block_size: int = 128,
            top_k: int = 16, return_block_scores: bool = False,
-           workspace: Optional[torch.Tensor] = None):
-    """Index branch: returns q2k [Hkv, B*Sq, top_k] int32 (and block scores)."""
+           workspace: Optional[torch.Tensor] = None, block_table=None, kv_len=None):
+    """Index branch: returns q2k [Hkv, B*Sq, top_k] int32 (and block scores).
+    With block_table and kv_len, k_idx is a paged cache [pages, 128, di]."""
     _require_cuda(q_idx, k_idx)
     B, Sq, Hkv, di = q_idx.shape
-    Skv = k_idx.shape[1]
+    Skv = k_idx.shape[1] if block_table is None else int(kv_len)
+    pg = _paged(block_table, kv_len, B, k_idx.shape[0], block_size)
+    if tuple(k_idx.shape) != ((k_idx.shape[0], 128, di) if pg else (B, Skv, di)):
+        raise ValueError(f"k_idx has shape {tuple(k_idx.shape)}")
     p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, top_k, q_idx.dtype, q_pos0,
-                     index_dtype=q_idx.dtype)
+                     index_dtype=q_idx.dtype, **pg)
     dev = q_idx.device
     q2k = torch.empty((Hkv, B * Sq, top_k), dtype=torch.int32, device=dev)
     nblk = -(-Skv // block_size)
@@ -239,16 +272,19 @@ def _check_qkv_dtypes(q, k, v):
 
 def attend(q, k, v, q2k, *, q_pos0: int = 0, block_size: int = 128,
            softmax_scale: float = 0.0, return_lse: bool = False,
-           workspace: Optional[torch.Tensor] = None, check_device_status: bool = False):
-    """Main branch over a given selection q2k [Hkv, B*Sq, top_k] (int32)."""
+           workspace: Optional[torch.Tensor] = None, check_device_status: bool = False,
+           block_table=None, kv_len=None):
+    """Main branch over a given selection q2k [Hkv, B*Sq, top_k] (int32).
+    With block_table and kv_len, k and v are paged caches [pages, 128, Hkv, D]."""
     _require_cuda(q, k, v, q2k)
-    B, Sq, Hq, D, Skv, Hkv, _ = _dims(q, k, v=v)
+    B, Sq, Hq, D, Skv, Hkv, _ = _dims(q, k, v=v, kv_len=kv_len)
+    pg = _paged(block_table, kv_len, B, k.shape[0], block_size)
     top_k = q2k.shape[2]
     if q2k.dtype != torch.int32 or tuple(q2k.shape[:2]) != (Hkv, B * Sq):
         raise ValueError("q2k must be int32 [Hkv, B*Sq, top_k]")
     _check_qkv_dtypes(q, k, v)
     p = make_problem(B, Sq, Skv, Hq, Hkv, D, 32, block_size, top_k, v.dtype, q_pos0,
-                     softmax_scale, qk_dtype=q.dtype)
+                     softmax_scale, qk_dtype=q.dtype, **pg)
     dev = q.device
     out = torch.empty(q.shape, dtype=v.dtype, device=dev)
     lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=dev) if return_lse else None
@@ -265,23 +301,25 @@ def attend(q, k, v, q2k, *, q_pos0: int = 0, block_size: int = 128,
 
 def index_kl(q, k, q_idx, k_idx, q2k, *, q_pos0: int = 0, block_size: int = 128,
              softmax_scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
-             check_device_status: bool = False):
+             check_device_status: bool = False, block_table=None, kv_len=None):
     """KL-alignment loss of the index branch and its gradients (training side).
 
     The selection q2k [Hkv, B*Sq, top_k] (int32, as :func:`select` returns it)
     and the teacher, from q and k, are constants.  Returns (loss, dq_idx, dk_idx):
     the mean KL(teacher || index) over the (row, group) pairs as a 0-d fp32
-    tensor, and its fp32 gradients shaped like q_idx and k_idx.
+    tensor, and its fp32 gradients shaped like q_idx and k_idx (with a paged
+    cache, dk_idx is shaped like the k_idx page pool).
     """
     _require_cuda(q, k, q_idx, k_idx, q2k)
-    B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx, k_idx=k_idx)
+    B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx, k_idx=k_idx, kv_len=kv_len)
+    pg = _paged(block_table, kv_len, B, k.shape[0], block_size)
     if q2k.dtype != torch.int32 or q2k.dim() != 3 or tuple(q2k.shape[:2]) != (Hkv, B * Sq):
         raise ValueError("q2k must be int32 [Hkv, B*Sq, top_k]")
     if k.dtype != q.dtype:
         raise ValueError(f"q and k dtypes differ: {q.dtype} vs {k.dtype}")
     main = torch.float32 if q.dtype == torch.float32 else torch.bfloat16
     p = make_problem(B, Sq, Skv, Hq, Hkv, D, di, block_size, q2k.shape[2], main, q_pos0,
-                     softmax_scale, index_dtype=q_idx.dtype, qk_dtype=q.dtype)
+                     softmax_scale, index_dtype=q_idx.dtype, qk_dtype=q.dtype, **pg)
     dev = q.device
     loss = torch.empty((), dtype=torch.float32, device=dev)
     dq = torch.empty(q_idx.shape, dtype=torch.float32, device=dev)
@@ -301,28 +339,33 @@ def index_kl(q, k, q_idx, k_idx, q2k, *, q_pos0: int = 0, block_size: int = 128,
 def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, top_k: int = 16,
             softmax_scale: float = 0.0, return_lse: bool = False, return_q2k: bool = False,
             workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-            device=None, check_device_status: bool = False):
+            device=None, check_device_status: bool = False, block_table=None, kv_len=None):
     """Index branch + main branch.  Returns out (and lse, q2k when asked).
 
     CUDA tensors are used in place.  Host tensors (ideally pinned) are copied to
     ``device`` (default ``cuda``) before the call and the results copied back.
     ``check_device_status`` waits for the call and raises if the device
-    recorded a problem (a bounded wait that gave up).
+    recorded a problem (a bounded wait that gave up).  With block_table ([B,
+    ceil(kv_len/128)] int32, on the device) and kv_len, k, v and k_idx are a paged
+    KV cache: [pages, 128, Hkv, D] and [pages, 128, di].
     """
     host = not q.is_cuda
     if host:
         dev = torch.device(device or "cuda")
         nb = q.is_pinned()
         q, k, v, q_idx, k_idx = (t.to(dev, non_blocking=nb) for t in (q, k, v, q_idx, k_idx))
+        if block_table is not None:
+            block_table = block_table.to(dev, non_blocking=nb)
     _require_cuda(q, k, v, q_idx, k_idx)
-    B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx, v=v, k_idx=k_idx)
+    B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx, v=v, k_idx=k_idx, kv_len=kv_len)
+    pg = _paged(block_table, kv_len, B, k.shape[0], block_size)
     _check_qkv_dtypes(q, k, v)
     if out is not None and (out.dtype != v.dtype or tuple(out.shape) != tuple(q.shape)
                             or not out.is_contiguous()):
         raise ValueError(f"out must be a contiguous {tuple(q.shape)} tensor of v's dtype "
                          f"{v.dtype}, got {tuple(out.shape)} {out.dtype}")
     p = make_problem(B, Sq, Skv, Hq, Hkv, D, di, block_size, top_k, v.dtype, q_pos0,
-                     softmax_scale, index_dtype=q_idx.dtype, qk_dtype=q.dtype)
+                     softmax_scale, index_dtype=q_idx.dtype, qk_dtype=q.dtype, **pg)
     dev = q.device
     o = out if (out is not None and not host) else torch.empty(q.shape, dtype=v.dtype, device=dev)
     lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=dev) if return_lse else None

@@ -20,6 +20,10 @@
  *        k, v     [batch, kv_len, num_kv_heads, head_dim]
  *        q_idx    [batch, q_len, num_kv_heads, index_dim]
  *        k_idx    [batch, kv_len, index_dim]       (one shared index-key head)
+ *    (with a paged KV cache, num_pages > 0, k, v and k_idx are page pools:
+ *        k, v     [num_pages, 128, num_kv_heads, head_dim]
+ *        k_idx    [num_pages, 128, index_dim]
+ *     and block_table [batch, ceil(kv_len/128)] names each block's page)
  *        q2k      [num_kv_heads, batch*q_len, top_k]  int32
  *        lse      [batch, q_len, num_q_heads]      float32
  *        block_scores [num_kv_heads, batch*q_len, nblk] float32,
@@ -37,8 +41,9 @@
  *  - Argument errors are returned synchronously, before any launch, and leave
  *    every output untouched.  A failed launch returns MSA_ERR_CUDA.  Problems
  *    found on the device (a q2k entry outside [-1, floor(t/block_size)] given
- *    to msa_attend) are recorded in the workspace status word, read with
- *    msa_device_status(); such entries are skipped.
+ *    to msa_attend: bit 1; a block_table page id outside [0, num_pages): bit 4)
+ *    are recorded in the workspace status word, read with msa_device_status();
+ *    such entries are skipped, such pages read as page 0.
  *  - q_len == 0 is a valid empty problem: the call returns MSA_OK without
  *    looking at the pointers or launching anything.
  */
@@ -99,6 +104,18 @@ typedef struct {
                              e4m3 and the main-branch scores q . k are formed from
                              them (bf16 problems; v, out and the partial states stay
                              bf16); other values are invalid                      */
+  int32_t num_pages;      /* 0: k, v and k_idx are contiguous per sequence (the
+                             layouts below).  > 0: paged KV cache: k and v are
+                             [num_pages, 128, num_kv_heads, head_dim] and k_idx
+                             [num_pages, 128, index_dim], and block_table maps
+                             block c of sequence b (tokens c*128 .. c*128+127) to
+                             page block_table[b * ceil(kv_len/128) + c]; pages may
+                             be shared between sequences.  Rows of a sequence's last
+                             page beyond kv_len are read and weighted by zero, so
+                             they must hold finite values.  Requires block_size 128 */
+  const int32_t* block_table; /* device, [batch, ceil(kv_len/128)] int32 page ids in
+                             [0, num_pages) (num_pages > 0), else ignored; an id
+                             outside that range sets status bit 4 and reads page 0 */
 } msa_problem_t;
 
 /* Bytes of workspace that `op` needs for problem `p` (0 if p is invalid).

@@ -271,6 +271,24 @@ def forward(q, k, v, q_idx, k_idx, q_pos0: int, block_size: int, top_k: int,
 # KL-alignment loss of the index branch (training side)
 # ---------------------------------------------------------------------------
 
+def gather_pages(cache, block_table, kv_len: int, page_size: int = 128) -> np.ndarray:
+    """The per-sequence layout [B, kv_len, ...] of a paged KV cache.
+
+    A paged cache stores each sequence's tokens in pages of ``page_size`` tokens:
+    token j of sequence b is row j % page_size of page block_table[b, j //
+    page_size] (the vLLM-style layout the serving path of the survey names).
+    This is that definition written out, one token at a time.
+    """
+    c = np.asarray(cache)
+    tab = np.asarray(block_table)
+    B = tab.shape[0]
+    out = np.empty((B, kv_len) + c.shape[2:], dtype=c.dtype)
+    for b in range(B):
+        for j in range(kv_len):
+            out[b, j] = c[tab[b, j // page_size], j % page_size]
+    return out
+
+
 def selected_tokens(blocks, t: int, block_size: int) -> np.ndarray:
     """The causally visible tokens 0..t of the selected blocks, ascending."""
     keys = []

@@ -44,16 +44,17 @@ def test_problem_struct_layout_matches_header(tmp_path):
     src = tmp_path / "layout.c"
     src.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "msa.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu\\n\", sizeof(msa_problem_t),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(msa_problem_t),"
         " offsetof(msa_problem_t,q_pos0), offsetof(msa_problem_t,softmax_scale),"
-        " offsetof(msa_problem_t,index_dtype), offsetof(msa_problem_t,qk_dtype));return 0;}\n")
+        " offsetof(msa_problem_t,index_dtype), offsetof(msa_problem_t,qk_dtype),"
+        " offsetof(msa_problem_t,num_pages), offsetof(msa_problem_t,block_table));return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
                    check=True)
     got = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     P = msa.Problem
     want = [ctypes.sizeof(P), P.q_pos0.offset, P.softmax_scale.offset, P.index_dtype.offset,
-            P.qk_dtype.offset]
+            P.qk_dtype.offset, P.num_pages.offset, P.block_table.offset]
     assert [int(x) for x in got] == want
 
 

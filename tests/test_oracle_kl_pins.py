@@ -116,3 +116,24 @@ def test_shift_invariance_of_each_sequence():
     scale = np.abs(dk).max()
     assert scale > 0
     np.testing.assert_allclose(dk.sum(axis=1), 0, atol=1e-14 * dk.shape[1] + 1e-12 * scale)
+
+
+def test_gather_pages_inverts_paging():
+    # page a contiguous cache by hand (a shuffled pool with unused pages) and
+    # gather it back; a two-sequence shared first page too
+    rng = np.random.default_rng(8)
+    B, L, H, D = 3, 300, 2, 4
+    kv = rng.standard_normal((B, L, H, D))
+    nblk = -(-L // 128)
+    pages = rng.permutation(B * nblk + 5)[: B * nblk].reshape(B, nblk)
+    pool = rng.standard_normal((B * nblk + 5, 128, H, D))
+    for b in range(B):
+        for c in range(nblk):
+            n = min(128, L - c * 128)
+            pool[pages[b, c], :n] = kv[b, c * 128: c * 128 + n]
+    np.testing.assert_array_equal(O.gather_pages(pool, pages, L), kv)
+    shared = pages.copy()
+    shared[1, 0] = shared[0, 0]
+    got = O.gather_pages(pool, shared, L)
+    np.testing.assert_array_equal(got[1, :128], kv[0, :128])
+    np.testing.assert_array_equal(got[1, 128:], kv[1, 128:])
