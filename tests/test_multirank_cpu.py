@@ -37,7 +37,7 @@ def _rank(rank, world, port, out):
 def test_two_gloo_ranks_agree_on_max_time():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a threaded process
     out = mgr.dict()
     mp.spawn(_rank, args=(world, port, out), nprocs=world, join=True)
     assert out[0] == out[1]
