@@ -31,7 +31,7 @@
 namespace msa {
 
 constexpr int kKlThreads = 128;
-constexpr int kHB = 16;       // query heads whose logits one pass keeps in registers
+constexpr int kHB = 8;        // query heads whose logits one pass keeps in registers
 constexpr int kDkChunk = 32;  // index dims per accumulation pass of kl_dk_kernel
 
 // Block-wide reductions over kKlThreads threads (scratch: 4 floats).
