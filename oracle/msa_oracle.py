@@ -276,7 +276,7 @@ def gather_pages(cache, block_table, kv_len: int, page_size: int = 128) -> np.nd
 
     A paged cache stores each sequence's tokens in pages of ``page_size`` tokens:
     token j of sequence b is row j % page_size of page block_table[b, j //
-    page_size] (the vLLM-style layout the serving path of the survey names).
+    page_size] (a vLLM-style block table).
     This is that definition written out, one token at a time.
     """
     c = np.asarray(cache)
