@@ -190,3 +190,46 @@ def test_status_strings_and_launch_counts(lib):
     assert msa.launch_count(p, msa.OP_SELECT) + msa.launch_count(p, msa.OP_ATTEND) == \
         msa.launch_count(p, msa.OP_FORWARD)
     assert "index" in msa.kernel_path(p) and "attn" in msa.kernel_path(p)
+
+
+def test_binding_checks_shapes_before_any_launch():
+    """Mismatched tensors and bad paging arguments are rejected in Python (CPU
+    tensors of the right shapes get as far as the CUDA check)."""
+    B, Sq, Skv, Hq, Hkv, D, di = 2, 4, 300, 16, 2, 128, 32
+    q = torch.zeros((B, Sq, Hq, D), dtype=torch.bfloat16)
+    k = torch.zeros((B, Skv, Hkv, D), dtype=torch.bfloat16)
+    qi = torch.zeros((B, Sq, Hkv, di), dtype=torch.bfloat16)
+    ki = torch.zeros((B, Skv, di), dtype=torch.bfloat16)
+    assert msa._dims(q, k, qi, v=k, k_idx=ki) == (B, Sq, Hq, D, Skv, Hkv, di)
+    with pytest.raises(ValueError):
+        msa._dims(q, k, qi, v=k[:, :-1], k_idx=ki)          # v shorter than k
+    with pytest.raises(ValueError):
+        msa._dims(q, k, qi, v=k, k_idx=ki[:1])              # k_idx batch differs
+    # paged: pools of 128-token pages, kv_len given
+    kp = torch.zeros((7, 128, Hkv, D), dtype=torch.bfloat16)
+    kip = torch.zeros((7, 128, di), dtype=torch.bfloat16)
+    assert msa._dims(q, kp, qi, v=kp, k_idx=kip, kv_len=Skv)[4] == Skv
+    with pytest.raises(ValueError):
+        msa._dims(q, kp, qi, v=kp, k_idx=kip[:, :64], kv_len=Skv)
+    with pytest.raises(ValueError):
+        msa._paged(None, Skv, B, 7, 128)                     # kv_len without a table
+    table = torch.zeros((B, 3), dtype=torch.int32)
+    with pytest.raises(ValueError):
+        msa._paged(table, None, B, 7, 128)                   # table without kv_len
+    with pytest.raises(ValueError):
+        msa._paged(table, Skv, B, 7, 128)                    # a host table
+    assert msa._paged(None, None, B, 7, 128) == {}
+
+
+def test_paged_problem_fields_reach_the_library(lib):
+    w = workload.WORKLOADS["decode_128k"]
+    p = msa.problem_of(w)
+    assert p.num_pages == 0 and not p.block_table
+    p.num_pages = 5
+    assert msa.workspace_size(p, msa.OP_FORWARD) == 0      # pages without a table
+    p.num_pages = -1
+    assert msa.workspace_size(p, msa.OP_FORWARD) == 0
+    p.num_pages, p.block_table = 4096, 1 << 20             # any non-null device address
+    assert msa.workspace_size(p, msa.OP_FORWARD) == msa.workspace_size(
+        msa.problem_of(w), msa.OP_FORWARD)
+    assert msa.launch_count(p) == msa.launch_count(msa.problem_of(w)) + 2  # table checks
