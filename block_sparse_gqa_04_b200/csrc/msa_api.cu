@@ -34,7 +34,10 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
   if (p->dtype != MSA_BF16 && p->dtype != MSA_F32) return MSA_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.0f) || isinf(p->softmax_scale)) return MSA_ERR_INVALID_ARG;
   const int G = p->num_q_heads / p->num_kv_heads;
-  if (p->block_size != 128) return MSA_ERR_UNSUPPORTED;
+  // 128-token blocks on every kernel; 64 and 32 on the CUDA-core kernels (the
+  // tensor-core kernels tile one 128-key block per MMA and say so)
+  if (p->block_size != 128 && p->block_size != 64 && p->block_size != 32)
+    return MSA_ERR_UNSUPPORTED;
   if (p->top_k > 32) return MSA_ERR_UNSUPPORTED;
   if (p->head_dim != 64 && p->head_dim != 128) return MSA_ERR_UNSUPPORTED;
   if (p->index_dim != 32 && p->index_dim != 64 && p->index_dim != 128) return MSA_ERR_UNSUPPORTED;
@@ -64,6 +67,7 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
   P->idx8 = p->index_dtype == MSA_FP8_E4M3;
   P->qk8 = p->qk_dtype == MSA_FP8_E4M3;
   if (p->num_pages < 0 || (p->num_pages > 0 && !p->block_table)) return MSA_ERR_INVALID_ARG;
+  if (p->num_pages > 0 && p->block_size != 128) return MSA_ERR_UNSUPPORTED;  // page = block
   P->table = p->num_pages > 0 ? p->block_table : nullptr;
   P->pages = p->num_pages;
   P->kv_rows = P->table ? (long long)P->pages * P->Bk : (long long)P->B * P->Skv;

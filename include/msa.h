@@ -92,7 +92,8 @@ typedef struct {
   int32_t num_kv_heads;   /* GQA groups = index-query heads                    */
   int32_t head_dim;       /* D of q, k, v                                      */
   int32_t index_dim;      /* d of q_idx, k_idx                                 */
-  int32_t block_size;     /* Bk, tokens per KV block (128)                     */
+  int32_t block_size;     /* Bk, tokens per KV block: 128 (every kernel), or 64
+                             and 32 (CUDA-core kernels only)                   */
   int32_t top_k;          /* blocks kept per (query, group), local one included */
   int32_t dtype;          /* msa_dtype_t of q, k, v, q_idx, k_idx and out (see
                              index_dtype and qk_dtype for fp8 inputs)          */

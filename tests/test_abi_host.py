@@ -72,7 +72,8 @@ def test_workspace_sizes(lib):
 
 @pytest.mark.parametrize("field,value,code", [
     ("num_q_heads", 63, 1),          # not a multiple of num_kv_heads
-    ("block_size", 64, 2),
+    ("block_size", 48, 2),
+    ("block_size", 256, 2),
     ("top_k", 33, 2),
     ("top_k", 0, 1),
     ("head_dim", 96, 2),

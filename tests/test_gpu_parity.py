@@ -58,6 +58,10 @@ SMALL = {
     "d64_g4": Workload("d64_g4", 2, 700, 700, 0, 16, 4, 64, 64, 128, 5, "bf16", 1),
     "f32_d128_g8": Workload("f32_d128_g8", 1, 600, 600, 0, 16, 2, 128, 128, 128, 4, "f32", 0),
     "g32_di32": Workload("g32_di32", 1, 520, 520, 0, 64, 2, 128, 32, 128, 3, "bf16", 1),
+    # 64- and 32-token blocks (CUDA-core kernels): prefill chunk, decode rows, fp32
+    "bk64_chunk": Workload("bk64_chunk", 2, 300, 1000, 700, 16, 4, 64, 32, 64, 6, "bf16", 1),
+    "bk64_decode": Workload("bk64_decode", 4, 1, 2000, 1999, 64, 4, 128, 128, 64, 16, "bf16", 2),
+    "bk32_f32": Workload("bk32_f32", 1, 200, 500, 300, 8, 2, 64, 32, 32, 5, "f32", 0),
 }
 # larger cases checked on sampled rows
 SAMPLED = {
