@@ -198,9 +198,10 @@ msa_status_t msa_select_static(const msa_problem_t* p, const void* q_idx, const 
  * (no gradient reaches q or k).  q, k, q_idx, k_idx take the problem's dtypes
  * (qk_dtype, index_dtype).  Workspace: msa_workspace_size(p, MSA_OP_INDEX_KL).
  * q2k entries outside the row's visible blocks are skipped and flag the status
- * word (1), as in msa_attend.  Runs on CUDA cores; MSA_ERR_UNSUPPORTED when the
- * per-(row, group) working set (group heads x head_dim + 2 x top_k x 128
- * floats) exceeds 200 KB of shared memory.  Other errors as msa_attend. */
+ * word (1), as in msa_attend.  Runs on CUDA cores; MSA_ERR_UNSUPPORTED for block
+ * sizes other than 128 and when the per-(row, group) working set (group heads x
+ * head_dim + 2 x top_k x 128 floats) exceeds 200 KB of shared memory.  Other
+ * errors as msa_attend. */
 msa_status_t msa_index_kl(const msa_problem_t* p, const void* q, const void* k,
                           const void* q_idx, const void* k_idx, const int32_t* q2k,
                           float* loss, float* dq_idx, float* dk_idx, void* ws, size_t ws_bytes,

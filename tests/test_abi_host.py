@@ -234,3 +234,13 @@ def test_paged_problem_fields_reach_the_library(lib):
     assert msa.workspace_size(p, msa.OP_FORWARD) == msa.workspace_size(
         msa.problem_of(w), msa.OP_FORWARD)
     assert msa.launch_count(p) == msa.launch_count(msa.problem_of(w)) + 2  # table checks
+
+
+def test_index_kl_needs_128_token_blocks(lib):
+    w = workload.WORKLOADS["prefill_32k"].with_(block_size=64)
+    p = msa.problem_of(w)
+    assert msa.workspace_size(p, msa.OP_FORWARD) > 0       # the forward takes 64
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected before any launch
+    st = lib.msa_index_kl(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                          1 << 40, None)
+    assert st == 2
