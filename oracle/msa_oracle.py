@@ -52,6 +52,8 @@ design notes of the repository):
       over those tokens; the loss is the mean over all (row, group) pairs.
   R19 gradient detach: the teacher and the selection are constants; the
       gradients flow into q_idx and k_idx only.
+  R21 in a packed variable-length batch, a sequence's query rows are its last
+      tokens (chunked prefill and decode), and sequences are independent.
 
 Additional source for the KL-alignment loss:
   [DK]  section "Træning og stabilisering": Top-k is not differentiable, so an
@@ -360,6 +362,42 @@ def index_kl(q, k, q_idx, k_idx, q2k, q_pos0: int, block_size: int,
                 dq[b, i, g] = ds @ kis[J]
                 dk[b, J] += np.outer(ds, qi)
     return float(kl.sum() / N), dq, dk, kl
+
+
+# ---------------------------------------------------------------------------
+# Variable-length batches (packed sequences)
+# ---------------------------------------------------------------------------
+
+def forward_varlen(q, k, v, q_idx, k_idx, cu_q, cu_k, block_size: int, top_k: int,
+                   scale: Optional[float] = None):
+    """The forward pass over a packed batch of sequences of different lengths.
+
+    [HF] "原因分析" gives the selection the packed shape [total_qo_len, heads,
+    topk]: the query rows of all sequences are concatenated.  Sequence b owns
+    query rows cu_q[b] .. cu_q[b+1]-1 and key rows cu_k[b] .. cu_k[b+1]-1 of the
+    packed q [total_q, Hq, D], q_idx [total_q, Hkv, di], k, v [total_k, Hkv, D]
+    and k_idx [total_k, di].  Reading R21: a sequence's queries are its last
+    Sq_b = cu_q[b+1] - cu_q[b] tokens (position L_b - Sq_b + i for its i-th row,
+    L_b = cu_k[b+1] - cu_k[b]), as in chunked prefill and decode; sequences never
+    see one another.  Returns (out [total_q, Hq, D], lse [total_q, Hq],
+    q2k [Hkv, total_q, top_k]).
+    """
+    cu_q, cu_k = np.asarray(cu_q), np.asarray(cu_k)
+    total_q, Hq, D = np.shape(q)
+    Hkv = np.shape(k)[1]
+    out = np.empty((total_q, Hq, D))
+    lse = np.empty((total_q, Hq))
+    q2k = np.full((Hkv, total_q, top_k), -1, dtype=np.int64)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0:
+            continue
+        one = lambda x, lo, hi: np.asarray(x)[lo:hi][None]  # noqa: E731  (batch of one)
+        o, l, sel = forward(one(q, q0, q1), one(k, k0, k1), one(v, k0, k1),
+                            one(q_idx, q0, q1), one(k_idx, k0, k1), (k1 - k0) - (q1 - q0),
+                            block_size, top_k, scale)
+        out[q0:q1], lse[q0:q1], q2k[:, q0:q1] = o[0], l[0], sel
+    return out, lse, q2k
 
 
 # ---------------------------------------------------------------------------

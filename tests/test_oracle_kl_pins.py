@@ -1,4 +1,5 @@
-"""Pins of the oracle's KL-alignment loss (index-branch training side).
+"""Pins of the oracle's KL-alignment loss (index-branch training side), of its
+page gather (paged KV cache) and of its packed variable-length forward.
 
 The loss follows snilld.dk "Træning og stabilisering" (the index branch is
 trained to match the group-averaged main-branch distribution over the selected
@@ -137,3 +138,44 @@ def test_gather_pages_inverts_paging():
     got = O.gather_pages(pool, shared, L)
     np.testing.assert_array_equal(got[1, :128], kv[0, :128])
     np.testing.assert_array_equal(got[1, 128:], kv[1, 128:])
+
+
+def _packed(seed, lens_k, lens_q, Hq=4, Hkv=2, D=8, di=4):
+    rng = np.random.default_rng(seed)
+    tk, tq = sum(lens_k), sum(lens_q)
+    x = dict(q=rng.standard_normal((tq, Hq, D)), k=rng.standard_normal((tk, Hkv, D)),
+             v=rng.standard_normal((tk, Hkv, D)), q_idx=rng.standard_normal((tq, Hkv, di)),
+             k_idx=rng.standard_normal((tk, di)))
+    cu_k = np.concatenate([[0], np.cumsum(lens_k)])
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)])
+    return x, cu_q, cu_k
+
+
+def test_varlen_with_equal_lengths_is_the_fixed_length_batch():
+    x, cu_q, cu_k = _packed(9, [300, 300, 300], [5, 5, 5])
+    out, lse, q2k = O.forward_varlen(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], cu_q, cu_k,
+                                     BK, 2)
+    B = 3
+    o2, l2, s2 = O.forward(x["q"].reshape(B, 5, 4, 8), x["k"].reshape(B, 300, 2, 8),
+                           x["v"].reshape(B, 300, 2, 8), x["q_idx"].reshape(B, 5, 2, 4),
+                           x["k_idx"].reshape(B, 300, 4), 295, BK, 2)
+    np.testing.assert_array_equal(out, o2.reshape(15, 4, 8))
+    np.testing.assert_array_equal(lse, l2.reshape(15, 4))
+    np.testing.assert_array_equal(q2k, s2)
+
+
+def test_varlen_with_a_full_budget_is_dense_causal_attention_per_sequence():
+    # top_k * Bk covers every sequence, so each sequence is dense causal GQA over
+    # its own keys only (an empty sequence and a decode row included)
+    lens_k, lens_q = [300, 1, 129, 70, 0], [7, 1, 2, 70, 0]
+    x, cu_q, cu_k = _packed(10, lens_k, lens_q)
+    out, lse, _ = O.forward_varlen(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], cu_q, cu_k,
+                                   BK, 3)
+    for b in range(len(lens_k)):
+        if lens_q[b] == 0:
+            continue
+        q0, q1, k0, k1 = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]
+        do, dl = O.dense_causal_gqa(x["q"][q0:q1][None], x["k"][k0:k1][None],
+                                    x["v"][k0:k1][None], lens_k[b] - lens_q[b])
+        np.testing.assert_allclose(out[q0:q1], do[0], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse[q0:q1], dl[0], rtol=1e-12, atol=1e-12)
