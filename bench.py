@@ -302,7 +302,7 @@ def run_e2e(msa, w, xh, out_h, steps, warmup):
 NCU_TRAFFIC = {
     # stage: (workload, source file, git blob id, bytes per launch)
     "attn": ("prefill_128k", "block_sparse_gqa_04_b200/csrc/attn_tc.cu",
-             "729fb128e5a8f77393df5edeb0c7da843b81022e", 13698565888 + 34591706368),
+             "4cf3db49c1787f57a16d2863f4918a39892c64af", 13698565888 + 34591706368),
 }
 
 

@@ -5,10 +5,11 @@
 // swapped; snilld.dk "Hvad er MSA i praksis": every query head of a group
 // attends over the causally visible tokens of the group's selected blocks).
 //
-// Shapes: bf16, head_dim 128, 16 query heads per group, block 128.  The work is
+// Shapes: bf16 (or fp8 q/k), head_dim 128, 16 query heads per group, block 128.  The work is
 // the flat list of 128-row tiles that the block -> query lists define: a tile is
 // 8 gathered queries x 16 heads of one (sequence, group, query chunk, block).
-// One persistent CTA per SM takes a contiguous share of the tiles.  Per tile:
+// One persistent CTA per SM takes the tiles dealt to it in chunks of kChunk
+// consecutive tiles (block-cyclic over the CTAs).  Per tile:
 //   * TMA loads the block's K and V (128 keys x 128 dims each, 128-byte swizzle)
 //     into one of two buffers, once per list, and gathers the 8 queries' Q rows
 //     (16 heads x 128 dims, 4 KB contiguous in memory) with one box per query
