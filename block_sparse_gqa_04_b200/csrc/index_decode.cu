@@ -21,8 +21,9 @@
 //   * warps 2-5 (one TMEM lane quarter each) read their keys' N scores, mask
 //     the keys a row cannot see, reduce each column with a warp redux over
 //     orderable keys and combine the four warps' maxima through shared memory.
-// Persistent CTAs (two per SM for the 16-wide form) take contiguous ranges of
-// items, so consecutive items mostly share one sequence.
+// Persistent CTAs (two per SM for the bf16 16-wide form, three for fp8, whose
+// stages are half the size) take contiguous ranges of items, so consecutive
+// items mostly share one sequence.
 #include <cudaTypedefs.h>
 
 #include <algorithm>

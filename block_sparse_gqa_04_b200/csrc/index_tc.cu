@@ -5,10 +5,10 @@
 // 原因分析: amax over each block, per index head; snilld.dk "Hvad er MSA i
 // praksis": one index-query head per GQA group, one shared index-key head).
 //
-// Shapes: bf16, index_dim 128, block 128, up to 4 groups.  One persistent CTA
-// per SM walks a contiguous share of the (sequence, 128-row query tile, key
-// block) triples that the causal mask leaves (triangle order, so every CTA gets
-// the same number of tiles).  For each triple and each group one MMA unit
+// Shapes: bf16 or fp8 (e4m3) index tensors, index_dim 128, block 128, up to 4
+// groups.  One persistent CTA per SM walks a contiguous share of the (sequence,
+// 128-row query tile, key block) triples that the causal mask leaves, with the
+// query tiles in the balanced order of tile_at below.  For each triple and each group one MMA unit
 // computes S[128 queries x 128 keys] = q_idx_g . k_idx_block^T in fp32:
 //   * TMEM lanes are query rows.  The index queries of the current query tile
 //     (all groups, 128 x 128 bf16 each) sit in TMEM columns 0..255 as the A
