@@ -103,14 +103,16 @@ def _rows(batch: int, q_len: int, rows: Optional[Iterable[int]]) -> list:
 # Index branch
 # ---------------------------------------------------------------------------
 
-def index_scores_row(q_vec, k_idx_seq, t: int) -> np.ndarray:
+def index_scores_row(q_vecs, k_idx_seq, t: int) -> np.ndarray:
     """Token scores s_j = q_vec . k_idx_seq[j] for every visible key j = 0..t.
 
     [DK] "Hvad er MSA i praksis" and [HU] "Hogyan működik...": one index-query
     head per GQA group is scored against the single shared index-key head over
     the causally visible key tokens.  Reading R1: the raw dot product.
+    ``q_vecs`` is one index query [di] (result [t+1]) or the index queries of
+    all groups of a row [Hkv, di] (result [t+1, Hkv], column g = group g).
     """
-    return _f64(k_idx_seq)[: t + 1] @ _f64(q_vec)
+    return _f64(k_idx_seq)[: t + 1] @ _f64(q_vecs).T
 
 
 def block_maxima_row(scores: np.ndarray, block_size: int) -> np.ndarray:
@@ -166,8 +168,7 @@ def block_scores(q_idx, k_idx, q_pos0: int, block_size: int,
         t = q_pos0 + i
         if b != kb_of:  # widen one sequence's index keys at a time
             kb, kb_of = _f64(k_idx[b]), b
-        # all groups at once: [t+1, di] @ [di, Hkv]
-        s = kb[: t + 1] @ _f64(q_idx[b, i]).T
+        s = index_scores_row(q_idx[b, i], kb, t)  # all groups at once: [t+1, Hkv]
         for g in range(Hkv):
             m = block_maxima_row(s[:, g], block_size)
             out[g, n, : m.shape[0]] = m

@@ -63,6 +63,37 @@ def test_golden_block_maxima_and_selection():
         assert sel[r["group"], at].tolist() == r["selection"], r["why"]
 
 
+def test_golden_token_scores():
+    """index_scores_row on the hand-worked keys: the raw dot products of tokens
+    0..t, the token at t itself included and t+1 left out, for one group and
+    for all groups of a row at once."""
+    gd = _golden()
+    q_idx, k_idx = _golden_inputs(gd)
+    ts = gd["token_scores"]
+    t = ts["t"]
+    qg = np.array(gd["q_idx_groups"], dtype=np.float64)
+    assert O.index_scores_row(qg[1], k_idx[0], t).tolist() == ts["group1"]
+    both = O.index_scores_row(qg, k_idx[0], t)
+    assert both.shape == (t + 1, 2)
+    assert both[:, 0].tolist() == ts["group0"] and both[:, 1].tolist() == ts["group1"]
+
+
+def test_golden_selection_metrics():
+    """The [HF] 验证方法 metrics on a hand-worked 2-group x 3-row example."""
+    m = _golden()["selection_metrics"]
+    got = O.selection_metrics(np.array(m["a"]), np.array(m["b"]))
+    n = m["pairs"]
+    assert got["total"] == n
+    assert got["divergent"] == m["divergent"]
+    assert got["mean_overlap"] == pytest.approx(m["overlap_sum"] / n, abs=1e-15)
+    assert got["distinct_a"] == pytest.approx(m["distinct_a_sum"] / n, abs=1e-15)
+    assert got["distinct_b"] == pytest.approx(m["distinct_b_sum"] / n, abs=1e-15)
+    # swapping the sides swaps only the two distinct counts
+    rev = O.selection_metrics(np.array(m["b"]), np.array(m["a"]))
+    assert rev["distinct_a"] == got["distinct_b"] and rev["distinct_b"] == got["distinct_a"]
+    assert rev["divergent"] == got["divergent"] and rev["mean_overlap"] == got["mean_overlap"]
+
+
 def test_golden_attention_closed_forms():
     gd = _golden()
     Bk = gd["block_size"]
@@ -346,12 +377,15 @@ def _mut_local_outside_k(bm, t, Bk, k):
 
 
 MUTANTS = ["no_local", "tie_high", "local_outside_k", "maxpool_sees_future",
-           "gqa_modulo", "missing_causal_in_local", "scale_sqrt_di"]
+           "gqa_modulo", "missing_causal_in_local", "scale_sqrt_di", "scores_drop_token_t",
+           "scores_see_token_t1", "metrics_count_padding", "metrics_overlap_union",
+           "metrics_distinct_b_from_a"]
 
 
 def _run_pins(monkeypatch_ctx):
     """Run a fixed subset of pins; return True if all pass."""
     checks = [test_golden_block_maxima_and_selection, test_golden_attention_closed_forms,
+              test_golden_token_scores, test_golden_selection_metrics,
               lambda: test_selection_exhaustive_subsets(),
               lambda: test_full_budget_equals_dense_causal_gqa(200, 32, 7),
               lambda: test_dense_mask_formulation(),
@@ -370,6 +404,7 @@ def test_planted_mistakes_are_caught(mutant, monkeypatch):
     orig_bmax_row = O.block_maxima_row
     orig_attend_row = O.attend_row
     orig_attend = O.attend
+    orig_metrics = O.selection_metrics
     if mutant == "no_local":
         monkeypatch.setattr(O, "select_row", _mut_no_local)
     elif mutant == "tie_high":
@@ -420,10 +455,37 @@ def test_planted_mistakes_are_caught(mutant, monkeypatch):
             return orig_attend_row(q_heads, k_seq_g, v_seq_g, blocks,
                                    min(len(k_seq_g) - 1, (t // Bk + 1) * Bk - 1), Bk, scale)
         monkeypatch.setattr(O, "attend_row", ar)
+    elif mutant == "scores_drop_token_t":
+        # the slice stops one token short: the query's own token is not scored
+        monkeypatch.setattr(O, "index_scores_row",
+                            lambda q, k, t: O._f64(k)[:t] @ O._f64(q).T)
+    elif mutant == "scores_see_token_t1":
+        # the slice reaches one token past the query
+        monkeypatch.setattr(O, "index_scores_row",
+                            lambda q, k, t: O._f64(k)[: t + 2] @ O._f64(q).T)
+    elif mutant.startswith("metrics_"):
+        def met(sel_a, sel_b):
+            a, b = np.asarray(sel_a), np.asarray(sel_b)
+            Hkv, R, _ = a.shape
+            d = ov = da = db = 0
+            for g in range(Hkv):
+                for r in range(R):
+                    keep = (lambda x: True) if mutant == "metrics_count_padding" else \
+                        (lambda x: x >= 0)
+                    sa = set(int(x) for x in a[g, r] if keep(x))
+                    sb = set(int(x) for x in b[g, r] if keep(x))
+                    d += int(sa != sb)
+                    ov += len(sa | sb) if mutant == "metrics_overlap_union" else len(sa & sb)
+                    da += len(sa)
+                    db += len(sa) if mutant == "metrics_distinct_b_from_a" else len(sb)
+            n = Hkv * R
+            return {"divergent": d, "total": n, "mean_overlap": ov / n,
+                    "distinct_a": da / n, "distinct_b": db / n}
+        monkeypatch.setattr(O, "selection_metrics", met)
     elif mutant == "scale_sqrt_di":
         def att(q, k, v, q2k, q_pos0, Bk, scale=None, rows=None):
             return orig_attend(q, k, v, q2k, q_pos0, Bk, 1.0 / math.sqrt(2 * O._f64(q).shape[3]),
                                rows)
         monkeypatch.setattr(O, "attend", att)
     assert not _run_pins(monkeypatch), f"planted mistake '{mutant}' passed every pin"
-    assert orig_select_row is not None
+    assert orig_select_row is not None and orig_metrics is not None
