@@ -185,6 +185,12 @@ def _oracle_rows(task):
     return len(rows)
 
 
+def oracle_rows(w: Workload) -> int:
+    """Rows of the oracle sample: 4096 for the prefill workloads (a few seconds
+    of wall time on 16 host cores at 128K), every row when there are fewer."""
+    return min(w.rows, 4096)
+
+
 def time_oracle(w: Workload, x: dict, n_rows: int, seed: int = 0) -> dict:
     """Times the oracle forward on ``n_rows`` evenly spread rows with a spawn
     pool over all host cores and extrapolates to the whole workload."""
@@ -335,24 +341,29 @@ def tensor_seconds(cnt, bf16_tflops):
             "attn": half / (bf16_tflops * r_qk * 1e12) + half / (bf16_tflops * 1e12)}
 
 
-def kernel_roofline(w, cnt, stage_ms, path, peaks, kv_sel_bytes, sustained=True):
+def kernel_roofline(w, cnt, stage_ms, path, peaks, kv_sel_bytes):
     """Roofline entry of the slowest stage of the step.  A contraction's peak is
     its dtype's: the measured bf16 peak, times the nominal fp8 ratio for fp8
-    operands (the attention mixes an fp8 S with a bf16 P V when q/k are fp8)."""
+    operands (the attention mixes an fp8 S with a bf16 P V when q/k are fp8).
+    The step lasts well under a second, so `frac` divides by the burst peak;
+    `frac_sustained` gives the same against the seconds-long sustained peak."""
     name = max(stage_ms, key=stage_ms.get)
     ms = stage_ms[name]
-    tflops_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
-    t_peak = tensor_seconds(cnt, tflops_peak)
+    t_peak = tensor_seconds(cnt, peaks["bf16_tflops"])
+    t_sus = tensor_seconds(cnt, peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
     alu_peak = SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    peak_sus = None
     if name == "index":
         tc = "index:tc" in path
         bound, unit, work = ("tensor" if tc else "alu"), "TFLOP/s", cnt["index_flops"]
         peak = work / t_peak["index"] / 1e12 if tc else alu_peak
+        peak_sus = work / t_sus["index"] / 1e12 if tc else None
         achieved = work / (ms * 1e-3) / 1e12
     elif name == "attn":
         tc = "attn:tc" in path
         bound, unit, work = ("tensor" if tc else "alu"), "TFLOP/s", cnt["main_flops"]
         peak = work / t_peak["attn"] / 1e12 if tc else alu_peak
+        peak_sus = work / t_sus["attn"] / 1e12 if tc else None
         achieved = work / (ms * 1e-3) / 1e12
     else:
         bound, unit = "hbm", "GB/s"
@@ -361,15 +372,19 @@ def kernel_roofline(w, cnt, stage_ms, path, peaks, kv_sel_bytes, sustained=True)
                 "combine": cnt["partial_bytes"] + cnt["out_bytes"] + cnt["q2k_bytes"]}[name]
         peak = peaks["hbm_gbs"]
         achieved = work / (ms * 1e-3) / 1e9
-    return {"kernel": name, "bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 2),
-            "unit": unit, "frac": round(achieved / peak, 4),
-            "traffic": measured_traffic(name, w.name),
-            "ms": round(ms, 4), "algorithmic_per_launch": work,
-            "peak_kind": ("sustained" + (" bf16 x 2 for fp8 operands" if
-                                         (cnt["index_fp8"] or cnt["qk_fp8"]) else ""))
-                         if (bound == "tensor" and sustained) else
-                         ("derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock" if bound == "alu"
-                          else "measured")}
+    res = {"kernel": name, "bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 2),
+           "unit": unit, "frac": round(achieved / peak, 4),
+           "traffic": measured_traffic(name, w.name),
+           "ms": round(ms, 4), "algorithmic_per_launch": work,
+           "peak_kind": ("measured burst bf16" + (" (x 2 for fp8 operands)" if
+                                                   (cnt["index_fp8"] or cnt["qk_fp8"]) else ""))
+                        if bound == "tensor" else
+                        ("derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock" if bound == "alu"
+                         else "measured copy bandwidth")}
+    if peak_sus:
+        res["frac_sustained"] = round(achieved / peak_sus, 4)
+        res["peak_sustained"] = round(peak_sus, 2)
+    return res
 
 
 def path_roofline(cnt, kv_sel_bytes, ms, peaks):
@@ -563,6 +578,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the prefill_32k and chunk_1m lines beside the headline")
     ap.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows (0 = auto)")
     ap.add_argument("--seq", type=int, default=0,
                     help="prefill length override (a smaller case of the same structure, "
@@ -607,8 +624,9 @@ def main():
             return
         dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
         x = make_inputs(w, seed=0, device=dev)
-        n_rows = a.cpu_rows or (64 if w.q_len > 1 else w.rows)
-        vals = [time_oracle(w, x, n_rows, seed=s) for s in range(a.warmup + a.steps)]
+        n_rows = a.cpu_rows or oracle_rows(w)
+        # every step times the same evenly spread rows as the cpu_baseline leg
+        vals = [time_oracle(w, x, n_rows) for _ in range(a.warmup + a.steps)]
         timed = vals[a.warmup:]
         v = statistics.mean(t["value"] for t in timed)
         ms = w.rows / v * 1e3
@@ -681,12 +699,30 @@ def main():
             "clocks": dres["clocks"]}
         dres.pop("x")
         x_main = None
+    extra_names = [] if (a.no_extra or a.seq or a.batch or a.index_kl) else \
+        [n for n in ("prefill_32k", "chunk_1m") if n != a.workload]
+    for name in extra_names:
+        # the other large workloads, each timed the same way (steps, warm-up,
+        # CUDA events, max over ranks) and reported beside the headline
+        we = WORKLOADS[name]
+        we = we.with_(name=we.name + suffix, index_dtype=a.index_dtype, qk_dtype=a.qk_dtype)
+        torch.cuda.empty_cache()
+        eres = measure_workload(msa, we, dev, a.steps, a.warmup, peaks, False, paged=a.paged)
+        eval_, ems = weak_value(we.rows, eres["ms"], world)
+        line[name] = {
+            "workload": we.name, "value": eval_, "unit": "query-tokens/s",
+            "ms_per_step": ems, "kernel_path": eres["path"],
+            "stage_ms": {k: round(v, 4) for k, v in eres["stage"].items()},
+            "roofline": kernel_roofline(we, eres["cnt"], eres["stage"], eres["path"], peaks,
+                                        eres["kv_sel"]),
+            "path_roofline": path_roofline(eres["cnt"], eres["kv_sel"], ems, peaks),
+            "gpu_launches": eres["launches"], "clocks": eres["clocks"]}
+        eres.pop("x")
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         # the oracle runs on host copies of the bench's own inputs
         xm = make_inputs(w, seed=0, device=dev)
         xm.pop("needles")
-        n_rows = a.cpu_rows or 8192  # about 10-20 s of oracle work on 16 cores
-        line["cpu_baseline"] = time_oracle(w, xm, n_rows)
+        line["cpu_baseline"] = time_oracle(w, xm, a.cpu_rows or oracle_rows(w))
     if rank == 0:
         print(json.dumps(line), flush=True)
     barrier(world)

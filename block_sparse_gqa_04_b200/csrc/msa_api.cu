@@ -120,10 +120,13 @@ Layout layout(const Problem& P, int op) {
 
 msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
-// Optional stage events (msa_set_stage_events).
+// Optional stage events (msa_set_stage_events).  Every entry point restarts
+// the numbering (stage_begin) so that each call records its own stages.
 cudaEvent_t const* g_events = nullptr;
 int g_nevents = 0;
 int g_next = 0;
+
+void stage_begin() { g_next = 0; }
 
 void stage_mark(cudaStream_t s) {
   if (g_events && g_next < g_nevents) cudaEventRecord(g_events[g_next++], s);
@@ -218,6 +221,7 @@ msa_status_t msa_select(const msa_problem_t* p, const void* q_idx, const void* k
   if (P.T == 0) return MSA_OK;
   if (cudaMemsetAsync(ws, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess)
     return MSA_ERR_CUDA;
+  stage_begin();
   return run_select(P, q_idx, k_idx, q2k, block_scores_opt, ws, (cudaStream_t)stream);
 }
 
@@ -236,6 +240,7 @@ msa_status_t msa_attend(const msa_problem_t* p, const void* q, const void* k, co
   if (P.T == 0) return MSA_OK;
   if (cudaMemsetAsync(ws, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess)
     return MSA_ERR_CUDA;
+  stage_begin();
   return run_attend(P, q, k, v, q2k, out, lse_opt, ws, layout(P, MSA_OP_ATTEND),
                     (cudaStream_t)stream);
 }
@@ -257,6 +262,7 @@ msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, c
   const Layout L = layout(P, MSA_OP_FORWARD);
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(ws, 0, sizeof(int32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  stage_begin();
   int32_t* q2k = q2k_opt ? q2k_opt : at<int32_t>(ws, L.q2k);
   // the select stage only needs the status word and bmax, which sit at the same
   // offsets in the forward layout

@@ -74,10 +74,11 @@ __device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false if
-// the wait gave up (kWaitLimit polls) or *abort became non-zero.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+// the wait gave up (`limit` polls, kWaitLimit unless a test passes a smaller
+// one) or *abort became non-zero.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t limit = kWaitLimit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_test(bar, parity)) return true;
     if (i >= 64) {
       if (*abort) return false;
@@ -90,8 +91,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 // Spins on the non-blocking test: for a thread that issues MMAs, whose pipe
 // runs dry while the thread waits (a try_wait costs ~200 cycles even when the
 // phase has already completed).  Bounded like mbar_wait.
-__device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+__device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t limit = kWaitLimit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_poll(bar, parity)) return true;
     if ((i & 1023) == 1023 && *abort) return false;
   }

@@ -27,7 +27,8 @@ STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 
 EXPORTED = ("msa_workspace_size", "msa_select", "msa_attend", "msa_forward",
             "msa_device_status", "msa_set_stage_events", "msa_launch_count", "msa_kernel_path",
-            "msa_status_string", "msa_select_static", "msa_index_kl")
+            "msa_status_string", "msa_select_static", "msa_index_kl",
+            "msa_selftest_wait_timeout")
 STAGES = ("index", "topk", "lists", "attn", "combine")
 
 
@@ -84,6 +85,8 @@ def load() -> ctypes.CDLL:
         lib.msa_select_static.restype = i32
         lib.msa_index_kl.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.msa_index_kl.restype = i32
+        lib.msa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, vp, vp]
+        lib.msa_selftest_wait_timeout.restype = i32
         _lib = lib
     return _lib
 
@@ -214,17 +217,34 @@ def _paged(block_table, kv_len, batch, num_pages, block_size):
     return {"num_pages": int(num_pages), "block_table": block_table}
 
 
+def _check_index_pair(q_idx: torch.Tensor, k_idx: torch.Tensor, paged: bool = False) -> int:
+    """q_idx [B, Sq, Hkv, di] and k_idx [B, Skv, di] (paged: [pages, 128, di])
+    of one dtype: the index kernels read k_idx with q_idx's element size and
+    batch, so a mismatch would read past the end of k_idx.  Returns Skv (the
+    rows per page for a paged cache)."""
+    if q_idx.dim() != 4:
+        raise ValueError(f"q_idx must be [B, Sq, Hkv, di], got {tuple(q_idx.shape)}")
+    B, _, _, di = q_idx.shape
+    if k_idx.dim() != 3 or k_idx.shape[2] != di or (
+            k_idx.shape[1] != 128 if paged else k_idx.shape[0] != B):
+        want = "[pages, 128, di]" if paged else f"[{B}, Skv, {di}]"
+        raise ValueError(f"k_idx has shape {tuple(k_idx.shape)}, expected {want}")
+    if k_idx.dtype != q_idx.dtype:
+        raise ValueError(f"q_idx and k_idx dtypes differ: {q_idx.dtype} vs {k_idx.dtype}")
+    return int(k_idx.shape[1])
+
+
 def select(q_idx: torch.Tensor, k_idx: torch.Tensor, *, q_pos0: int = 0, block_size: int = 128,
            top_k: int = 16, return_block_scores: bool = False,
            workspace: Optional[torch.Tensor] = None, block_table=None, kv_len=None):
     """Index branch: returns q2k [Hkv, B*Sq, top_k] int32 (and block scores).
     With block_table and kv_len, k_idx is a paged cache [pages, 128, di]."""
+    Skv = _check_index_pair(q_idx, k_idx, paged=block_table is not None)
     _require_cuda(q_idx, k_idx)
     B, Sq, Hkv, di = q_idx.shape
-    Skv = k_idx.shape[1] if block_table is None else int(kv_len)
+    if block_table is not None:
+        Skv = int(kv_len) if kv_len is not None else None
     pg = _paged(block_table, kv_len, B, k_idx.shape[0], block_size)
-    if tuple(k_idx.shape) != ((k_idx.shape[0], 128, di) if pg else (B, Skv, di)):
-        raise ValueError(f"k_idx has shape {tuple(k_idx.shape)}")
     p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, top_k, q_idx.dtype, q_pos0,
                      index_dtype=q_idx.dtype, **pg)
     dev = q_idx.device
@@ -247,9 +267,9 @@ def select_static(q_idx: torch.Tensor, k_idx: torch.Tensor, q2k: torch.Tensor, *
     one-element int32 device tensor that receives the device status word).
     For callers that cannot lend the library device memory; the library's
     fixed scratch is shared, so calls must not overlap on the GPU."""
+    Skv = _check_index_pair(q_idx, k_idx)
     _require_cuda(q_idx, k_idx, q2k, device_status)
     B, Sq, Hkv, di = q_idx.shape
-    Skv = k_idx.shape[1]
     if q2k.dtype != torch.int32 or tuple(q2k.shape[:2]) != (Hkv, B * Sq):
         raise ValueError("q2k must be int32 [Hkv, B*Sq, top_k]")
     if device_status is not None and device_status.dtype != torch.int32:
@@ -310,6 +330,7 @@ def index_kl(q, k, q_idx, k_idx, q2k, *, q_pos0: int = 0, block_size: int = 128,
     tensor, and its fp32 gradients shaped like q_idx and k_idx (with a paged
     cache, dk_idx is shaped like the k_idx page pool).
     """
+    _check_index_pair(q_idx, k_idx, paged=block_table is not None)
     _require_cuda(q, k, q_idx, k_idx, q2k)
     B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx, k_idx=k_idx, kv_len=kv_len)
     pg = _paged(block_table, kv_len, B, k.shape[0], block_size)
@@ -336,6 +357,18 @@ def index_kl(q, k, q_idx, k_idx, q2k, *, q_pos0: int = 0, block_size: int = 128,
     return loss, dq, dk
 
 
+def selftest_wait_timeout(limit: int, device=None):
+    """Runs the library's bounded-wait exit on purpose (msa_selftest_wait_timeout)
+    and returns (status word, number of warps that gave up) after a sync."""
+    dev = torch.device(device or "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    gave_up = torch.zeros(1, dtype=torch.int32, device=dev)
+    _check(load().msa_selftest_wait_timeout(int(limit), _ptr(status), _ptr(gave_up),
+                                            _stream(dev)), "msa_selftest_wait_timeout")
+    torch.cuda.synchronize(dev)
+    return int(status.item()), int(gave_up.item())
+
+
 def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, top_k: int = 16,
             softmax_scale: float = 0.0, return_lse: bool = False, return_q2k: bool = False,
             workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
@@ -349,6 +382,7 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
     ceil(kv_len/128)] int32, on the device) and kv_len, k, v and k_idx are a paged
     KV cache: [pages, 128, Hkv, D] and [pages, 128, di].
     """
+    _check_index_pair(q_idx, k_idx, paged=block_table is not None)
     host = not q.is_cuda
     if host:
         dev = torch.device(device or "cuda")

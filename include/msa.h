@@ -175,8 +175,13 @@ msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, c
  *    serialised by the caller.
  *  - Each call clears the status word first (the only scratch that must start
  *    at zero).  device_status_opt: optional device int32; if not NULL it
- *    receives, in stream order, the call's status word (0 = fine; 2 = a bounded
- *    wait inside a tensor-core kernel gave up).
+ *    receives, in stream order, the call's status word, a bitmask as in
+ *    msa_device_status (0 = fine).
+ *  - The buffer's address is cached per device index for the life of the
+ *    process: it assumes one CUDA context per device.  After cudaDeviceReset
+ *    (or anything else that tears down and recreates the device's primary
+ *    context) the cached address is stale; do not call this entry point
+ *    again in that process.
  * Other arguments and errors as msa_select. */
 msa_status_t msa_select_static(const msa_problem_t* p, const void* q_idx, const void* k_idx,
                                int32_t* q2k, int32_t* device_status_opt, void* stream);
@@ -208,19 +213,25 @@ msa_status_t msa_index_kl(const msa_problem_t* p, const void* q, const void* k,
                           void* stream);
 
 /* Reads the workspace status word written by the last call that used `ws`:
- * waits for `stream`, stores the device code (0 = fine) in *code and returns
- * MSA_OK, or MSA_ERR_DEVICE if the code is not 0.  This call synchronises. */
+ * waits for `stream`, stores the device code in *code and returns MSA_OK if it
+ * is 0, else MSA_ERR_DEVICE.  The code is a bitmask (an OR of every problem the
+ * call's kernels met): 1 = a q2k entry outside the row's visible blocks
+ * (skipped), 2 = a bounded wait inside a tensor-core kernel gave up (the
+ * kernel's output is incomplete), 4 = a block_table page id outside
+ * [0, num_pages) (read as page 0).  This call synchronises. */
 msa_status_t msa_device_status(const void* ws, int32_t* code, void* stream);
 
 /* Stage timing (a measurement aid, not part of the method).  When `events` is
- * not NULL, every later call records events[i] (cudaEvent_t values) on its
- * stream right after its i-th stage, for i < n, so the caller can time each
- * kernel with cudaEventElapsedTime against an event recorded before the call.
- * Stages of msa_forward in order: 0 index scores, 1 top-k select, 2 block ->
- * query lists (four small kernels), 3 KV-outer attention, 4 combine;
- * msa_select records 0-1 and msa_attend 2-4 (numbered from 0 within the call).
- * The setting is process-wide and not thread-safe; NULL turns it off.
- * Returns the number of stages of msa_forward. */
+ * not NULL, every later call of msa_select, msa_attend or msa_forward records
+ * events[i] (cudaEvent_t values) on its stream right after its i-th stage, for
+ * i < n, so the caller can time each kernel with cudaEventElapsedTime against
+ * an event recorded before the call; each call numbers its stages from 0, so
+ * the same events are recorded again by the next call.  Stages of msa_forward
+ * in order: 0 index scores, 1 top-k select, 2 block -> query lists (a few small
+ * kernels), 3 KV-outer attention, 4 combine; msa_select records its stages 0-1
+ * and msa_attend its stages 0-2 (lists, attention, combine).  The setting is
+ * process-wide and not thread-safe; NULL turns it off.  Returns the number of
+ * stages of msa_forward. */
 int32_t msa_set_stage_events(void* const* events, int32_t n);
 
 /* Number of kernel launches one call of `op` makes for problem `p` (without
@@ -230,6 +241,20 @@ int32_t msa_launch_count(const msa_problem_t* p, int32_t op);
 /* Which kernel family a call of `op` runs for `p`: a static string naming the
  * index-branch and main-branch kernels ("tc" = tcgen05/TMA path, "simt"). */
 const char* msa_kernel_path(const msa_problem_t* p, int32_t op);
+
+/* Self-test of the bounded waits (a diagnostic, not part of the method).
+ * Every wait of the tensor-core kernels gives up after a fixed number of polls,
+ * raises an abort flag, ORs bit 2 into the status word and returns after
+ * freeing its TMEM, so that a wait that can never end leaves the GPU usable.
+ * This entry point runs that exit on purpose: one small CTA holds TMEM, waits
+ * on an mbarrier nothing arrives on (the MMA thread's spin and the other warps'
+ * sleeping wait) with `limit` polls (1 .. 2^24), gives up, ORs 2 into *status
+ * (device int32) and adds 1 to *gave_up (device int32) per giving-up warp, 3 in
+ * all.  It issues no copy and no MMA, so nothing is in flight when it exits.
+ * Enqueued on `stream`; MSA_ERR_INVALID_ARG for null or misaligned pointers or
+ * a limit out of range. */
+msa_status_t msa_selftest_wait_timeout(uint32_t limit, int32_t* status, int32_t* gave_up,
+                                       void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* msa_status_string(msa_status_t s);

@@ -244,3 +244,38 @@ def test_index_kl_needs_128_token_blocks(lib):
     st = lib.msa_index_kl(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, fake,
                           1 << 40, None)
     assert st == 2
+
+
+def test_index_pair_shape_and_dtype_are_checked_before_the_device():
+    """select, select_static, forward and index_kl reject a k_idx whose batch,
+    index dim or dtype disagrees with q_idx: the index kernels read k_idx with
+    q_idx's batch and element size, so such a call would read past its end.
+    Tensors of the right shapes get as far as the CUDA check."""
+    B, Sq, Skv, Hq, Hkv, D, di = 2, 4, 300, 16, 2, 128, 32
+    bf = torch.bfloat16
+    q = torch.zeros((B, Sq, Hq, D), dtype=bf)
+    k = torch.zeros((B, Skv, Hkv, D), dtype=bf)
+    qi = torch.zeros((B, Sq, Hkv, di), dtype=bf)
+    ki = torch.zeros((B, Skv, di), dtype=bf)
+    q2k = torch.zeros((Hkv, B * Sq, 4), dtype=torch.int32)
+    bad = {"batch": torch.zeros((1, Skv, di), dtype=bf),
+           "index dim": torch.zeros((B, Skv, di // 2), dtype=bf),
+           "rank": torch.zeros((B, Skv, 1, di), dtype=bf),
+           "dtype": torch.zeros((B, Skv, di), dtype=torch.float8_e4m3fn)}
+    calls = {
+        "select": lambda kk: msa.select(qi, kk),
+        "select_static": lambda kk: msa.select_static(qi, kk, q2k),
+        "forward": lambda kk: msa.forward(q, k, k, qi, kk),
+        "index_kl": lambda kk: msa.index_kl(q, k, qi, kk, q2k),
+    }
+    for name, call in calls.items():
+        for why, kk in bad.items():
+            with pytest.raises(ValueError, match="k_idx|dtypes differ"):
+                call(kk)
+        if name != "forward":   # host tensors: forward copies them, others stop here
+            with pytest.raises(ValueError, match="CUDA"):
+                call(ki)
+    # a paged k_idx pool is [pages, 128, di]
+    with pytest.raises(ValueError, match="k_idx"):
+        msa._check_index_pair(qi, torch.zeros((7, 64, di), dtype=bf), paged=True)
+    assert msa._check_index_pair(qi, torch.zeros((7, 128, di), dtype=bf), paged=True) == 128
