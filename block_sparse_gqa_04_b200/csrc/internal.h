@@ -38,6 +38,8 @@ struct Problem {
 
 // Shape checks of the C ABI: fills *P from *p or returns why it cannot.
 msa_status_t resolve_problem(const msa_problem_t* p, Problem* P);
+// MSA_OK for cudaSuccess, else MSA_ERR_CUDA with `e` kept for msa_last_cuda_error.
+msa_status_t status_of(cudaError_t e);
 
 // Views into the caller's workspace.
 struct Lists {

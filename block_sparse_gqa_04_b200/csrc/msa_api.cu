@@ -118,7 +118,14 @@ Layout layout(const Problem& P, int op) {
   return L;
 }
 
-msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+// The CUDA error behind the last MSA_ERR_CUDA of this thread (msa_last_cuda_error).
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+msa_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MSA_OK;
+  g_last_cuda_error = e;
+  return MSA_ERR_CUDA;
+}
 
 // Optional stage events (msa_set_stage_events).  Every entry point restarts
 // the numbering (stage_begin) so that each call records its own stages.
@@ -196,6 +203,7 @@ msa_status_t run_attend(const Problem& P, const void* q, const void* k, const vo
 
 namespace msa {
 msa_status_t resolve_problem(const msa_problem_t* p, Problem* P) { return resolve(p, P); }
+msa_status_t status_of(cudaError_t e) { return cuda_status(e); }
 }  // namespace msa
 
 extern "C" {
@@ -219,8 +227,8 @@ msa_status_t msa_select(const msa_problem_t* p, const void* q_idx, const void* k
     return MSA_ERR_INVALID_ARG;
   if ((st = check_ws(P, MSA_OP_SELECT, ws, ws_bytes)) != MSA_OK) return st;
   if (P.T == 0) return MSA_OK;
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess)
-    return MSA_ERR_CUDA;
+  if (msa_status_t cst = cuda_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), (cudaStream_t)stream)))
+    return cst;
   stage_begin();
   return run_select(P, q_idx, k_idx, q2k, block_scores_opt, ws, (cudaStream_t)stream);
 }
@@ -238,8 +246,8 @@ msa_status_t msa_attend(const msa_problem_t* p, const void* q, const void* k, co
     return MSA_ERR_INVALID_ARG;
   if ((st = check_ws(P, MSA_OP_ATTEND, ws, ws_bytes)) != MSA_OK) return st;
   if (P.T == 0) return MSA_OK;
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess)
-    return MSA_ERR_CUDA;
+  if (msa_status_t cst = cuda_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), (cudaStream_t)stream)))
+    return cst;
   stage_begin();
   return run_attend(P, q, k, v, q2k, out, lse_opt, ws, layout(P, MSA_OP_ATTEND),
                     (cudaStream_t)stream);
@@ -261,7 +269,7 @@ msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, c
   if (P.T == 0) return MSA_OK;
   const Layout L = layout(P, MSA_OP_FORWARD);
   cudaStream_t s = (cudaStream_t)stream;
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  if (msa_status_t cst = cuda_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), s))) return cst;
   stage_begin();
   int32_t* q2k = q2k_opt ? q2k_opt : at<int32_t>(ws, L.q2k);
   // the select stage only needs the status word and bmax, which sit at the same
@@ -289,7 +297,7 @@ msa_status_t msa_index_kl(const msa_problem_t* p, const void* q, const void* k,
   if ((st = check_ws(P, MSA_OP_INDEX_KL, ws, ws_bytes)) != MSA_OK) return st;
   const Layout L = layout(P, MSA_OP_INDEX_KL);
   cudaStream_t s = (cudaStream_t)stream;
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), s) != cudaSuccess) return MSA_ERR_CUDA;
+  if (msa_status_t cst = cuda_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), s))) return cst;
   msa::Lists lists{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.cursor),
                    at<int32_t>(ws, L.list_off), at<int32_t>(ws, L.tile_off),
                    at<int32_t>(ws, L.entries), at<int32_t>(ws, L.pos), nullptr,
@@ -307,9 +315,10 @@ msa_status_t msa_device_status(const void* ws, int32_t* code, void* stream) {
   if (!ws || !code) return MSA_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   int32_t h = 0;
-  if (cudaMemcpyAsync(&h, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return MSA_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return MSA_ERR_CUDA;
+  if (msa_status_t cst = cuda_status(cudaMemcpyAsync(&h, ws, sizeof(int32_t),
+                                                     cudaMemcpyDeviceToHost, s)))
+    return cst;
+  if (msa_status_t cst = cuda_status(cudaStreamSynchronize(s))) return cst;
   *code = h;
   return h == 0 ? MSA_OK : MSA_ERR_DEVICE;
 }
@@ -356,6 +365,11 @@ const char* msa_kernel_path(const msa_problem_t* p, int32_t op) {
     case MSA_OP_INDEX_KL: return "kl:simt";
   }
   return "invalid";
+}
+
+const char* msa_last_cuda_error(int32_t* code_opt) {
+  if (code_opt) *code_opt = int32_t(g_last_cuda_error);
+  return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
 }
 
 const char* msa_status_string(msa_status_t s) {

@@ -70,7 +70,7 @@ extern "C" msa_status_t msa_select_static(const msa_problem_t* p, const void* q_
   if (bmax_bytes > kMaxBmaxBytes) return MSA_ERR_TOO_LARGE;
 
   void* scratch = nullptr;
-  if (scratch_on_current_device(&scratch) != cudaSuccess) return MSA_ERR_CUDA;
+  if (msa_status_t cst = msa::status_of(scratch_on_current_device(&scratch))) return cst;
   int32_t* status = static_cast<int32_t*>(scratch);
   float* bmax = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kStatusBytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -84,5 +84,5 @@ extern "C" msa_status_t msa_select_static(const msa_problem_t* p, const void* q_
   if (e == cudaSuccess) e = msa::launch_topk(P, bmax, q2k, s);
   if (e == cudaSuccess && device_status_opt)
     e = cudaMemcpyAsync(device_status_opt, status, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
-  return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+  return msa::status_of(e);
 }

@@ -64,5 +64,5 @@ extern "C" msa_status_t msa_selftest_wait_timeout(uint32_t limit, int32_t* statu
     return MSA_ERR_INVALID_ARG;
   msa::wait_timeout_kernel<<<1, 128, 0, static_cast<cudaStream_t>(stream)>>>(limit, status,
                                                                               gave_up);
-  return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+  return msa::status_of(cudaGetLastError());
 }

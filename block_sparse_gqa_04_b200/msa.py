@@ -28,13 +28,17 @@ STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 EXPORTED = ("msa_workspace_size", "msa_select", "msa_attend", "msa_forward",
             "msa_device_status", "msa_set_stage_events", "msa_launch_count", "msa_kernel_path",
             "msa_status_string", "msa_select_static", "msa_index_kl",
-            "msa_selftest_wait_timeout")
+            "msa_selftest_wait_timeout", "msa_last_cuda_error")
 STAGES = ("index", "topk", "lists", "attn", "combine")
 
 
 class MsaError(RuntimeError):
     def __init__(self, code: int, where: str):
-        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        msg = f"{where}: {STATUS.get(code, code)}"
+        if code == 4 and _lib is not None:  # the CUDA error behind MSA_ERR_CUDA
+            c = ctypes.c_int32(0)
+            msg += f" ({_lib.msa_last_cuda_error(ctypes.byref(c)).decode()}, cudaError {c.value})"
+        super().__init__(msg)
         self.code = code
 
 
@@ -87,6 +91,8 @@ def load() -> ctypes.CDLL:
         lib.msa_index_kl.restype = i32
         lib.msa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, vp, vp]
         lib.msa_selftest_wait_timeout.restype = i32
+        lib.msa_last_cuda_error.argtypes = [ctypes.POINTER(i32)]
+        lib.msa_last_cuda_error.restype = ctypes.c_char_p
         _lib = lib
     return _lib
 

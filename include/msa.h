@@ -256,6 +256,11 @@ const char* msa_kernel_path(const msa_problem_t* p, int32_t op);
 msa_status_t msa_selftest_wait_timeout(uint32_t limit, int32_t* status, int32_t* gave_up,
                                        void* stream);
 
+/* The CUDA error behind the last MSA_ERR_CUDA returned to the calling thread:
+ * its cudaError_t value in *code_opt (if not NULL; 0 = none yet) and its
+ * description (static storage). */
+const char* msa_last_cuda_error(int32_t* code_opt);
+
 /* Human-readable name of a status code (static storage). */
 const char* msa_status_string(msa_status_t s);
 
