@@ -92,6 +92,7 @@ struct Bars {
   uint64_t s_full[2], p_full[2], o_full[2], buf_empty[2];
   uint64_t d_full[kDesc], d_empty[kDesc];
   TileDesc desc[kDesc];
+  uint64_t mma_done;       // the MMA thread's final commit (drain before TMEM is freed)
   uint32_t tmem_base;
   int abort;
 };
@@ -216,6 +217,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       tc::mbar_init(&bars->d_full[d], 1);
       tc::mbar_init(&bars->d_empty[d], 5);  // the MMA thread and the four softmax warps
     }
+    tc::mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     tc::fence_mbar_init();
   }
@@ -245,6 +247,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     int kv_stage = 0, q_stage = 0;
     uint32_t kv_phase = 0, q_phase = 0;
     int prev_lid = -1;
+    tc::ArmedRing q_armed, kv_armed;  // lane 0: copies issued into each ring
     auto fetch = [&](int j, TileRec& r) -> bool {
       const long long tile = tile_of(j);
       if (tile >= total) return false;
@@ -286,6 +289,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             if (good) {
               uint64_t* fb = &bars->kv_full[kv_stage];
               tc::mbar_arrive_expect_tx(fb, C::kKVBytes);
+              kv_armed.note(kv_stage, kv_phase);
               uint8_t* dst = kvbuf + kv_stage * C::kKVBytes;
               const int key0 = int(block_row(P, tb, tc_));
               tc::tma_load_3d(dst, &tmap_k, fb, 0, tg, key0);  // fp8: all 128 dims
@@ -295,7 +299,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
           }
           good = good && tc::mbar_wait(&bars->q_empty[q_stage], q_phase ^ 1, abort);
-          if (good) tc::mbar_arrive_expect_tx(&bars->q_full[q_stage], uint32_t(tn) * C::kQBox);
+          if (good) {
+            tc::mbar_arrive_expect_tx(&bars->q_full[q_stage], uint32_t(tn) * C::kQBox);
+            q_armed.note(q_stage, q_phase);
+          }
         }
         // the Q boxes of the tile, issued together: lane e copies query e
         if (__shfl_sync(MSA_FULL_MASK, good, 0) && lane < tn) {
@@ -339,6 +346,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       cur = nxt;
       cur_ok = nxt_ok;
     }
+    // every copy issued has landed before the CTA can leave (on the abort path
+    // too: the copies complete whether or not anyone consumes them)
+    if (lane == 0 && !(q_armed.drain(bars->q_full) && kv_armed.drain(bars->kv_full))) failed = true;
     if (lane != 0) failed = false;  // lane 0 speaks for the warp
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -418,13 +428,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
           }
         }
+        // the idle loop polls without sleeping: a sleep delays the issue of the
+        // next MMA group by up to its length while the pipe runs dry
         if (progress) {
           idle = 0;
-        } else {
-          if (++idle > tc::kWaitLimit || (idle > 64 && *abort)) { failed = true; break; }
-          if (idle > 8) __nanosleep(20);
+        } else if (++idle > tc::kWaitLimit || (idle > 64 && *abort)) {
+          failed = true;
+          break;
         }
       }
+      // every MMA issued has completed before TMEM is freed
+      if (!tc::mma_drain(&bars->mma_done)) failed = true;
     }
   } else {
     // ---------------- softmax + epilogue (two warpgroups) ----------------

@@ -195,6 +195,7 @@ combine_tma_kernel(Problem P, const int32_t* __restrict__ pos,
   if (warp == 8) {
     // ---------------- loader ----------------
     int k = 0;
+    tc::ArmedRing armed;  // lane 0: stages it has armed for copies
     for (long long u = blockIdx.x; u < units && !failed; u += gridDim.x) {
       const int32_t* ps = pos + u * P.K;              // pos[g][r][:] with u = g * T + r
       for (int b = 0; b < nb; ++b, ++k) {
@@ -209,6 +210,7 @@ combine_tma_kernel(Problem P, const int32_t* __restrict__ pos,
         if (lane == 0) {
           bars->mask[st] = m;
           tc::mbar_arrive_expect_tx(&bars->full[st], __popc(m) * (kCSlotBytes + kCLseBytes));
+          armed.note(st, (k / kCStages) & 1);
         }
         __syncwarp();
         if (e >= 0) {
@@ -227,6 +229,9 @@ combine_tma_kernel(Problem P, const int32_t* __restrict__ pos,
         }
       }
     }
+    // every copy issued has landed before the CTA can leave
+    if (lane == 0 && !armed.drain(bars->full)) failed = true;
+    if (lane != 0) failed = false;
   } else {
     // ---------------- merge: thread = (head hh, 16-byte chunk ch) ----------------
     const int hh = threadIdx.x >> 4, ch = threadIdx.x & 15;

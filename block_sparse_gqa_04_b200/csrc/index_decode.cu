@@ -67,6 +67,7 @@ struct Shared {
   uint64_t acc_full[kSlots], acc_empty[kSlots];
   uint32_t red[kSlots][4][N];   // per accumulator: the four warps' column maxima
   int qseq[Cfg<N, FP8>::kStages];  // sequence whose queries each stage holds (-1: none)
+  uint64_t mma_done;       // the MMA thread's final commit (drain before TMEM is freed)
   uint32_t tmem_base;
   int abort;
 };
@@ -131,6 +132,7 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       tc::mbar_init(&sh->acc_full[s], 1);
       tc::mbar_init(&sh->acc_empty[s], 4);
     }
+    tc::mbar_init(&sh->mma_done, 1);
     sh->abort = 0;
     tc::fence_mbar_init();
   }
@@ -152,6 +154,7 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
     uint4 qv[kQv];
     int qb = -1;
     int k = 0;
+    tc::ArmedRing armed;  // lane 0: stages whose k_idx copy it issued
     for (long long it = i0; it < i1; ++it, ++k) {
       const int s = k % S;
       const uint32_t ph = (k / S) & 1;
@@ -172,6 +175,7 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       uint8_t* st = stages + s * C::kStageBytes;
       if (lane == 0) {
         tc::mbar_arrive_expect_tx(&sh->full[s], C::kKBytes);
+        armed.note(s, ph);
         const int row = int(block_row(P, b, c));
         tc::tma_load_2d(st, &tmap_k, &sh->full[s], 0, row);
         if (!FP8) tc::tma_load_2d(st + kKHalf, &tmap_k, &sh->full[s], 64, row);
@@ -198,6 +202,10 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
         tc::mbar_arrive(&sh->full[s]);
       }
     }
+    // every copy issued has landed before the CTA can leave (each armed stage
+    // also got the second arrival, right after its copy was issued)
+    if (lane == 0 && !armed.drain(sh->full)) failed = true;
+    if (lane != 0) failed = false;
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -225,6 +233,8 @@ index_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
         tc::mma_commit(&sh->acc_full[slot]);
         tc::mma_commit(&sh->empty[s]);
       }
+      // every MMA issued has completed before TMEM is freed
+      if (!tc::mma_drain(&sh->mma_done)) failed = true;
     }
   } else {
     // ---------------- epilogue: masked column maxima ----------------

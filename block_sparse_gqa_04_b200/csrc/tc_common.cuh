@@ -100,6 +100,37 @@ __device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, volati
   return false;
 }
 
+// Bounded wait that ignores the abort flag: a CTA that gives up drains the work
+// it has already started (TMA copies landing in its shared memory, MMAs
+// writing its TMEM) before it frees TMEM and exits.  Returns false only if the
+// phase did not complete within kWaitLimit polls.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_test(bar, parity)) return true;
+    if (i >= 64) __nanosleep(64);
+  }
+  return false;
+}
+
+// The full barriers of a ring that a producer thread has armed (arrive with an
+// expected transaction count, then copies that complete it): which ones, and
+// the parity of each one's last armed phase.  drain() waits for those phases,
+// i.e. until every copy the thread issued into the ring has landed; a phase
+// that the consumer already saw complete returns at once.
+struct ArmedRing {
+  uint32_t armed = 0, parity = 0;
+  __device__ __forceinline__ void note(int s, uint32_t phase) {
+    armed |= 1u << s;
+    parity = (parity & ~(1u << s)) | ((phase & 1u) << s);
+  }
+  __device__ __forceinline__ bool drain(uint64_t* full) const {
+    bool ok = true;
+    for (int s = 0; s < 32; ++s)
+      if ((armed >> s) & 1u) ok = mbar_drain(&full[s], (parity >> s) & 1u) && ok;
+    return ok;
+  }
+};
+
 // ---------------------------------------------------------------------------
 // TMA
 // ---------------------------------------------------------------------------
@@ -242,6 +273,15 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_addr(bar))
       : "memory");
+}
+
+// Waits (bounded, abort flag ignored) until every MMA this thread issued has
+// completed, through `bar`, a barrier initialised with count 1 and used for
+// nothing else (phase 0).  Called by the MMA-issuing thread before TMEM is
+// freed, on the normal and the abort path alike.
+__device__ __forceinline__ bool mma_drain(uint64_t* bar) {
+  mma_commit(bar);
+  return mbar_drain(bar, 0);
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread i gets lane (base+i).
