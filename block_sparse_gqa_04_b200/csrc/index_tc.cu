@@ -23,6 +23,18 @@
 // thread: masked max over the row's 128 columns, one fp32 store per unit).
 // The epilogue is two warpgroups, one per accumulator, so that two units drain
 // at once while the tensor cores fill the next.
+//
+// Streaming selection (FUSE): instead of writing the block maxima, each
+// epilogue thread keeps, for each group its warpgroup drains, the top (k-1)
+// keys (orderable score, lower id on ties) of the earlier blocks c < floor(t/Bk)
+// of its query row, as a min-heap in shared memory with its root in registers
+// ("MiniMax lancerer MSA" (snilld.dk), section "Teknisk forklaring hvorfor
+// kompleksiteten skifter": the top-k over raw block scores is where the gain
+// can be lost, so the block scores never make an HBM round trip).  A query
+// tile's blocks may be split between the contiguous shares of neighbouring
+// CTAs; each CTA writes its partial list for the tile to its own slot, and
+// select_merge_kernel takes the top (k-1) over the tile's slots, adds the
+// local block and writes the ascending selection.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -39,6 +51,9 @@ constexpr int kThreads = 320;               // TMA, MMA, two epilogue warpgroups
 constexpr int kMaxGroups = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 256;           // accumulators follow the A region
+constexpr int kEpiThreads = 256;            // the two epilogue warpgroups
+constexpr int kMaxKeep = 15;                // streaming selection: top_k - 1 <= 15
+constexpr size_t kListBytes = size_t(2) * kMaxKeep * kEpiThreads * 8;  // two groups per thread
 
 // Element type of the index tensors: bf16 (kind::f16, two 64-dim halves per key
 // row) or fp8 e4m3 (kind::f8f6f4, one 128-byte half, half the bytes).
@@ -52,6 +67,7 @@ struct Idx {
   static constexpr uint32_t kIdesc =
       FP8 ? tc::idesc_e4m3_f32(128, 128) : tc::idesc_bf16_f32(128, 128, 0, 0);
   static constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + 256;
+  static constexpr size_t kSmemBytesFused = kSmemBytes + kListBytes;
 };
 
 // Blocks query tile m (128 rows) of a sequence can see.
@@ -116,6 +132,25 @@ struct Walk {
   }
 };
 
+// The CTA whose contiguous share of the pair index contains pair L, for shares
+// [total*x/grid, total*(x+1)/grid) (the largest x with total*x/grid <= L).
+__host__ __device__ inline int cta_of_pair(long long L, long long total, int grid) {
+  return int(((L + 1) * grid + total - 1) / total) - 1;
+}
+
+// Position of query tile m in the order of tile_at.
+__host__ __device__ inline int order_of_tile(const Problem& P, int m) {
+  const int M = mtiles(P);
+  return m < (M + 1) / 2 ? 2 * m : 2 * (M - 1 - m) + 1;
+}
+
+// Slots of partial selection lists per (group, row): the most CTA shares one
+// query tile's pairs can be split into.
+inline int select_slots(const Problem& P, long long total, int grid) {
+  const long long share = total / grid;  // >= 1: grid <= total
+  return int((P.nblk + share - 1) / share) + 1;
+}
+
 struct Bars {
   uint64_t full[kStages];
   uint64_t empty[kStages];
@@ -123,21 +158,25 @@ struct Bars {
   uint64_t acc_empty[2];
   uint64_t a_full;
   uint64_t a_empty;
+  uint64_t mma_done;       // the MMA thread's final commit (drain before TMEM is freed)
   uint32_t tmem_base;
   int abort;
 };
 
-template <bool FP8>
+template <bool FP8, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1)
 index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
                 const uint8_t* __restrict__ q_idx, float* __restrict__ bmax,
-                int* __restrict__ status, long long per_seq) {
+                uint64_t* __restrict__ cand, int nslot, int* __restrict__ status,
+                long long per_seq) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
   using X = Idx<FP8>;
   Bars* bars = reinterpret_cast<Bars*>(smem + kStages * X::kStageBytes);
+  // FUSE: kept keys, [group of the warpgroup][entry][epilogue thread]
+  uint64_t* keep = reinterpret_cast<uint64_t*>(smem + kStages * X::kStageBytes + 256);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -152,6 +191,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
     }
     tc::mbar_init(&bars->a_full, 8);
     tc::mbar_init(&bars->a_empty, 1);
+    tc::mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     tc::fence_mbar_init();
   }
@@ -174,9 +214,11 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       w.start(P, L0, per_seq);
       int stage = 0;
       uint32_t phase = 0;
+      tc::ArmedRing armed;
       for (long long L = L0; L < L1; ++L) {
         if (!tc::mbar_wait(&bars->empty[stage], phase ^ 1, abort)) { failed = true; break; }
         tc::mbar_arrive_expect_tx(&bars->full[stage], X::kStageBytes);
+        armed.note(stage, phase);
         const int row = int(block_row(P, w.b, w.c));
         uint8_t* dst = stages + stage * X::kStageBytes;
         tc::tma_load_2d(dst, &tmap_k, &bars->full[stage], 0, row);
@@ -184,6 +226,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
         if (++stage == kStages) { stage = 0; phase ^= 1; }
         w.next(P);
       }
+      // every copy issued has landed before the CTA can leave
+      if (!armed.drain(bars->full)) failed = true;
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -229,6 +273,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
         seg_start = w.next(P);
         if (seg_start || L + 1 == L1) tc::mma_commit(&bars->a_empty);
       }
+      // every MMA issued has completed before TMEM is freed
+      if (!tc::mma_drain(&bars->mma_done)) failed = true;
     }
   } else {
     // ---------------- index-query loader + epilogue (two warpgroups) ----------------
@@ -236,6 +282,12 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
     const int quarter = warp & 3;           // TMEM lanes this warp may touch
     const int row = quarter * 32 + lane;    // query row inside the tile
     const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+    const int et = threadIdx.x - 64;        // epilogue thread: the keep lists' column
+    const int nkeep = P.K - 1;
+    // per group of this warpgroup (g = ewg + 2j): number of kept keys, the
+    // smallest of them (0 while fewer than nkeep are kept)
+    int cnt0 = 0, cnt1 = 0;
+    uint64_t mkey0 = 0, mkey1 = 0;
     if (L0 < L1) {
       Walk w;
       w.start(P, L0, per_seq);
@@ -280,7 +332,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
           if (lane == 0) tc::mbar_arrive(&bars->a_full);
         }
         const long long t = P.q_pos0 + i;
-        const long long lim = t - (long long)w.c * P.Bk;  // last visible column
+        const long long lim = t - (long long)w.c * 128;   // last visible column (Bk = 128)
+        const bool earlier = w.c < int(t >> 7);             // c < floor(t / 128)
         for (int g = 0; g < P.Hkv; ++g, ++k) {
           if ((k & 1) != ewg) continue;     // the other warpgroup's unit
           const uint32_t par = (k >> 1) & 1;
@@ -313,7 +366,69 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
           }
           const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-          if (valid) bmax[((long long)g * P.T + r) * P.nblk + w.c] = m;
+          if (!FUSE) {
+            if (valid) bmax[((long long)g * P.T + r) * P.nblk + w.c] = m;
+          } else if (valid && earlier && nkeep > 0) {
+            // an earlier block of this row (c < floor(t/Bk)): keep its key if
+            // it is among the nkeep largest so far
+            const int j = g >> 1;
+            uint64_t* kl = keep + size_t(j) * kMaxKeep * kEpiThreads + et;
+            const uint64_t key = block_key(m, w.c);
+            // the kept keys form a binary min-heap (root = smallest kept key,
+            // also held in mkey): filling sifts a key up, replacing the root
+            // sifts the new key down, at most log2(16) levels either way
+            auto offer = [&](int& cnt, uint64_t& mkey) {
+              int pos;
+              if (cnt < nkeep) {
+                pos = cnt++;
+                while (pos > 0) {
+                  const int up = (pos - 1) >> 1;
+                  const uint64_t pk = kl[up * kEpiThreads];
+                  if (pk <= key) break;
+                  kl[pos * kEpiThreads] = pk;
+                  pos = up;
+                }
+              } else if (key > mkey) {
+                pos = 0;
+                for (;;) {
+                  const int l = 2 * pos + 1;
+                  if (l >= nkeep) break;
+                  uint64_t ck = kl[l * kEpiThreads];
+                  int c2 = l;
+                  if (l + 1 < nkeep) {
+                    const uint64_t rk = kl[(l + 1) * kEpiThreads];
+                    if (rk < ck) { ck = rk; c2 = l + 1; }
+                  }
+                  if (ck >= key) break;
+                  kl[pos * kEpiThreads] = ck;
+                  pos = c2;
+                }
+              } else {
+                return;
+              }
+              kl[pos * kEpiThreads] = key;
+              mkey = cnt < nkeep ? 0 : kl[0];
+            };
+            if (j == 0) offer(cnt0, mkey0);
+            else offer(cnt1, mkey1);
+          }
+        }
+        if (FUSE && nkeep > 0 && (w.c + 1 == w.nc || L + 1 == L1)) {
+          // end of this CTA's share of the query tile: its partial lists go to
+          // the CTA's slot among the tile's shares (unused entries are 0, below
+          // every key)
+          if (valid) {
+            const long long T0 = (long long)w.b * per_seq + pairs_before_at(P, w.u, per_seq);
+            const int slot = int(blockIdx.x) - cta_of_pair(T0, per_seq * P.B, gridDim.x);
+            for (int j = 0; 2 * j + ewg < P.Hkv; ++j) {
+              const int g = 2 * j + ewg;
+              const int cnt = j ? cnt1 : cnt0;
+              const uint64_t* kl = keep + size_t(j) * kMaxKeep * kEpiThreads + et;
+              uint64_t* dst = cand + ((size_t(g) * nslot + slot) * nkeep) * P.T + r;
+              for (int e = 0; e < nkeep; ++e) dst[size_t(e) * P.T] = e < cnt ? kl[e * kEpiThreads] : 0;
+            }
+          }
+          cnt0 = cnt1 = 0;
         }
         seg_start = w.next(P);
       }
@@ -328,6 +443,72 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Final selection from the partial lists, one thread per (group, row): the
+// top (k-1) keys over the slots of the row's query tile (each slot holds the
+// top (k-1) of one CTA's share of the tile's blocks, so their union holds the
+// row's top (k-1)), then the local block; ids ascending, -1 padded.
+__global__ void __launch_bounds__(256) select_merge_kernel(Problem P,
+                                                           const uint64_t* __restrict__ cand,
+                                                           int nslot, long long per_seq, int grid,
+                                                           int32_t* __restrict__ q2k) {
+  const long long n = (long long)P.Hkv * P.T;
+  const long long total = per_seq * P.B;
+  const int nkeep = P.K - 1;
+  for (long long id = blockIdx.x * (long long)blockDim.x + threadIdx.x; id < n;
+       id += (long long)gridDim.x * blockDim.x) {
+    const int g = int(id / P.T), r = int(id % P.T);
+    const int b = r / P.Sq, i = r % P.Sq;
+    const long long t = P.q_pos0 + i;
+    const int c_t = int(t / P.Bk);
+    const int need = min(P.K, c_t + 1) - 1;  // earlier blocks to keep
+    // keys kept so far, largest first (0 = none)
+    uint64_t top[kMaxKeep];
+#pragma unroll
+    for (int e = 0; e < kMaxKeep; ++e) top[e] = 0;
+    if (need > 0) {
+      const int m = i / 128;
+      const long long T0 = (long long)b * per_seq + pairs_before_at(P, order_of_tile(P, m), per_seq);
+      const int x0 = cta_of_pair(T0, total, grid);
+      const int x1 = cta_of_pair(T0 + tile_blocks(P, m) - 1, total, grid);
+      for (int sl = 0; sl <= x1 - x0; ++sl) {
+        const uint64_t* src = cand + ((size_t(g) * nslot + sl) * nkeep) * P.T + r;
+        for (int e = 0; e < nkeep; ++e) {
+          uint64_t x = src[size_t(e) * P.T];
+          if (x > top[kMaxKeep - 1]) {
+            // insertion into the descending list (branch-free exchange chain)
+#pragma unroll
+            for (int q = 0; q < kMaxKeep; ++q) {
+              const uint64_t hi = x > top[q] ? x : top[q];
+              x = x > top[q] ? top[q] : x;
+              top[q] = hi;
+            }
+          }
+        }
+      }
+    }
+    // the kept block ids (INT_MAX past `need`), sorted ascending by an
+    // odd-even transposition network; every kept id is below c_t
+    int id16[kMaxKeep];
+#pragma unroll
+    for (int e = 0; e < kMaxKeep; ++e) id16[e] = e < need ? key_block(top[e]) : INT_MAX;
+#pragma unroll
+    for (int round = 0; round < kMaxKeep; ++round) {
+#pragma unroll
+      for (int e = round & 1; e + 1 < kMaxKeep; e += 2) {
+        const int lo = min(id16[e], id16[e + 1]), hi = max(id16[e], id16[e + 1]);
+        id16[e] = lo;
+        id16[e + 1] = hi;
+      }
+    }
+    int32_t* out = q2k + ((long long)g * P.T + r) * P.K;
+#pragma unroll
+    for (int e = 0; e < kMaxKeep + 1; ++e) {
+      if (e >= P.K) break;
+      out[e] = e < need ? id16[e] : (e == need ? c_t : -1);
+    }
   }
 }
 
@@ -362,15 +543,35 @@ bool index_tc_supported(const Problem& P) {
          P.kv_rows < (1LL << 31);
 }
 
-template <bool FP8>
-static cudaError_t launch_t(const Problem& P, const void* q_idx, const void* k_idx, float* bmax,
-                           int32_t* status, cudaStream_t s) {
+bool index_select_fused_supported(const Problem& P) {
+  return index_tc_supported(P) && P.K - 1 <= kMaxKeep && (P.Hkv == 2 || P.Hkv == 4);
+}
+
+namespace {
+
+struct Split {
+  long long per_seq, total;
+  int grid, nslot;
+};
+
+Split split_of(const Problem& P) {
+  Split sp;
+  sp.per_seq = pairs_per_seq(P);
+  sp.total = sp.per_seq * P.B;
+  sp.grid = int(std::min<long long>(sm_count(), sp.total));
+  sp.nslot = select_slots(P, sp.total, sp.grid);
+  return sp;
+}
+
+template <bool FP8, bool FUSE>
+cudaError_t launch_t(const Problem& P, const void* q_idx, const void* k_idx, float* bmax,
+                     uint64_t* cand, int32_t* status, cudaStream_t s) {
   using X = Idx<FP8>;
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   // k_idx rows of 128 dims, copied as 128-byte-wide boxes of 128 keys (128-byte swizzle)
   CUtensorMap map;
-  cuuint64_t dims[2] = {FP8 ? 128u : 128u, cuuint64_t(P.kv_rows)};
+  cuuint64_t dims[2] = {128u, cuuint64_t(P.kv_rows)};
   cuuint64_t strides[1] = {cuuint64_t(X::kRowBytes)};
   cuuint32_t box[2] = {FP8 ? 128u : 64u, 128};
   cuuint32_t estr[2] = {1, 1};
@@ -379,22 +580,44 @@ static cudaError_t launch_t(const Problem& P, const void* q_idx, const void* k_i
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  const long long per_seq = pairs_per_seq(P);
-  const long long total = per_seq * P.B;
-  const int grid = int(std::min<long long>(sm_count(), total));
-  cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<FP8>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(X::kSmemBytes));
+  const Split sp = split_of(P);
+  const size_t smem = FUSE ? X::kSmemBytesFused : X::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<FP8, FUSE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  index_tc_kernel<FP8><<<grid, kThreads, X::kSmemBytes, s>>>(
-      map, P, static_cast<const uint8_t*>(q_idx), bmax, status, per_seq);
+  index_tc_kernel<FP8, FUSE><<<sp.grid, kThreads, smem, s>>>(
+      map, P, static_cast<const uint8_t*>(q_idx), bmax, cand, sp.nslot, status, sp.per_seq);
   return cudaGetLastError();
 }
 
+}  // namespace
+
 cudaError_t launch_index_tc(const Problem& P, const void* q_idx, const void* k_idx,
                             float* bmax, int32_t* status, cudaStream_t s) {
-  return P.idx8 ? launch_t<true>(P, q_idx, k_idx, bmax, status, s)
-                : launch_t<false>(P, q_idx, k_idx, bmax, status, s);
+  return P.idx8 ? launch_t<true, false>(P, q_idx, k_idx, bmax, nullptr, status, s)
+                : launch_t<false, false>(P, q_idx, k_idx, bmax, nullptr, status, s);
+}
+
+size_t index_select_cand_bytes(const Problem& P) {
+  const Split sp = split_of(P);
+  return size_t(P.Hkv) * sp.nslot * std::max(1, P.K - 1) * size_t(P.T) * sizeof(uint64_t);
+}
+
+cudaError_t launch_index_select(const Problem& P, const void* q_idx, const void* k_idx,
+                                void* cand, int32_t* status, cudaStream_t s) {
+  uint64_t* c = static_cast<uint64_t*>(cand);
+  return P.idx8 ? launch_t<true, true>(P, q_idx, k_idx, nullptr, c, status, s)
+                : launch_t<false, true>(P, q_idx, k_idx, nullptr, c, status, s);
+}
+
+cudaError_t launch_select_merge(const Problem& P, const void* cand, int32_t* q2k,
+                                cudaStream_t s) {
+  const Split sp = split_of(P);
+  const long long n = (long long)P.Hkv * P.T;
+  const unsigned blocks = unsigned(std::min<long long>((n + 255) / 256, 148LL * 16));
+  select_merge_kernel<<<blocks, 256, 0, s>>>(P, static_cast<const uint64_t*>(cand), sp.nslot,
+                                              sp.per_seq, sp.grid, q2k);
+  return cudaGetLastError();
 }
 
 }  // namespace msa

@@ -87,6 +87,16 @@ cudaError_t launch_index_simt(const Problem& P, const void* q_idx, const void* k
 bool index_tc_supported(const Problem& P);
 cudaError_t launch_index_tc(const Problem& P, const void* q_idx, const void* k_idx,
                             float* bmax, int32_t* status, cudaStream_t s);
+// Selection fused into the tcgen05 index kernel (no block maxima in HBM): the
+// index kernel leaves partial top (k-1) lists per (group, row) in `cand`
+// (index_select_cand_bytes), and the merge kernel writes q2k.  For index_tc
+// problems with top_k <= 16 and 2 or 4 groups.
+bool index_select_fused_supported(const Problem& P);
+size_t index_select_cand_bytes(const Problem& P);
+cudaError_t launch_index_select(const Problem& P, const void* q_idx, const void* k_idx,
+                                void* cand, int32_t* status, cudaStream_t s);
+cudaError_t launch_select_merge(const Problem& P, const void* cand, int32_t* q2k,
+                                cudaStream_t s);
 // Block maxima for a few query rows per sequence (decode): a TMA-fed stream over
 // k_idx (bf16, index_dim 128).
 bool index_decode_supported(const Problem& P);

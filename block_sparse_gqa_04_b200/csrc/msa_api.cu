@@ -93,7 +93,12 @@ Layout layout(const Problem& P, int op) {
   const bool sel = op == MSA_OP_SELECT || op == MSA_OP_FORWARD;
   const bool att = op == MSA_OP_ATTEND || op == MSA_OP_FORWARD;
   const bool kl = op == MSA_OP_INDEX_KL;
-  L.bmax = sel ? take(size_t(P.Hkv) * T * P.nblk * sizeof(float)) : 0;
+  // the index branch's scratch: partial selection lists when the selection is
+  // fused into the index kernel, else the block maxima
+  L.bmax = sel ? take(msa::index_select_fused_supported(P)
+                          ? msa::index_select_cand_bytes(P)
+                          : size_t(P.Hkv) * T * P.nblk * sizeof(float))
+               : 0;
   L.q2k = op == MSA_OP_FORWARD ? take(size_t(P.Hkv) * T * P.K * sizeof(int32_t)) : 0;
   if (att || kl) {
     L.counts = take(size_t(P.nlists) * 4);
@@ -153,6 +158,19 @@ msa_status_t run_select(const Problem& P, const void* q_idx, const void* k_idx, 
   const Layout L = layout(P, MSA_OP_SELECT);
   float* bmax = bscores ? bscores : at<float>(ws, L.bmax);
   cudaError_t e = msa::launch_check_table(P, at<int32_t>(ws, L.status), s);
+  if (!bscores && msa::index_select_fused_supported(P)) {
+    // selection streamed inside the index kernel, then a merge of the partial lists
+    if (e == cudaSuccess) {
+      e = msa::launch_index_select(P, q_idx, k_idx, at<void>(ws, L.bmax),
+                                   at<int32_t>(ws, L.status), s);
+      stage_mark(s);
+    }
+    if (e == cudaSuccess) {
+      e = msa::launch_select_merge(P, at<void>(ws, L.bmax), q2k, s);
+      stage_mark(s);
+    }
+    return cuda_status(e);
+  }
   if (bscores && e == cudaSuccess)
     e = msa::launch_fill(bscores, size_t(P.Hkv) * P.T * P.nblk, -INFINITY, s);
   if (e == cudaSuccess) {
