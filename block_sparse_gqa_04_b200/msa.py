@@ -375,6 +375,84 @@ def selftest_wait_timeout(limit: int, device=None):
     return int(status.item()), int(gave_up.item())
 
 
+# Per device: the streams that carry host -> device and device -> host copies of
+# forward calls made with host tensors, so that copies overlap the kernels.
+_copy_streams = {}
+
+
+def _copy_stream_pair(dev: torch.device):
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    if key not in _copy_streams:
+        _copy_streams[key] = (torch.cuda.Stream(key), torch.cuda.Stream(key))
+    return _copy_streams[key]
+
+
+def host_output_stream(device=None) -> torch.cuda.Stream:
+    """The stream that carries the output copies of forward calls with host
+    tensors and a pinned host ``out`` (wait on it to order work after them)."""
+    return _copy_stream_pair(torch.device(device or "cuda"))[1]
+
+
+def wait_host_outputs(device=None) -> None:
+    """Waits until the output copies of every earlier forward call with host
+    tensors and a pinned host ``out`` have landed."""
+    dev = torch.device(device or "cuda")
+    _copy_stream_pair(dev)[1].synchronize()
+
+
+def _forward_host(q, k, v, q_idx, k_idx, block_table, out, dev, kw, ret_lse, ret_q2k):
+    """forward() on host tensors.  The index tensors are copied first, on a copy
+    stream, and the index branch starts as soon as they have landed, while q, k
+    and v are still on their way; the main branch waits for those.  With a
+    pinned ``out`` the result is copied back on a second copy stream and the
+    call returns without waiting, so that the output copy of one call overlaps
+    the input copy and the kernels of the next (PCIe carries both directions at
+    once); ``torch.cuda.synchronize()`` or :func:`wait_host_outputs` completes
+    it.  Otherwise the result is returned as a new host tensor."""
+    comp = torch.cuda.current_stream(dev)
+    h2d, d2h = _copy_stream_pair(dev)
+    nb = q.is_pinned()
+    with torch.cuda.stream(h2d):
+        qi_d, ki_d = q_idx.to(dev, non_blocking=nb), k_idx.to(dev, non_blocking=nb)
+        bt_d = block_table.to(dev, non_blocking=nb) if block_table is not None else None
+        ev_idx = torch.cuda.Event()
+        ev_idx.record(h2d)
+        q_d, k_d, v_d = (t.to(dev, non_blocking=nb) for t in (q, k, v))
+        ev_qkv = torch.cuda.Event()
+        ev_qkv.record(h2d)
+    # the buffers were allocated on the copy stream and are used on this one
+    for t in (qi_d, ki_d, q_d, k_d, v_d) + ((bt_d,) if bt_d is not None else ()):
+        t.record_stream(comp)
+    pg = dict(block_table=bt_d, kv_len=kw.pop("kv_len"))
+    comp.wait_event(ev_idx)
+    q2k = select(qi_d, ki_d, q_pos0=kw["q_pos0"], block_size=kw["block_size"],
+                 top_k=kw["top_k"], **pg)
+    comp.wait_event(ev_qkv)
+    o = attend(q_d, k_d, v_d, q2k, return_lse=ret_lse, check_device_status=kw["check"],
+               q_pos0=kw["q_pos0"], block_size=kw["block_size"],
+               softmax_scale=kw["softmax_scale"], **pg)
+    o, lse = o if ret_lse else (o, None)
+    if out is not None and out.is_pinned():
+        ev_done = torch.cuda.Event()
+        ev_done.record(comp)
+        d2h.wait_event(ev_done)
+        o.record_stream(d2h)
+        with torch.cuda.stream(d2h):
+            out.copy_(o, non_blocking=True)
+        o = out
+    elif out is not None:
+        out.copy_(o)
+        o = out
+    else:
+        o = o.cpu()
+    res = (o,)
+    if ret_lse:
+        res += (lse.cpu(),)
+    if ret_q2k:
+        res += (q2k.cpu(),)
+    return res[0] if len(res) == 1 else res
+
+
 def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, top_k: int = 16,
             softmax_scale: float = 0.0, return_lse: bool = False, return_q2k: bool = False,
             workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
@@ -382,20 +460,28 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
     """Index branch + main branch.  Returns out (and lse, q2k when asked).
 
     CUDA tensors are used in place.  Host tensors (ideally pinned) are copied to
-    ``device`` (default ``cuda``) before the call and the results copied back.
-    ``check_device_status`` waits for the call and raises if the device
-    recorded a problem (a bounded wait that gave up).  With block_table ([B,
-    ceil(kv_len/128)] int32, on the device) and kv_len, k, v and k_idx are a paged
-    KV cache: [pages, 128, Hkv, D] and [pages, 128, di].
+    ``device`` (default ``cuda``) and the results copied back, overlapped with
+    the kernels (see :func:`_forward_host`; with a pinned host ``out`` the call
+    returns before the output has landed).  ``check_device_status`` waits for
+    the call and raises if the device recorded a problem (a bounded wait that
+    gave up).  With block_table ([B, ceil(kv_len/128)] int32) and kv_len, k, v
+    and k_idx are a paged KV cache: [pages, 128, Hkv, D] and [pages, 128, di].
     """
     _check_index_pair(q_idx, k_idx, paged=block_table is not None)
-    host = not q.is_cuda
-    if host:
-        dev = torch.device(device or "cuda")
-        nb = q.is_pinned()
-        q, k, v, q_idx, k_idx = (t.to(dev, non_blocking=nb) for t in (q, k, v, q_idx, k_idx))
-        if block_table is not None:
-            block_table = block_table.to(dev, non_blocking=nb)
+    if not q.is_cuda:
+        for t in (k, v, q_idx, k_idx):
+            if t.is_cuda:
+                raise ValueError("forward takes all tensors on the host or all on the device")
+        if out is not None and (out.is_cuda or out.dtype != v.dtype or
+                                tuple(out.shape) != tuple(q.shape) or not out.is_contiguous()):
+            raise ValueError("with host inputs, out must be a contiguous host tensor shaped "
+                             "like q with v's dtype")
+        _dims(q, k, q_idx, v=v, k_idx=k_idx, kv_len=kv_len)
+        _check_qkv_dtypes(q, k, v)
+        kw = dict(q_pos0=q_pos0, block_size=block_size, top_k=top_k, kv_len=kv_len,
+                  softmax_scale=softmax_scale, check=check_device_status)
+        return _forward_host(q, k, v, q_idx, k_idx, block_table, out,
+                             torch.device(device or "cuda"), kw, return_lse, return_q2k)
     _require_cuda(q, k, v, q_idx, k_idx)
     B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx, v=v, k_idx=k_idx, kv_len=kv_len)
     pg = _paged(block_table, kv_len, B, k.shape[0], block_size)
@@ -407,7 +493,7 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
     p = make_problem(B, Sq, Skv, Hq, Hkv, D, di, block_size, top_k, v.dtype, q_pos0,
                      softmax_scale, index_dtype=q_idx.dtype, qk_dtype=q.dtype, **pg)
     dev = q.device
-    o = out if (out is not None and not host) else torch.empty(q.shape, dtype=v.dtype, device=dev)
+    o = out if out is not None else torch.empty(q.shape, dtype=v.dtype, device=dev)
     lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=dev) if return_lse else None
     q2k = (torch.empty((Hkv, B * Sq, top_k), dtype=torch.int32, device=dev)
            if return_q2k else None)
@@ -420,14 +506,6 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
         code = ctypes.c_int32(0)
         _check(load().msa_device_status(ctypes.c_void_p(wp), ctypes.byref(code), _stream(dev)),
                "msa_forward (device status)")
-    if host:
-        if out is not None:
-            out.copy_(o, non_blocking=out.is_pinned())
-            o = out
-        else:
-            o = o.cpu()
-        lse = None if lse is None else lse.cpu()
-        q2k = None if q2k is None else q2k.cpu()
     res = (o,)
     if return_lse:
         res += (lse,)

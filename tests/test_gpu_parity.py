@@ -239,3 +239,25 @@ def test_named_workload_full_size(name):
     assert dec > 0 and agree == dec
     _cache.clear()
     torch.cuda.empty_cache()
+
+
+def test_host_buffers_pipelined_calls():
+    """Consecutive calls with pinned host buffers and a pinned host out: each
+    call returns before its output copy has landed, so one call's output copy
+    overlaps the next call's input copy; after the copy stream is drained every
+    output equals the device result, and lse / q2k come back too."""
+    w = SMALL["chunk_unaligned"]
+    cpu, gpu = _inputs(w)
+    dev_out, dev_lse, dev_q2k = _run_forward(w, gpu)
+    host = {k: v.cpu().pin_memory() for k, v in gpu.items()}
+    outs = [torch.empty(dev_out.shape, dtype=dev_out.dtype).pin_memory() for _ in range(3)]
+    for o in outs:
+        msa.forward(host["q"], host["k"], host["v"], host["q_idx"], host["k_idx"],
+                    q_pos0=w.q_pos0, top_k=w.top_k, out=o)
+    msa.wait_host_outputs()
+    for o in outs:
+        assert torch.equal(o, dev_out.cpu())
+    o, lse, q2k = msa.forward(host["q"], host["k"], host["v"], host["q_idx"], host["k_idx"],
+                              q_pos0=w.q_pos0, top_k=w.top_k, return_lse=True, return_q2k=True)
+    assert torch.equal(o, dev_out.cpu()) and torch.equal(lse, dev_lse.cpu())
+    assert torch.equal(q2k, dev_q2k.cpu())
