@@ -103,6 +103,13 @@ bool index_decode_supported(const Problem& P);
 cudaError_t launch_index_decode(const Problem& P, const void* q_idx, const void* k_idx,
                                 float* bmax, int32_t* status, cudaStream_t s);
 cudaError_t launch_topk(const Problem& P, const float* bmax, int32_t* q2k, cudaStream_t s);
+// One query row per sequence whose rows all keep top_k blocks (q_pos0 >=
+// (top_k-1)*Bk): the top-k kernel also writes the block -> query lists (entries,
+// positions, tile records), in the layout launch_lists_direct gives them.
+bool topk_writes_lists(const Problem& P);
+struct Lists;
+cudaError_t launch_topk_lists(const Problem& P, const float* bmax, int32_t* q2k, const Lists& L,
+                              cudaStream_t s);
 
 // --- block -> query lists ---------------------------------------------------
 cudaError_t launch_invert(const Problem& P, const int32_t* q2k, const Lists& L,

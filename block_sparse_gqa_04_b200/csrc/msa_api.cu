@@ -153,8 +153,18 @@ msa_status_t check_ws(const Problem& P, int op, const void* ws, size_t ws_bytes)
   return MSA_OK;
 }
 
+msa::Lists lists_of(void* ws, const Layout& L) {
+  return msa::Lists{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.cursor),
+                    at<int32_t>(ws, L.list_off), at<int32_t>(ws, L.tile_off),
+                    at<int32_t>(ws, L.entries), at<int32_t>(ws, L.pos),
+                    at<int32_t>(ws, L.tiles), at<int32_t>(ws, L.seg_sums)};
+}
+
+// run_select's top-k also writes the block -> query lists (lists != nullptr):
+// msa_forward on one query row per sequence whose rows all keep top_k blocks.
 msa_status_t run_select(const Problem& P, const void* q_idx, const void* k_idx, int32_t* q2k,
-                        float* bscores, void* ws, cudaStream_t s) {
+                        float* bscores, void* ws, cudaStream_t s,
+                        const msa::Lists* lists = nullptr) {
   const Layout L = layout(P, MSA_OP_SELECT);
   float* bmax = bscores ? bscores : at<float>(ws, L.bmax);
   cudaError_t e = msa::launch_check_table(P, at<int32_t>(ws, L.status), s);
@@ -181,23 +191,21 @@ msa_status_t run_select(const Problem& P, const void* q_idx, const void* k_idx, 
     stage_mark(s);
   }
   if (e == cudaSuccess) {
-    e = msa::launch_topk(P, bmax, q2k, s);
+    e = lists ? msa::launch_topk_lists(P, bmax, q2k, *lists, s) : msa::launch_topk(P, bmax, q2k, s);
     stage_mark(s);
   }
   return cuda_status(e);
 }
 
+// lists_ready: the top-k kernel of the same call has written the lists already.
 msa_status_t run_attend(const Problem& P, const void* q, const void* k, const void* v,
                         const int32_t* q2k, void* out, float* lse, void* ws, const Layout& L,
-                        cudaStream_t s) {
-  msa::Lists lists{at<int32_t>(ws, L.counts), at<int32_t>(ws, L.cursor),
-                   at<int32_t>(ws, L.list_off), at<int32_t>(ws, L.tile_off),
-                   at<int32_t>(ws, L.entries), at<int32_t>(ws, L.pos),
-                   at<int32_t>(ws, L.tiles), at<int32_t>(ws, L.seg_sums)};
+                        cudaStream_t s, bool lists_ready = false) {
+  const msa::Lists lists = lists_of(ws, L);
   msa::Partials part{at<void>(ws, L.part_o), at<float>(ws, L.part_lse)};
   const bool tc = msa::attn_tc_supported(P);
   cudaError_t e = msa::launch_check_table(P, at<int32_t>(ws, L.status), s);
-  if (e != cudaSuccess) {
+  if (e != cudaSuccess || lists_ready) {
   } else if (msa::lists_direct(P)) {
     e = msa::launch_lists_direct(P, q2k, lists, at<int32_t>(ws, L.status), s);
   } else {
@@ -292,9 +300,11 @@ msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, c
   int32_t* q2k = q2k_opt ? q2k_opt : at<int32_t>(ws, L.q2k);
   // the select stage only needs the status word and bmax, which sit at the same
   // offsets in the forward layout
-  st = run_select(P, q_idx, k_idx, q2k, nullptr, ws, s);
+  const bool topk_lists = msa::topk_writes_lists(P) && !msa::index_select_fused_supported(P);
+  const msa::Lists lists = lists_of(ws, L);
+  st = run_select(P, q_idx, k_idx, q2k, nullptr, ws, s, topk_lists ? &lists : nullptr);
   if (st != MSA_OK) return st;
-  return run_attend(P, q, k, v, q2k, out, lse_opt, ws, L, s);
+  return run_attend(P, q, k, v, q2k, out, lse_opt, ws, L, s, topk_lists);
 }
 
 msa_status_t msa_index_kl(const msa_problem_t* p, const void* q, const void* k,
@@ -361,7 +371,9 @@ int32_t msa_launch_count(const msa_problem_t* p, int32_t op) {
   switch (op) {
     case MSA_OP_SELECT: return sel;
     case MSA_OP_ATTEND: return att;
-    case MSA_OP_FORWARD: return sel + att;
+    case MSA_OP_FORWARD:
+      // the decode top-k writes the lists itself (one launch fewer)
+      return sel + att - (msa::topk_writes_lists(P) && !msa::index_select_fused_supported(P));
     case MSA_OP_INDEX_KL: return chk + msa::kLaunchesInvert + 3;  // lists, rows, dk, sum
   }
   return 0;

@@ -43,8 +43,14 @@ __device__ __forceinline__ int warp_rank_u64(uint64_t v, int n) {
   return r;
 }
 
+// LISTS: one query row per sequence and every row keeps top_k blocks, so each
+// block -> query list holds at most one entry and the lists are the identity
+// layout (entry = (group, row, slot)); the kernel then also writes the entries,
+// their positions and the one-query tile records the attention kernel reads,
+// in place of the separate list kernel.
+template <bool LISTS>
 __global__ void __launch_bounds__(256) topk_kernel(Problem P, const float* __restrict__ bmax,
-                                                   int32_t* __restrict__ q2k) {
+                                                   int32_t* __restrict__ q2k, Lists L) {
   __shared__ uint64_t cand_all[kTopkWarps][kCandCap];
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
@@ -121,13 +127,45 @@ __global__ void __launch_bounds__(256) topk_kernel(Problem P, const float* __res
   if (lane == need) mine = c_t;
   const int sorted = warp_sort_asc(mine);
   if (lane < P.K) q2k[((long long)g * P.T + r) * P.K + lane] = lane < ksel ? sorted : -1;
+  if (LISTS && lane < P.K) {
+    const int e = int(((long long)g * P.T + r) * P.K + lane);  // ksel == K on every row
+    L.entries[e] = (r << 5) | lane;
+    L.pos[e] = e;
+    TileRec rec;
+    rec.c = sorted;
+    rec.g = g;
+    rec.b = r / P.Sq;
+    rec.e0 = e;
+    rec.n = 1;
+    rec.tend = e + 1;
+    rec.lid = e;
+    rec.pad = 0;
+    rec.rows[0] = r;
+#pragma unroll
+    for (int x = 1; x < 8; ++x) rec.rows[x] = 0;
+    reinterpret_cast<TileRec*>(L.tiles)[e] = rec;
+    if (wid == 0 && lane == 0) L.tile_off[P.nlists] = P.Hkv * P.T * P.K;
+  }
 }
 
 cudaError_t launch_topk(const Problem& P, const float* bmax, int32_t* q2k, cudaStream_t s) {
   long long warps = (long long)P.Hkv * P.T;
   if (warps == 0) return cudaSuccess;
   long long blocks = (warps + kTopkWarps - 1) / kTopkWarps;
-  topk_kernel<<<unsigned(blocks), 32 * kTopkWarps, 0, s>>>(P, bmax, q2k);
+  topk_kernel<false><<<unsigned(blocks), 32 * kTopkWarps, 0, s>>>(P, bmax, q2k, Lists{});
+  return cudaGetLastError();
+}
+
+bool topk_writes_lists(const Problem& P) {
+  return lists_direct(P) && P.q_pos0 >= (long long)(P.K - 1) * P.Bk;
+}
+
+cudaError_t launch_topk_lists(const Problem& P, const float* bmax, int32_t* q2k, const Lists& L,
+                              cudaStream_t s) {
+  long long warps = (long long)P.Hkv * P.T;
+  if (warps == 0) return cudaSuccess;
+  long long blocks = (warps + kTopkWarps - 1) / kTopkWarps;
+  topk_kernel<true><<<unsigned(blocks), 32 * kTopkWarps, 0, s>>>(P, bmax, q2k, L);
   return cudaGetLastError();
 }
 

@@ -31,6 +31,10 @@ SMALL = {
     "decode_rows4": Workload("decode_rows4", 3, 4, 3000, 2942, 32, 4, 128, 128, 128, 8, "bf16", 2),
     "decode_rows8": Workload("decode_rows8", 2, 8, 5000, 4990, 64, 4, 128, 128, 128, 16, "bf16", 2),
     "decode_g2": Workload("decode_g2", 4, 1, 1500, 1499, 16, 2, 128, 128, 128, 4, "bf16", 1),
+    # decode rows that see fewer than top_k blocks (the top-k kernel does not
+    # write the lists then: the separate list kernel compacts the valid slots)
+    "decode_short": Workload("decode_short", 4, 1, 1000, 999, 64, 4, 128, 128, 128, 16, "bf16",
+                             1),
     # fp8 (e4m3) index tensors: tensor-core prefill index, decode index at both
     # query widths, and the SIMT index kernel (index_dim 64)
     "fp8_prefill": Workload("fp8_prefill", 1, 2125, 2125, 0, 64, 4, 128, 128, 128, 16, "bf16", 2,
