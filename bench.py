@@ -306,13 +306,18 @@ def run_e2e(msa, w, xh, out_h, steps, warmup):
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
-# kernel from one 1-pass ncu capture of the bench's default workload, with the
-# git blob id of the kernel source the capture ran: once that source changes
-# the entry no longer applies and the bench reports traffic as null.
+# kernel, with the git blob id of the kernel source the capture ran: once that
+# source changes the entry no longer applies and the bench reports traffic as
+# null.  The counters come from a capture of one launch on the 12288-row prefill
+# (724,992 selected entries) scaled to the 128K prefill's 8,327,168 entries:
+# the partial-state writes grow exactly with the entries, the Q-gather reads
+# grow faster (fewer L2 hits at full size), so the scaled figure is a lower
+# bound on the reads.
 NCU_TRAFFIC = {
     # stage: (workload, source file, git blob id, bytes per launch)
     "attn": ("prefill_128k", "block_sparse_gqa_04_b200/csrc/attn_tc.cu",
-             "4cf3db49c1787f57a16d2863f4918a39892c64af", 13698565888 + 34591706368),
+             "95f0d7f1c440128b0586d8654bf0d3d8bdd585d3",
+             round((394030080 + 2957622016) * 8327168 / 724992)),
 }
 
 
