@@ -28,7 +28,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from block_sparse_gqa_04_b200.workload import WORKLOADS, Workload, make_inputs, sample_rows  # noqa: E402
+from block_sparse_gqa_04_b200.workload import (VARLEN_MIX, WORKLOADS, Workload,  # noqa: E402
+                                                make_inputs, make_varlen_inputs, sample_rows)
 
 METRIC = "128K prefill query-tokens/s & decode tok/s on 1 B200; % tensor/HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
@@ -410,6 +411,48 @@ def path_roofline(cnt, kv_sel_bytes, ms, peaks):
                     "bytes) / HBM peak)"}
 
 
+def measure_varlen(msa, dev, steps, warmup, peaks, lens=VARLEN_MIX):
+    """The packed variable-length batch ``lens`` (msa_forward_varlen) on inputs
+    resident in HBM: ``steps`` timed calls after ``warmup``, CUDA events on the
+    launching stream.  Algorithmic work and the path roofline are the sums over
+    the sequences, each counted as its own one-sequence workload."""
+    lens_q, lens_k = lens
+    Hq, Hkv, D, di, k = 64, 4, 128, 128, 16
+    x = make_varlen_inputs(lens_q, lens_k, Hq, Hkv, D, di, "bf16", seed=0, device=dev)
+    p, cq, ck = msa.varlen_problem(x["cu_q"], x["cu_k"], Hq, Hkv, D, di, top_k=k)
+    ws = torch.empty(msa.varlen_workspace_size(p, cq, ck) + 256, dtype=torch.uint8, device=dev)
+    out = torch.empty(x["q"].shape, dtype=x["v"].dtype, device=dev)
+    args = (x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], x["cu_q"], x["cu_k"])
+    _, q2k = msa.forward_varlen(*args, top_k=k, workspace=ws, out=out, return_q2k=True)
+    cnt = None
+    kv_sel = 0.0
+    for b, (nq, nk) in enumerate(zip(lens_q, lens_k)):
+        if nq == 0:
+            continue
+        wb = Workload(f"varlen_seq{b}", 1, nq, nk, nk - nq, Hq, Hkv, D, di, 128, k, "bf16", 0)
+        c = counts(wb)
+        cnt = c if cnt is None else {n: (cnt[n] + c[n] if isinstance(c[n], float) else c[n])
+                                     for n in c}
+        q0 = x["cu_q"][b]
+        kv_sel += selected_kv_bytes(wb, q2k[:, q0:q0 + nq])
+    del q2k
+    for _ in range(warmup):
+        msa.forward_varlen(*args, top_k=k, workspace=ws, out=out)
+    start, end = _events(2)
+    idx = dev.index if dev.index is not None else 0
+    with ClockSampler(idx) as clk:
+        torch.cuda.synchronize()
+        start.record()
+        for _ in range(steps):
+            msa.forward_varlen(*args, top_k=k, workspace=ws, out=out)
+        end.record()
+        torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    return {"rows": sum(lens_q), "ms": ms, "cnt": cnt, "kv_sel": kv_sel,
+            "launches": msa.varlen_launch_count(p, cq, ck) * steps, "clocks": clk.summary(),
+            "sequences": len(lens_q)}
+
+
 def page_inputs(x, w, dev, seed=0):
     """Moves k, v and k_idx into a shuffled pool of 128-token pages (64 spare
     pages, zero tails) and returns the forward's paging kwargs.  Untimed."""
@@ -727,6 +770,17 @@ def main():
             "path_roofline": path_roofline(eres["cnt"], eres["kv_sel"], ems, peaks),
             "gpu_launches": eres["launches"], "clocks": eres["clocks"]}
         eres.pop("x")
+    if extra_names and not (a.index_dtype or a.qk_dtype or a.paged):
+        # a packed batch of sequences of different lengths (msa_forward_varlen)
+        torch.cuda.empty_cache()
+        vres = measure_varlen(msa, dev, a.steps, a.warmup, peaks)
+        vval, vms = weak_value(vres["rows"], vres["ms"], world)
+        line["varlen_mix"] = {
+            "workload": "varlen_mix", "sequences": vres["sequences"],
+            "query_rows": vres["rows"], "value": vval, "unit": "query-tokens/s",
+            "ms_per_step": vms, "path_roofline": path_roofline(vres["cnt"], vres["kv_sel"], vms,
+                                                               peaks),
+            "gpu_launches": vres["launches"], "clocks": vres["clocks"]}
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         # the oracle runs on host copies of the bench's own inputs
         xm = make_inputs(w, seed=0, device=dev)

@@ -543,8 +543,13 @@ bool index_tc_supported(const Problem& P) {
          P.kv_rows < (1LL << 31);
 }
 
+// The streamed selection pays off in bf16, where the epilogue's extra work hides
+// under the MMAs (index + merge 8.46 ms against 8.3-8.7 ms for the GEMM and the
+// top-k kernel at 128K, and 2.4 GB less DRAM traffic).  With fp8 index tensors the
+// MMAs take half as long and the epilogue bounds the kernel (7.23 against 6.38 ms),
+// so fp8 keeps the block maxima and the top-k kernel.
 bool index_select_fused_supported(const Problem& P) {
-  return index_tc_supported(P) && P.K - 1 <= kMaxKeep && (P.Hkv == 2 || P.Hkv == 4);
+  return index_tc_supported(P) && !P.idx8 && P.K - 1 <= kMaxKeep && (P.Hkv == 2 || P.Hkv == 4);
 }
 
 namespace {

@@ -225,6 +225,94 @@ msa_status_t run_attend(const Problem& P, const void* q, const void* k, const vo
   return cuda_status(e);
 }
 
+// Index branch, selection and main branch of one resolved problem whose
+// workspace is checked and whose status word is already cleared; q2k is the
+// caller's buffer or, when NULL, the workspace's own.
+msa_status_t forward_one(const Problem& P, const void* q, const void* k, const void* v,
+                         const void* q_idx, const void* k_idx, void* out, float* lse,
+                         int32_t* q2k_opt, void* ws, cudaStream_t s) {
+  const Layout L = layout(P, MSA_OP_FORWARD);
+  int32_t* q2k = q2k_opt ? q2k_opt : at<int32_t>(ws, L.q2k);
+  // the select stage only needs the status word and bmax, which sit at the same
+  // offsets in the forward layout
+  const bool topk_lists = msa::topk_writes_lists(P) && !msa::index_select_fused_supported(P);
+  const msa::Lists lists = lists_of(ws, L);
+  msa_status_t st = run_select(P, q_idx, k_idx, q2k, nullptr, ws, s, topk_lists ? &lists : nullptr);
+  if (st != MSA_OK) return st;
+  return run_attend(P, q, k, v, q2k, out, lse, ws, L, s, topk_lists);
+}
+
+// A packed variable-length batch as runs of consecutive sequences with the
+// same (query rows, keys): each run is one fixed-length batched problem, since
+// equal-length sequences packed back to back are exactly the [batch, len, ...]
+// layout.  Sequences without query rows are left out (they end a run).
+struct Run {
+  int b0, nseq, nq, nk;
+};
+
+constexpr int kMaxVarlenSeqs = 1 << 20;
+
+msa_status_t varlen_runs(const msa_problem_t* p, const int32_t* cu_q, const int32_t* cu_k,
+                         Run* runs, int* nruns, long long* total_q) {
+  if (!p || !cu_q || !cu_k || p->batch < 1 || p->batch > kMaxVarlenSeqs)
+    return MSA_ERR_INVALID_ARG;
+  if (p->num_pages != 0) return MSA_ERR_UNSUPPORTED;
+  if (cu_q[0] != 0 || cu_k[0] != 0) return MSA_ERR_INVALID_ARG;
+  int n = 0;
+  for (int b = 0; b < p->batch; ++b) {
+    const long long nq = (long long)cu_q[b + 1] - cu_q[b];
+    const long long nk = (long long)cu_k[b + 1] - cu_k[b];
+    if (nq < 0 || nk < 0 || nq > nk) return MSA_ERR_INVALID_ARG;
+    if (nq == 0) continue;
+    if (n > 0 && runs[n - 1].b0 + runs[n - 1].nseq == b && runs[n - 1].nq == nq &&
+        runs[n - 1].nk == nk) {
+      ++runs[n - 1].nseq;
+    } else {
+      runs[n++] = Run{b, 1, int(nq), int(nk)};
+    }
+  }
+  *nruns = n;
+  *total_q = cu_q[p->batch];
+  return MSA_OK;
+}
+
+// The fixed-length problem of one run.
+msa_problem_t run_problem(const msa_problem_t* p, const Run& r) {
+  msa_problem_t q = *p;
+  q.batch = r.nseq;
+  q.q_len = r.nq;
+  q.kv_len = r.nk;
+  q.q_pos0 = r.nk - r.nq;  // a sequence's query rows are its last tokens
+  return q;
+}
+
+// Runs of a packed batch, resolved; the run list lives on the heap (one entry
+// per sequence at most).
+struct VarlenPlan {
+  Run* runs = nullptr;
+  int n = 0;
+  long long total_q = 0;
+  size_t ws = 0;  // workspace of the largest run (runs reuse it one after another)
+  ~VarlenPlan() { delete[] runs; }
+};
+
+msa_status_t plan_varlen(const msa_problem_t* p, const int32_t* cu_q, const int32_t* cu_k,
+                         VarlenPlan* plan) {
+  if (!p || p->batch < 1 || p->batch > kMaxVarlenSeqs) return MSA_ERR_INVALID_ARG;
+  plan->runs = new Run[p->batch];
+  msa_status_t st = varlen_runs(p, cu_q, cu_k, plan->runs, &plan->n, &plan->total_q);
+  if (st != MSA_OK) return st;
+  plan->ws = align_up(sizeof(int32_t));
+  for (int i = 0; i < plan->n; ++i) {
+    const msa_problem_t rp = run_problem(p, plan->runs[i]);
+    Problem P;
+    if ((st = resolve(&rp, &P)) != MSA_OK) return st;
+    const size_t w = layout(P, MSA_OP_FORWARD).total;
+    if (w > plan->ws) plan->ws = w;
+  }
+  return MSA_OK;
+}
+
 }  // namespace
 
 namespace msa {
@@ -293,18 +381,83 @@ msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, c
     return MSA_ERR_INVALID_ARG;
   if ((st = check_ws(P, MSA_OP_FORWARD, ws, ws_bytes)) != MSA_OK) return st;
   if (P.T == 0) return MSA_OK;
-  const Layout L = layout(P, MSA_OP_FORWARD);
   cudaStream_t s = (cudaStream_t)stream;
   if (msa_status_t cst = cuda_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), s))) return cst;
   stage_begin();
-  int32_t* q2k = q2k_opt ? q2k_opt : at<int32_t>(ws, L.q2k);
-  // the select stage only needs the status word and bmax, which sit at the same
-  // offsets in the forward layout
-  const bool topk_lists = msa::topk_writes_lists(P) && !msa::index_select_fused_supported(P);
-  const msa::Lists lists = lists_of(ws, L);
-  st = run_select(P, q_idx, k_idx, q2k, nullptr, ws, s, topk_lists ? &lists : nullptr);
+  return forward_one(P, q, k, v, q_idx, k_idx, out, lse_opt, q2k_opt, ws, s);
+}
+
+size_t msa_varlen_workspace_size(const msa_problem_t* p, const int32_t* cu_seqlens_q,
+                                 const int32_t* cu_seqlens_k) {
+  VarlenPlan plan;
+  if (plan_varlen(p, cu_seqlens_q, cu_seqlens_k, &plan) != MSA_OK) return 0;
+  return plan.ws;
+}
+
+int32_t msa_varlen_launch_count(const msa_problem_t* p, const int32_t* cu_seqlens_q,
+                                const int32_t* cu_seqlens_k) {
+  VarlenPlan plan;
+  if (plan_varlen(p, cu_seqlens_q, cu_seqlens_k, &plan) != MSA_OK) return 0;
+  int32_t n = 0;
+  for (int i = 0; i < plan.n; ++i) {
+    const msa_problem_t rp = run_problem(p, plan.runs[i]);
+    n += msa_launch_count(&rp, MSA_OP_FORWARD);
+  }
+  return n;  // the q2k copies (q2k_opt) are memory copies, not kernel launches
+}
+
+msa_status_t msa_forward_varlen(const msa_problem_t* p, const int32_t* cu_seqlens_q,
+                                const int32_t* cu_seqlens_k, const void* q, const void* k,
+                                const void* v, const void* q_idx, const void* k_idx, void* out,
+                                float* lse_opt, int32_t* q2k_opt, void* ws, size_t ws_bytes,
+                                void* stream) {
+  VarlenPlan plan;
+  msa_status_t st = plan_varlen(p, cu_seqlens_q, cu_seqlens_k, &plan);
   if (st != MSA_OK) return st;
-  return run_attend(P, q, k, v, q2k, out, lse_opt, ws, L, s, topk_lists);
+  if (plan.total_q == 0) return MSA_OK;  // no query row: nothing to do
+  if (!q || !k || !v || !q_idx || !k_idx || !out) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_idx) ||
+      !aligned16(k_idx) || !aligned16(out) || (lse_opt && !aligned16(lse_opt)) ||
+      (q2k_opt && !aligned16(q2k_opt)))
+    return MSA_ERR_INVALID_ARG;
+  // the runs' log-normalisers start at row offsets of num_q_heads floats
+  if (lse_opt && p->num_q_heads % 4 != 0) return MSA_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return MSA_ERR_INVALID_ARG;
+  if (ws_bytes < plan.ws) return MSA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  // one status word for the whole call: the runs OR their flags into it
+  if (msa_status_t cst = cuda_status(cudaMemsetAsync(ws, 0, sizeof(int32_t), s))) return cst;
+  stage_begin();
+  const size_t esz = p->dtype == MSA_F32 ? 4 : 2;
+  const size_t esz_qk = p->qk_dtype == MSA_FP8_E4M3 ? 1 : esz;
+  const size_t esz_idx = p->index_dtype == MSA_FP8_E4M3 ? 1 : esz;
+  const size_t qrow = size_t(p->num_q_heads) * p->head_dim;   // elements per query row
+  const size_t krow = size_t(p->num_kv_heads) * p->head_dim;  // per key row
+  for (int i = 0; i < plan.n; ++i) {
+    const Run& r = plan.runs[i];
+    const msa_problem_t rp = run_problem(p, r);
+    Problem P;
+    if ((st = resolve(&rp, &P)) != MSA_OK) return st;
+    const size_t q0 = size_t(cu_seqlens_q[r.b0]), k0 = size_t(cu_seqlens_k[r.b0]);
+    const char* qb = static_cast<const char*>(q) + q0 * qrow * esz_qk;
+    const char* kb = static_cast<const char*>(k) + k0 * krow * esz_qk;
+    const char* vb = static_cast<const char*>(v) + k0 * krow * esz;
+    const char* qib = static_cast<const char*>(q_idx) + q0 * p->num_kv_heads * p->index_dim * esz_idx;
+    const char* kib = static_cast<const char*>(k_idx) + k0 * p->index_dim * esz_idx;
+    char* ob = static_cast<char*>(out) + q0 * qrow * esz;
+    float* lb = lse_opt ? lse_opt + q0 * p->num_q_heads : nullptr;
+    if ((st = forward_one(P, qb, kb, vb, qib, kib, ob, lb, nullptr, ws, s)) != MSA_OK) return st;
+    if (q2k_opt) {
+      // the run's [Hkv, rows, top_k] selection into the packed [Hkv, total_q, top_k]
+      const Layout L = layout(P, MSA_OP_FORWARD);
+      const size_t w = size_t(P.T) * P.K * sizeof(int32_t);
+      if (msa_status_t cst = cuda_status(cudaMemcpy2DAsync(
+              q2k_opt + q0 * P.K, size_t(plan.total_q) * P.K * sizeof(int32_t),
+              at<int32_t>(ws, L.q2k), w, w, size_t(P.Hkv), cudaMemcpyDeviceToDevice, s)))
+        return cst;
+    }
+  }
+  return MSA_OK;
 }
 
 msa_status_t msa_index_kl(const msa_problem_t* p, const void* q, const void* k,

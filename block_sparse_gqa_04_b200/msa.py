@@ -28,7 +28,8 @@ STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 EXPORTED = ("msa_workspace_size", "msa_select", "msa_attend", "msa_forward",
             "msa_device_status", "msa_set_stage_events", "msa_launch_count", "msa_kernel_path",
             "msa_status_string", "msa_select_static", "msa_index_kl",
-            "msa_selftest_wait_timeout", "msa_last_cuda_error")
+            "msa_selftest_wait_timeout", "msa_last_cuda_error", "msa_forward_varlen",
+            "msa_varlen_workspace_size", "msa_varlen_launch_count")
 STAGES = ("index", "topk", "lists", "attn", "combine")
 
 
@@ -93,6 +94,13 @@ def load() -> ctypes.CDLL:
         lib.msa_selftest_wait_timeout.restype = i32
         lib.msa_last_cuda_error.argtypes = [ctypes.POINTER(i32)]
         lib.msa_last_cuda_error.restype = ctypes.c_char_p
+        cu = ctypes.POINTER(i32)
+        lib.msa_forward_varlen.argtypes = [pp, cu, cu, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.msa_forward_varlen.restype = i32
+        lib.msa_varlen_workspace_size.argtypes = [pp, cu, cu]
+        lib.msa_varlen_workspace_size.restype = sz
+        lib.msa_varlen_launch_count.argtypes = [pp, cu, cu]
+        lib.msa_varlen_launch_count.restype = i32
         _lib = lib
     return _lib
 
@@ -506,6 +514,101 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
         code = ctypes.c_int32(0)
         _check(load().msa_device_status(ctypes.c_void_p(wp), ctypes.byref(code), _stream(dev)),
                "msa_forward (device status)")
+    res = (o,)
+    if return_lse:
+        res += (lse,)
+    if return_q2k:
+        res += (q2k,)
+    return res[0] if len(res) == 1 else res
+
+
+def _cu_seqlens(cu, name: str):
+    """A host prefix-sum array of sequence lengths as a ctypes int32 array."""
+    if isinstance(cu, torch.Tensor):
+        if cu.is_cuda:
+            raise ValueError(f"{name} is read on the host: pass a CPU tensor or a list")
+        cu = cu.tolist()
+    vals = [int(x) for x in cu]
+    if len(vals) < 2:
+        raise ValueError(f"{name} needs batch + 1 >= 2 entries")
+    return (ctypes.c_int32 * len(vals))(*vals), vals
+
+
+def varlen_problem(cu_seqlens_q, cu_seqlens_k, num_q_heads, num_kv_heads, head_dim, index_dim,
+                   block_size=128, top_k=16, dtype=torch.bfloat16, softmax_scale=0.0,
+                   index_dtype=None, qk_dtype=None):
+    """(Problem, cu_q, cu_k) of a packed batch for the varlen entry points."""
+    cq, vq = _cu_seqlens(cu_seqlens_q, "cu_seqlens_q")
+    ck, vk = _cu_seqlens(cu_seqlens_k, "cu_seqlens_k")
+    if len(vq) != len(vk):
+        raise ValueError("cu_seqlens_q and cu_seqlens_k differ in length")
+    p = make_problem(len(vq) - 1, 0, 1, num_q_heads, num_kv_heads, head_dim, index_dim,
+                     block_size, top_k, dtype, 0, softmax_scale, index_dtype=index_dtype,
+                     qk_dtype=qk_dtype)
+    return p, cq, ck
+
+
+def varlen_workspace_size(p: Problem, cu_q, cu_k) -> int:
+    return int(load().msa_varlen_workspace_size(ctypes.byref(p), cu_q, cu_k))
+
+
+def varlen_launch_count(p: Problem, cu_q, cu_k) -> int:
+    return int(load().msa_varlen_launch_count(ctypes.byref(p), cu_q, cu_k))
+
+
+def forward_varlen(q, k, v, q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, *, block_size: int = 128,
+                   top_k: int = 16, softmax_scale: float = 0.0, return_lse: bool = False,
+                   return_q2k: bool = False, workspace: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, check_device_status: bool = False):
+    """Forward pass over a packed batch of sequences of different lengths
+    (msa_forward_varlen).  CUDA tensors q [total_q, Hq, D], k, v [total_k, Hkv, D],
+    q_idx [total_q, Hkv, di], k_idx [total_k, di]; cu_seqlens_q / cu_seqlens_k:
+    host prefix sums (lists or CPU tensors) of batch + 1 entries.  Sequence b's
+    query rows are its last cu_seqlens_q[b+1] - cu_seqlens_q[b] tokens.  Returns
+    out [total_q, Hq, D] (and lse [total_q, Hq], q2k [Hkv, total_q, top_k])."""
+    _require_cuda(q, k, v, q_idx, k_idx)
+    if q.dim() != 3 or k.dim() != 3 or q_idx.dim() != 3 or k_idx.dim() != 2:
+        raise ValueError("varlen tensors are packed: q [total_q, Hq, D], k, v [total_k, Hkv, D], "
+                         "q_idx [total_q, Hkv, di], k_idx [total_k, di]")
+    total_q, Hq, D = q.shape
+    total_k, Hkv, _ = k.shape
+    di = q_idx.shape[2]
+    want = {"k": (k, (total_k, Hkv, D)), "v": (v, (total_k, Hkv, D)),
+            "q_idx": (q_idx, (total_q, Hkv, di)), "k_idx": (k_idx, (total_k, di))}
+    for name, (t, shape) in want.items():
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
+    if k_idx.dtype != q_idx.dtype:
+        raise ValueError(f"q_idx and k_idx dtypes differ: {q_idx.dtype} vs {k_idx.dtype}")
+    _check_qkv_dtypes(q, k, v)
+    p, cq, ck = varlen_problem(cu_seqlens_q, cu_seqlens_k, Hq, Hkv, D, di, block_size, top_k,
+                               v.dtype, softmax_scale, index_dtype=q_idx.dtype,
+                               qk_dtype=q.dtype)
+    if cq[len(cq) - 1] != total_q or ck[len(ck) - 1] != total_k:
+        raise ValueError(f"the prefix sums end at {cq[len(cq) - 1]} / {ck[len(ck) - 1]}, "
+                         f"the tensors hold {total_q} / {total_k} rows")
+    if out is not None and (out.dtype != v.dtype or tuple(out.shape) != tuple(q.shape)
+                            or not out.is_contiguous() or not out.is_cuda):
+        raise ValueError(f"out must be a contiguous CUDA {tuple(q.shape)} tensor of v's dtype")
+    dev = q.device
+    o = out if out is not None else torch.empty(q.shape, dtype=v.dtype, device=dev)
+    lse = torch.empty((total_q, Hq), dtype=torch.float32, device=dev) if return_lse else None
+    q2k = (torch.full((Hkv, total_q, top_k), -1, dtype=torch.int32, device=dev)
+           if return_q2k else None)
+    if workspace is None:
+        n = varlen_workspace_size(p, cq, ck)
+        if n == 0:
+            raise MsaError(1, "msa_varlen_workspace_size")
+        workspace = torch.empty(n + 256, dtype=torch.uint8, device=dev)
+    wp, wn = _ws_view(workspace)
+    _check(load().msa_forward_varlen(ctypes.byref(p), cq, ck, _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(q_idx), _ptr(k_idx), _ptr(o), _ptr(lse), _ptr(q2k),
+                                     ctypes.c_void_p(wp), wn, _stream(dev)),
+           "msa_forward_varlen")
+    if check_device_status:
+        code = ctypes.c_int32(0)
+        _check(load().msa_device_status(ctypes.c_void_p(wp), ctypes.byref(code), _stream(dev)),
+               "msa_forward_varlen (device status)")
     res = (o,)
     if return_lse:
         res += (lse,)

@@ -86,6 +86,13 @@ WORKLOADS: Dict[str, Workload] = {
                          "bf16", 64),
 }
 
+# A packed serving-style batch for the variable-length entry point (prefill_128k
+# shapes: 64 query heads, 4 groups, head_dim and index_dim 128, top 16, bf16):
+# (query rows, keys) per sequence: two fresh prefills, two prefill chunks at
+# 32K and 64K context and sixteen decode rows at 128K (one run of equal lengths).
+VARLEN_MIX = ([8192, 16384, 2048] + [1] * 16 + [4096],
+              [8192, 16384, 32768] + [131072] * 16 + [65536])
+
 _CHUNK_ELEMS = 1 << 24
 
 
@@ -171,3 +178,34 @@ def sample_rows(w: Workload, n: int, seed: int = 0) -> list:
 def scaled(w: Workload, name: Optional[str] = None, **kw) -> Workload:
     """A smaller test case with the same structure as ``w``."""
     return w.with_(name=name or (w.name + "_scaled"), **kw)
+
+
+def make_varlen_inputs(lens_q, lens_k, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                       index_dim: int, dtype: str = "bf16", seed: int = 0,
+                       device="cpu") -> Dict[str, object]:
+    """Packed inputs of a batch of sequences of different lengths: sequence b
+    has lens_q[b] query rows (its last tokens) and lens_k[b] keys.  Same draws
+    as make_inputs (N(0,1) scaled by 1/sqrt(d) for bf16, order q, k, v, q_idx,
+    k_idx, one generator), over the packed rows, without needles; returns q
+    [total_q, Hq, D], k, v [total_k, Hkv, D], q_idx [total_q, Hkv, di], k_idx
+    [total_k, di] and the prefix sums cu_q, cu_k (Python lists)."""
+    if len(lens_q) != len(lens_k) or any(a < 0 or a > b for a, b in zip(lens_q, lens_k)):
+        raise ValueError("need 0 <= lens_q[b] <= lens_k[b] for every sequence")
+    gen = torch.Generator(device=device).manual_seed(seed)
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    s_main = 1.0 if dtype == "f32" else 1.0 / math.sqrt(head_dim)
+    s_idx = 1.0 if dtype == "f32" else 1.0 / math.sqrt(index_dim)
+    tq, tk = sum(lens_q), sum(lens_k)
+    cu_q, cu_k = [0], [0]
+    for a, b in zip(lens_q, lens_k):
+        cu_q.append(cu_q[-1] + a)
+        cu_k.append(cu_k[-1] + b)
+    return {
+        "q": _draw(gen, (tq, num_q_heads, head_dim), s_main, dt),
+        "k": _draw(gen, (tk, num_kv_heads, head_dim), s_main, dt),
+        "v": _draw(gen, (tk, num_kv_heads, head_dim), s_main, dt),
+        "q_idx": _draw(gen, (tq, num_kv_heads, index_dim), s_idx, dt),
+        "k_idx": _draw(gen, (tk, index_dim), s_idx, dt),
+        "cu_q": cu_q,
+        "cu_k": cu_k,
+    }

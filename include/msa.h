@@ -156,6 +156,44 @@ msa_status_t msa_forward(const msa_problem_t* p, const void* q, const void* k, c
                          const void* q_idx, const void* k_idx, void* out, float* lse_opt,
                          int32_t* q2k_opt, void* ws, size_t ws_bytes, void* stream);
 
+/* Packed variable-length batch ("Substantial numerical differences with Minimax
+ * MSA attention vs Minimax's Reference", section 原因分析: the selection has the
+ * packed shape [total_qo_len, heads, topk], the query rows of all sequences
+ * concatenated).  Sequence b owns query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ * and key rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1 of the packed, token-major
+ *   q, out [total_q, num_q_heads, head_dim]   q_idx [total_q, num_kv_heads, index_dim]
+ *   k, v   [total_k, num_kv_heads, head_dim]  k_idx [total_k, index_dim]
+ *   lse_opt [total_q, num_q_heads] fp32       q2k_opt [num_kv_heads, total_q, top_k] int32
+ * Its n_q = cu_seqlens_q[b+1] - cu_seqlens_q[b] query rows are its last n_q tokens
+ * (positions n_k - n_q + i, n_k = cu_seqlens_k[b+1] - cu_seqlens_k[b]), as in
+ * chunked prefill and decode; 0 <= n_q <= n_k; sequences never see one another.
+ * cu_seqlens_q and cu_seqlens_k are HOST arrays of batch + 1 int32 prefix sums
+ * starting at 0 (the call reads them before it returns).  p: batch = number of
+ * sequences; q_len, kv_len and q_pos0 are ignored; num_pages must be 0
+ * (MSA_ERR_UNSUPPORTED otherwise); the other fields and every shape rule as in
+ * msa_forward, applied to each sequence.  lse_opt requires num_q_heads % 4 == 0.
+ * Consecutive sequences with equal (n_q, n_k) form one batched problem and run
+ * as one set of kernel launches; the runs execute one after another on `stream`
+ * in the same workspace (msa_varlen_workspace_size bytes: that of the largest
+ * run); sequences without query rows cost nothing.  Returns before any launch
+ * for bad lengths (a decreasing prefix sum, n_q > n_k), null or misaligned
+ * pointers, or a short workspace.  Stage events (msa_set_stage_events) cover the
+ * first run. */
+msa_status_t msa_forward_varlen(const msa_problem_t* p, const int32_t* cu_seqlens_q,
+                                const int32_t* cu_seqlens_k, const void* q, const void* k,
+                                const void* v, const void* q_idx, const void* k_idx, void* out,
+                                float* lse_opt, int32_t* q2k_opt, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/* Workspace bytes of msa_forward_varlen for these lengths (0 if invalid). */
+size_t msa_varlen_workspace_size(const msa_problem_t* p, const int32_t* cu_seqlens_q,
+                                 const int32_t* cu_seqlens_k);
+
+/* Kernel launches one msa_forward_varlen call makes for these lengths (the sum
+ * over its runs of msa_launch_count(run, MSA_OP_FORWARD)); 0 if invalid. */
+int32_t msa_varlen_launch_count(const msa_problem_t* p, const int32_t* cu_seqlens_q,
+                                const int32_t* cu_seqlens_k);
+
 /* msa_select without a workspace: the same index branch and selection,
  * writing the same q2k, with its scratch in a fixed 256-byte-aligned device
  * buffer inside this library (status word + block maxima), so the call

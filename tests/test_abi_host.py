@@ -279,3 +279,72 @@ def test_index_pair_shape_and_dtype_are_checked_before_the_device():
     with pytest.raises(ValueError, match="k_idx"):
         msa._check_index_pair(qi, torch.zeros((7, 64, di), dtype=bf), paged=True)
     assert msa._check_index_pair(qi, torch.zeros((7, 128, di), dtype=bf), paged=True) == 128
+
+
+def _varlen(cu_q, cu_k, **kw):
+    args = dict(num_q_heads=32, num_kv_heads=2, head_dim=128, index_dim=128, top_k=4)
+    args.update(kw)
+    return msa.varlen_problem(cu_q, cu_k, **args)
+
+
+def test_varlen_runs_sizes_and_launch_counts(lib):
+    # runs of consecutive equal (q rows, keys); empty sequences end a run and cost nothing
+    cu_q, cu_k = [0, 1, 2, 2, 202, 402, 403], [0, 700, 1400, 1450, 2350, 3250, 3950]
+    p, cq, ck = _varlen(cu_q, cu_k)
+    runs = [(2, 1, 700), (2, 200, 900), (1, 1, 700)]
+    mk = lambda n, sq, skv: msa.make_problem(n, sq, skv, 32, 2, 128, 128, top_k=4,  # noqa: E731
+                                             q_pos0=skv - sq)
+    assert msa.varlen_launch_count(p, cq, ck) == sum(msa.launch_count(mk(*r)) for r in runs)
+    assert msa.varlen_workspace_size(p, cq, ck) == max(msa.workspace_size(mk(*r)) for r in runs)
+    # one run when every length is equal: the batched problem
+    p, cq, ck = _varlen([0, 5, 10, 15], [0, 300, 600, 900])
+    assert msa.varlen_workspace_size(p, cq, ck) == msa.workspace_size(mk(3, 5, 300))
+    # only empty sequences: nothing to launch, a status word of workspace
+    p, cq, ck = _varlen([0, 0, 0], [0, 10, 20])
+    assert msa.varlen_launch_count(p, cq, ck) == 0
+    assert msa.varlen_workspace_size(p, cq, ck) == 256
+
+
+@pytest.mark.parametrize("cu_q,cu_k", [
+    ([0, 5], [0, 4]),             # more query rows than keys
+    ([0, 3, 2], [0, 10, 20]),     # decreasing prefix sum
+    ([1, 3], [0, 10]),            # does not start at 0
+    ([0, 3], [0, -1]),
+])
+def test_varlen_bad_lengths_are_rejected(lib, cu_q, cu_k):
+    p, cq, ck = _varlen(cu_q, cu_k)
+    assert msa.varlen_workspace_size(p, cq, ck) == 0
+    assert msa.varlen_launch_count(p, cq, ck) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    code = lib.msa_forward_varlen(ctypes.byref(p), cq, ck, fake, fake, fake, fake, fake, fake,
+                                  None, None, fake, 1 << 30, None)
+    assert code == 1  # MSA_ERR_INVALID_ARG, before any CUDA call
+
+
+def test_varlen_argument_checks_before_any_launch(lib):
+    p, cq, ck = _varlen([0, 100, 101], [0, 100, 700])
+    need = msa.varlen_workspace_size(p, cq, ck)
+    a = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: every check fails first
+    f = lib.msa_forward_varlen
+    args = lambda **o: [o.get(n, a) for n in ("q", "k", "v", "qi", "ki", "out")]  # noqa: E731
+    assert f(ctypes.byref(p), cq, ck, *args(q=None), None, None, a, need, None) == 1
+    assert f(ctypes.byref(p), cq, ck, *args(k=ctypes.c_void_p((1 << 20) + 8)), None, None, a,
+             need, None) == 1
+    assert f(ctypes.byref(p), cq, ck, *args(), None, None, a, need - 1, None) == 3
+    assert f(ctypes.byref(p), cq, ck, *args(), None, None, ctypes.c_void_p((1 << 20) + 16),
+             need, None) == 1  # workspace not on a 256-byte boundary
+    # lse rows start at multiples of num_q_heads floats: 16-byte aligned only for Hq % 4 == 0
+    p2, cq2, ck2 = _varlen([0, 100, 101], [0, 100, 700], num_q_heads=2, num_kv_heads=2)
+    assert f(ctypes.byref(p2), cq2, ck2, *args(), a, None, a, 1 << 30, None) == 1
+    # a paged cache is not a packed batch
+    p.num_pages = 4
+    assert msa.varlen_workspace_size(p, cq, ck) == 0
+    assert f(ctypes.byref(p), cq, ck, *args(), None, None, a, 1 << 30, None) == 2
+
+
+def test_varlen_binding_checks_shapes_before_any_launch():
+    # CPU tensors never reach the library; shape and prefix-sum mismatches are
+    # caught in Python
+    x = workload.make_varlen_inputs([3, 2], [10, 4], 8, 2, 64, 32)
+    with pytest.raises(ValueError):
+        msa.forward_varlen(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], x["cu_q"], x["cu_k"])

@@ -4,11 +4,13 @@ two-kernel path (block maxima to HBM, then the top-k kernel).
 Both paths rank the same fp32 block maxima computed by the same epilogue, so
 their selections must agree bit for bit on every row, decided or not.  msa.select
 with return_block_scores takes the two-kernel path; without it (and in
-msa.forward) the streamed path runs whenever the index kernel is the tcgen05 one,
-top_k <= 16 and there are 2 or 4 groups.  The cases split query tiles across the
-contiguous shares of several CTAs (long sequences and the 1M-token chunk), use
-two groups with a chunk that does not start on a block boundary, fp8 index
-tensors, a batch of sequences and top_k = 1.
+msa.forward) the streamed path runs whenever the index kernel is the tcgen05 one
+with bf16 index tensors, top_k <= 16 and there are 2 or 4 groups (fp8 index
+tensors keep the two-kernel path, which is faster for them).  The cases split
+query tiles across the contiguous shares of several CTAs (long sequences and the
+1M-token chunk), use two groups with a chunk that does not start on a block
+boundary, a batch of sequences and top_k = 1 and 5; the fp8 case checks that
+both calls agree on the path fp8 takes.
 """
 import pytest
 import torch
