@@ -54,6 +54,12 @@ design notes of the repository):
       gradients flow into q_idx and k_idx only.
   R21 in a packed variable-length batch, a sequence's query rows are its last
       tokens (chunked prefill and decode), and sequences are independent.
+  R22 NVFP4 index tensors ([HU] "Elérhetőség" lists NVFP4 among the kernel
+      precisions and says no more): NVIDIA's NVFP4 format, e2m1 elements (two
+      per byte, the even element in the low nibble) with one unsigned e4m3
+      (ue4m3) scale per 16 consecutive elements along index_dim, no second
+      per-tensor scale (a positive factor changes no selection, R1).  The
+      scores are taken over the decoded values.
 
 Additional source for the KL-alignment loss:
   [DK]  section "Træning og stabilisering": Top-k is not differentiable, so an
@@ -97,6 +103,48 @@ def _take(x, idx: np.ndarray) -> np.ndarray:
 
 def _rows(batch: int, q_len: int, rows: Optional[Iterable[int]]) -> list:
     return list(range(batch * q_len)) if rows is None else [int(r) for r in rows]
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 index tensors (reading R22), decoded from the format's definition
+# ---------------------------------------------------------------------------
+
+NVFP4_GROUP = 16  # elements per ue4m3 scale
+
+
+def e2m1_value(code: int) -> float:
+    """One 4-bit e2m1 code: bit 3 sign, bits 2-1 exponent (bias 1), bit 0
+    mantissa; exponent 0 is subnormal (mantissa x 0.5)."""
+    sign = -1.0 if code & 8 else 1.0
+    e, m = (code >> 1) & 3, code & 1
+    mag = 0.5 * m if e == 0 else 2.0 ** (e - 1) * (1.0 + 0.5 * m)
+    return sign * mag
+
+
+def ue4m3_value(code: int) -> float:
+    """One unsigned e4m3 scale byte: bits 6-3 exponent (bias 7), bits 2-0
+    mantissa, exponent 0 subnormal (mantissa/8 x 2^-6); 0x7f is NaN and the
+    top bit must be clear."""
+    if code & 0x80 or code == 0x7F:
+        return math.nan
+    e, m = (code >> 3) & 15, code & 7
+    return (m / 8.0) * 2.0 ** -6 if e == 0 else 2.0 ** (e - 7) * (1.0 + m / 8.0)
+
+
+def nvfp4_decode(codes, scales) -> np.ndarray:
+    """Values of NVFP4 tensors: ``codes`` [..., d/2] bytes (element 2i in the low
+    nibble of byte i, 2i+1 in the high nibble), ``scales`` [..., d/16] ue4m3
+    bytes.  Returns float64 [..., d]: element j = e2m1(code j) x scale[j // 16]."""
+    c = np.asarray(_np(codes)).astype(np.int64)
+    sc = np.asarray(_np(scales)).astype(np.int64)
+    d = c.shape[-1] * 2
+    assert sc.shape[-1] * NVFP4_GROUP == d, "one scale per 16 elements"
+    lut_e = np.array([e2m1_value(i) for i in range(16)])
+    lut_s = np.array([ue4m3_value(i) for i in range(256)])
+    nib = np.empty(c.shape[:-1] + (d,), dtype=np.int64)
+    nib[..., 0::2] = c & 15
+    nib[..., 1::2] = (c >> 4) & 15
+    return lut_e[nib] * np.repeat(lut_s[sc], NVFP4_GROUP, axis=-1)
 
 
 # ---------------------------------------------------------------------------
