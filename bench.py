@@ -57,7 +57,10 @@ def counts(w: Workload) -> dict:
     index_flops = 2.0 * w.index_dim * w.num_kv_heads * vis_keys
     main_flops = 4.0 * w.head_dim * w.num_q_heads * w.block_size * sel_blocks  # S and P V
     esz = 4 if w.dtype == "f32" else 2
-    kidx_bytes = float(B * w.kv_len * w.index_dim * (1 if w.index_dtype == "fp8" else esz))
+    # NVFP4: half a byte per element plus one scale byte per 16 elements
+    kidx_row = {"fp8": w.index_dim, "nvfp4": w.index_dim // 2 + w.index_dim // 16}.get(
+        w.index_dtype, w.index_dim * esz)
+    kidx_bytes = float(B * w.kv_len * kidx_row)
     bmax_read = float(B * w.num_kv_heads * np.sum(c_t) * 4)
     partial_bytes = float(w.num_q_heads * sel_blocks * (w.head_dim * esz + 4))
     out_bytes = float(w.rows * w.num_q_heads * w.head_dim * esz)
@@ -477,10 +480,13 @@ def page_inputs(x, w, dev, seed=0):
 def measure_workload(msa, w, dev, steps, warmup, peaks, with_e2e, paged=False):
     x = make_inputs(w, seed=0, device=dev)
     x.pop("needles")
-    p = msa.problem_of(w)
     extra = {}
+    if "q_idx_scale" in x:  # NVFP4 index tensors: codes + scales
+        extra["index_scales"] = (x["q_idx_scale"], x["k_idx_scale"])
+    p = msa.problem_of(w, index_scales=extra.get("index_scales"))
     if paged:
-        extra, npages = page_inputs(x, w, dev)
+        pextra, npages = page_inputs(x, w, dev)
+        extra.update(pextra)
         p = msa.make_problem(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
                              w.head_dim, w.index_dim, w.block_size, w.top_k, w.torch_dtype,
                              w.q_pos0, index_dtype=w.torch_index_dtype,
@@ -501,7 +507,7 @@ def measure_workload(msa, w, dev, steps, warmup, peaks, with_e2e, paged=False):
         ms, stage = run_steps(msa, w, x, ws, out, steps, warmup, extra=extra)
     res = {"w": w, "ms": ms, "stage": stage, "path": path, "cnt": cnt, "kv_sel": kv_sel,
            "clocks": clk.summary(), "launches": msa.launch_count(p) * steps, "x": x}
-    if with_e2e and not paged:
+    if with_e2e and not paged and w.index_dtype != "nvfp4":
         xh = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "q_idx", "k_idx")}
         del ws
         torch.cuda.empty_cache()
@@ -636,7 +642,7 @@ def main():
     ap.add_argument("--seq", type=int, default=0,
                     help="prefill length override (a smaller case of the same structure, "
                          "e.g. for profiling); needles scale with the length")
-    ap.add_argument("--index-dtype", default="", choices=["", "fp8"],
+    ap.add_argument("--index-dtype", default="", choices=["", "fp8", "nvfp4"],
                     help="fp8: q_idx and k_idx in fp8 e4m3 (bf16 workloads)")
     ap.add_argument("--qk-dtype", default="", choices=["", "fp8"],
                     help="fp8: the main branch's q and k in fp8 e4m3, v bf16 (bf16 workloads)")
@@ -652,6 +658,8 @@ def main():
     a = ap.parse_args()
     if a.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if a.index_dtype == "nvfp4" and (a.paged or a.index_kl or a.impl == "reference"):
+        raise SystemExit("--index-dtype nvfp4 is measured on contiguous forward steps only")
     world, rank, local = dist_setup()
     w = WORKLOADS[a.workload]
     if a.seq:
@@ -710,6 +718,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": ("f32" if w.dtype == "f32" else
+                  "e2m1+bf16" if w.index_dtype == "nvfp4" else
                   "e4m3+bf16" if (w.index_dtype == "fp8" or w.qk_dtype == "fp8") else "bf16"),
         "data": "synthetic (seeded N(0,1/d) inputs with planted needle blocks)",
         "config": dict(workload_config(w, world), kernel_path=main_res["path"],
@@ -781,7 +790,7 @@ def main():
             "ms_per_step": vms, "path_roofline": path_roofline(vres["cnt"], vres["kv_sel"], vms,
                                                                peaks),
             "gpu_launches": vres["launches"], "clocks": vres["clocks"]}
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and w.index_dtype != "nvfp4":
         # the oracle runs on host copies of the bench's own inputs
         xm = make_inputs(w, seed=0, device=dev)
         xm.pop("needles")

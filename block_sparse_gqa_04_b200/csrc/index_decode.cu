@@ -323,7 +323,7 @@ int sm_count() {
 
 bool index_decode_supported(const Problem& P) {
   const int rg = P.Sq * P.Hkv;
-  return !P.f32 && P.DI == 128 && P.Bk == 128 && P.Sq <= 8 && rg >= 1 && rg <= kMaxRG &&
+  return !P.f32 && !P.idx4 && P.DI == 128 && P.Bk == 128 && P.Sq <= 8 && rg >= 1 && rg <= kMaxRG &&
          P.kv_rows < (1LL << 31);
 }
 

@@ -300,7 +300,7 @@ static cudaError_t launch_kl_t(const Problem& P, const void* q, const void* k, c
 }
 
 bool index_kl_supported(const Problem& P) {
-  return kl_rows_smem(P) <= 200 * 1024 && P.D % 8 == 0 && P.DI % kDkChunk == 0 &&
+  return !P.idx4 && kl_rows_smem(P) <= 200 * 1024 && P.D % 8 == 0 && P.DI % kDkChunk == 0 &&
          P.Bk == kKlThreads && P.K <= 32;
 }
 

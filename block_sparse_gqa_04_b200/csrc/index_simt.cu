@@ -163,6 +163,7 @@ static cudaError_t dispatch_di(const Problem& P, const void* qi, const void* ki,
 
 cudaError_t launch_index_simt(const Problem& P, const void* q_idx, const void* k_idx,
                               float* bmax, cudaStream_t s) {
+  if (P.idx4) return cudaErrorInvalidValue;  // NVFP4 codes go through nvfp4.cu
   if (P.idx8) return dispatch_di<__nv_fp8_e4m3>(P, q_idx, k_idx, bmax, s);
   return P.f32 ? dispatch_di<float>(P, q_idx, k_idx, bmax, s)
                : dispatch_di<__nv_bfloat16>(P, q_idx, k_idx, bmax, s);

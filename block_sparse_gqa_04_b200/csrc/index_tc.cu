@@ -539,7 +539,7 @@ int sm_count() {
 }  // namespace
 
 bool index_tc_supported(const Problem& P) {
-  return !P.f32 && P.DI == 128 && P.Bk == 128 && P.Hkv <= kMaxGroups && P.Sq > 8 &&
+  return !P.f32 && !P.idx4 && P.DI == 128 && P.Bk == 128 && P.Hkv <= kMaxGroups && P.Sq > 8 &&
          P.kv_rows < (1LL << 31);
 }
 

@@ -27,6 +27,9 @@ struct Problem {
   float scale;      // main-branch logit scale
   bool f32;         // fp32 tensors (else bf16)
   bool idx8;        // q_idx and k_idx are fp8 e4m3 (bf16 problems)
+  bool idx4;        // q_idx and k_idx are NVFP4 codes with ue4m3 scales qsc, ksc
+  const uint8_t* qsc;  // NVFP4: [T, Hkv, DI/16] scales of q_idx
+  const uint8_t* ksc;  // NVFP4: [kv_rows, DI/16] scales of k_idx
   bool qk8;         // q and k are fp8 e4m3, v bf16 (bf16 problems)
   // KV storage: contiguous per sequence (table == nullptr) or a pool of
   // `pages` pages of Bk tokens named by table[b * nblk + c]
@@ -103,6 +106,13 @@ bool index_decode_supported(const Problem& P);
 cudaError_t launch_index_decode(const Problem& P, const void* q_idx, const void* k_idx,
                                 float* bmax, int32_t* status, cudaStream_t s);
 cudaError_t launch_topk(const Problem& P, const float* bmax, int32_t* q2k, cudaStream_t s);
+// NVFP4 index tensors: block maxima straight from the codes for a few rows per
+// sequence (decode), or a bf16 copy of codes x scales for the other index kernels.
+bool nvfp4_keys_supported(const Problem& P);
+cudaError_t launch_index_nvfp4_keys(const Problem& P, const void* q_codes, const void* k_codes,
+                                    float* bmax, cudaStream_t s);
+cudaError_t launch_dequant_nvfp4(const void* codes, const uint8_t* scales, void* out_bf16,
+                                 long long rows, int di, cudaStream_t s);
 // One query row per sequence whose rows all keep top_k blocks (q_pos0 >=
 // (top_k-1)*Bk): the top-k kernel also writes the block -> query lists (entries,
 // positions, tile records), in the layout launch_lists_direct gives them.

@@ -21,7 +21,10 @@ bool pow2_divides_128(int g) { return g >= 1 && g <= 128 && (128 % g) == 0; }
 // Shape checks shared by every entry point.
 msa_status_t resolve(const msa_problem_t* p, Problem* P) {
   if (!p) return MSA_ERR_INVALID_ARG;
-  if (p->index_dtype != 0 && !(p->index_dtype == MSA_FP8_E4M3 && p->dtype == MSA_BF16))
+  if (p->index_dtype != 0 && !((p->index_dtype == MSA_FP8_E4M3 || p->index_dtype == MSA_NVFP4) &&
+                                p->dtype == MSA_BF16))
+    return MSA_ERR_INVALID_ARG;
+  if (p->index_dtype == MSA_NVFP4 && (!p->q_idx_scale || !p->k_idx_scale))
     return MSA_ERR_INVALID_ARG;
   if (p->qk_dtype != 0 && !(p->qk_dtype == MSA_FP8_E4M3 && p->dtype == MSA_BF16))
     return MSA_ERR_INVALID_ARG;
@@ -65,6 +68,9 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
   P->scale = p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / sqrtf((float)p->head_dim);
   P->f32 = p->dtype == MSA_F32;
   P->idx8 = p->index_dtype == MSA_FP8_E4M3;
+  P->idx4 = p->index_dtype == MSA_NVFP4;
+  P->qsc = P->idx4 ? p->q_idx_scale : nullptr;
+  P->ksc = P->idx4 ? p->k_idx_scale : nullptr;
   P->qk8 = p->qk_dtype == MSA_FP8_E4M3;
   if (p->num_pages < 0 || (p->num_pages > 0 && !p->block_table)) return MSA_ERR_INVALID_ARG;
   if (p->num_pages > 0 && p->block_size != 128) return MSA_ERR_UNSUPPORTED;  // page = block
@@ -80,8 +86,21 @@ msa_status_t resolve(const msa_problem_t* p, Problem* P) {
 // Workspace layout (each region 256-byte aligned, in this order).
 struct Layout {
   size_t status, bmax, q2k, counts, cursor, list_off, tile_off, entries, pos, tiles, seg_sums,
-      part_o, part_lse, kl_rows, kl_ds, total;
+      part_o, part_lse, kl_rows, kl_ds, idx_q, idx_k, total;
 };
+
+// NVFP4 index tensors that the key-streaming kernel does not take are decoded
+// to bf16 in the workspace first; the index branch then runs on this problem.
+bool nvfp4_decoded(const Problem& P) { return P.idx4 && !msa::nvfp4_keys_supported(P); }
+
+Problem index_problem(const Problem& P) {
+  Problem Q = P;
+  if (nvfp4_decoded(P)) {
+    Q.idx4 = false;
+    Q.qsc = Q.ksc = nullptr;
+  }
+  return Q;
+}
 
 Layout layout(const Problem& P, int op) {
   Layout L{};
@@ -93,12 +112,17 @@ Layout layout(const Problem& P, int op) {
   const bool sel = op == MSA_OP_SELECT || op == MSA_OP_FORWARD;
   const bool att = op == MSA_OP_ATTEND || op == MSA_OP_FORWARD;
   const bool kl = op == MSA_OP_INDEX_KL;
+  const Problem PI = index_problem(P);
   // the index branch's scratch: partial selection lists when the selection is
   // fused into the index kernel, else the block maxima
-  L.bmax = sel ? take(msa::index_select_fused_supported(P)
-                          ? msa::index_select_cand_bytes(P)
+  L.bmax = sel ? take(msa::index_select_fused_supported(PI)
+                          ? msa::index_select_cand_bytes(PI)
                           : size_t(P.Hkv) * T * P.nblk * sizeof(float))
                : 0;
+  if (sel && nvfp4_decoded(P)) {  // bf16 copies of q_idx and k_idx
+    L.idx_q = take(T * P.Hkv * P.DI * 2);
+    L.idx_k = take(size_t(P.kv_rows) * P.DI * 2);
+  }
   L.q2k = op == MSA_OP_FORWARD ? take(size_t(P.Hkv) * T * P.K * sizeof(int32_t)) : 0;
   if (att || kl) {
     L.counts = take(size_t(P.nlists) * 4);
@@ -162,12 +186,23 @@ msa::Lists lists_of(void* ws, const Layout& L) {
 
 // run_select's top-k also writes the block -> query lists (lists != nullptr):
 // msa_forward on one query row per sequence whose rows all keep top_k blocks.
-msa_status_t run_select(const Problem& P, const void* q_idx, const void* k_idx, int32_t* q2k,
+msa_status_t run_select(const Problem& P0, const void* q_idx, const void* k_idx, int32_t* q2k,
                         float* bscores, void* ws, cudaStream_t s,
                         const msa::Lists* lists = nullptr) {
-  const Layout L = layout(P, MSA_OP_SELECT);
+  const Layout L = layout(P0, MSA_OP_SELECT);
   float* bmax = bscores ? bscores : at<float>(ws, L.bmax);
-  cudaError_t e = msa::launch_check_table(P, at<int32_t>(ws, L.status), s);
+  cudaError_t e = msa::launch_check_table(P0, at<int32_t>(ws, L.status), s);
+  // NVFP4 codes: the key-streaming kernel reads them as they are; otherwise
+  // they are decoded (exactly) to bf16 and the bf16 kernels run on the copies
+  if (e == cudaSuccess && nvfp4_decoded(P0)) {
+    e = msa::launch_dequant_nvfp4(q_idx, P0.qsc, at<void>(ws, L.idx_q),
+                                  (long long)P0.T * P0.Hkv, P0.DI, s);
+    if (e == cudaSuccess)
+      e = msa::launch_dequant_nvfp4(k_idx, P0.ksc, at<void>(ws, L.idx_k), P0.kv_rows, P0.DI, s);
+    q_idx = at<void>(ws, L.idx_q);
+    k_idx = at<void>(ws, L.idx_k);
+  }
+  const Problem P = index_problem(P0);
   if (!bscores && msa::index_select_fused_supported(P)) {
     // selection streamed inside the index kernel, then a merge of the partial lists
     if (e == cudaSuccess) {
@@ -185,7 +220,8 @@ msa_status_t run_select(const Problem& P, const void* q_idx, const void* k_idx, 
     e = msa::launch_fill(bscores, size_t(P.Hkv) * P.T * P.nblk, -INFINITY, s);
   if (e == cudaSuccess) {
     int32_t* status = at<int32_t>(ws, L.status);
-    e = msa::index_tc_supported(P)       ? msa::launch_index_tc(P, q_idx, k_idx, bmax, status, s)
+    e = P.idx4                           ? msa::launch_index_nvfp4_keys(P, q_idx, k_idx, bmax, s)
+        : msa::index_tc_supported(P)     ? msa::launch_index_tc(P, q_idx, k_idx, bmax, status, s)
         : msa::index_decode_supported(P) ? msa::launch_index_decode(P, q_idx, k_idx, bmax, status, s)
                                          : msa::launch_index_simt(P, q_idx, k_idx, bmax, s);
     stage_mark(s);
@@ -235,7 +271,8 @@ msa_status_t forward_one(const Problem& P, const void* q, const void* k, const v
   int32_t* q2k = q2k_opt ? q2k_opt : at<int32_t>(ws, L.q2k);
   // the select stage only needs the status word and bmax, which sit at the same
   // offsets in the forward layout
-  const bool topk_lists = msa::topk_writes_lists(P) && !msa::index_select_fused_supported(P);
+  const bool topk_lists =
+      msa::topk_writes_lists(P) && !msa::index_select_fused_supported(index_problem(P));
   const msa::Lists lists = lists_of(ws, L);
   msa_status_t st = run_select(P, q_idx, k_idx, q2k, nullptr, ws, s, topk_lists ? &lists : nullptr);
   if (st != MSA_OK) return st;
@@ -515,7 +552,7 @@ int32_t msa_launch_count(const msa_problem_t* p, int32_t op) {
   Problem P;
   if (resolve(p, &P) != MSA_OK || P.T == 0) return 0;
   const int chk = P.table ? 1 : 0;                  // block table check (paged)
-  const int sel = chk + 2;                         // index + top-k
+  const int sel = chk + 2 + (nvfp4_decoded(P) ? 2 : 0);  // (NVFP4 decode x 2) index + top-k
   // lists (+ tile records on the tensor-core path) + attention + combine
   const int att = chk +
                   (msa::lists_direct(P) ? 1
@@ -526,7 +563,8 @@ int32_t msa_launch_count(const msa_problem_t* p, int32_t op) {
     case MSA_OP_ATTEND: return att;
     case MSA_OP_FORWARD:
       // the decode top-k writes the lists itself (one launch fewer)
-      return sel + att - (msa::topk_writes_lists(P) && !msa::index_select_fused_supported(P));
+      return sel + att - (msa::topk_writes_lists(P) &&
+                          !msa::index_select_fused_supported(index_problem(P)));
     case MSA_OP_INDEX_KL: return chk + msa::kLaunchesInvert + 3;  // lists, rows, dk, sum
   }
   return 0;
@@ -536,11 +574,14 @@ const char* msa_kernel_path(const msa_problem_t* p, int32_t op) {
   Problem P;
   if (resolve(p, &P) != MSA_OK) return "invalid";
   const bool atc = msa::attn_tc_supported(P);
-  const int ik = msa::index_tc_supported(P) ? 0 : msa::index_decode_supported(P) ? 1 : 2;
-  static const char* sel[3] = {"index:tc", "index:stream", "index:simt"};
-  static const char* fwd[3][2] = {{"index:tc attn:simt", "index:tc attn:tc"},
+  const Problem PI = index_problem(P);
+  const int ik = PI.idx4 ? 3
+                 : msa::index_tc_supported(PI) ? 0 : msa::index_decode_supported(PI) ? 1 : 2;
+  static const char* sel[4] = {"index:tc", "index:stream", "index:simt", "index:nvfp4-keys"};
+  static const char* fwd[4][2] = {{"index:tc attn:simt", "index:tc attn:tc"},
                                   {"index:stream attn:simt", "index:stream attn:tc"},
-                                  {"index:simt attn:simt", "index:simt attn:tc"}};
+                                  {"index:simt attn:simt", "index:simt attn:tc"},
+                                  {"index:nvfp4-keys attn:simt", "index:nvfp4-keys attn:tc"}};
   switch (op) {
     case MSA_OP_SELECT: return sel[ik];
     case MSA_OP_ATTEND: return atc ? "attn:tc" : "attn:simt";

@@ -68,6 +68,9 @@ extern "C" msa_status_t msa_select_static(const msa_problem_t* p, const void* q_
     return MSA_ERR_INVALID_ARG;
   const size_t bmax_bytes = size_t(P.Hkv) * size_t(P.T) * size_t(P.nblk) * sizeof(float);
   if (bmax_bytes > kMaxBmaxBytes) return MSA_ERR_TOO_LARGE;
+  // NVFP4 only where the key-streaming kernel reads the codes directly (the
+  // other index kernels need a bf16 copy, which has no room here)
+  if (P.idx4 && !msa::nvfp4_keys_supported(P)) return MSA_ERR_UNSUPPORTED;
 
   void* scratch = nullptr;
   if (msa_status_t cst = msa::status_of(scratch_on_current_device(&scratch))) return cst;
@@ -78,7 +81,8 @@ extern "C" msa_status_t msa_select_static(const msa_problem_t* p, const void* q_
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
   if (e == cudaSuccess) e = msa::launch_check_table(P, status, s);
   if (e == cudaSuccess)
-    e = msa::index_tc_supported(P)       ? msa::launch_index_tc(P, q_idx, k_idx, bmax, status, s)
+    e = P.idx4                           ? msa::launch_index_nvfp4_keys(P, q_idx, k_idx, bmax, s)
+        : msa::index_tc_supported(P)     ? msa::launch_index_tc(P, q_idx, k_idx, bmax, status, s)
         : msa::index_decode_supported(P) ? msa::launch_index_decode(P, q_idx, k_idx, bmax, status, s)
                                          : msa::launch_index_simt(P, q_idx, k_idx, bmax, s);
   if (e == cudaSuccess) e = msa::launch_topk(P, bmax, q2k, s);

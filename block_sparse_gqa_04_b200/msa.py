@@ -18,7 +18,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
-MSA_BF16, MSA_F32, MSA_FP8_E4M3 = 0, 1, 2
+MSA_BF16, MSA_F32, MSA_FP8_E4M3, MSA_NVFP4 = 0, 1, 2, 3
 OP_SELECT, OP_ATTEND, OP_FORWARD, OP_INDEX_KL = 0, 1, 2, 3
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
@@ -52,6 +52,7 @@ class Problem(ctypes.Structure):
         ("q_pos0", ctypes.c_int64), ("softmax_scale", ctypes.c_float),
         ("index_dtype", ctypes.c_int32), ("qk_dtype", ctypes.c_int32),
         ("num_pages", ctypes.c_int32), ("block_table", ctypes.c_void_p),
+        ("q_idx_scale", ctypes.c_void_p), ("k_idx_scale", ctypes.c_void_p),
     ]
 
 
@@ -108,28 +109,37 @@ def load() -> ctypes.CDLL:
 def make_problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
                  block_size=128, top_k=16, dtype=torch.bfloat16, q_pos0=0,
                  softmax_scale=0.0, index_dtype=None, qk_dtype=None, num_pages=0,
-                 block_table=None) -> Problem:
+                 block_table=None, index_scales=None) -> Problem:
     """dtype: torch dtype of v and out (and of every other tensor unless stated:
     fp32 or bf16); index_dtype / qk_dtype: torch dtype of q_idx/k_idx / of q/k
     when it differs (torch.float8_e4m3fn for fp8 tensors).  num_pages > 0 with
     block_table (an int32 CUDA tensor [batch, ceil(kv_len/128)]) describes a
-    paged KV cache: k, v [num_pages, 128, Hkv, D], k_idx [num_pages, 128, di]."""
+    paged KV cache: k, v [num_pages, 128, Hkv, D], k_idx [num_pages, 128, di].
+    index_scales = (q_idx_scale, k_idx_scale), uint8 CUDA tensors, makes the
+    index tensors NVFP4 (index_dim counts elements, two per stored byte)."""
     fp8 = torch.float8_e4m3fn
     main = MSA_F32 if dtype == torch.float32 else MSA_BF16
     idx = MSA_FP8_E4M3 if (index_dtype == fp8 or dtype == fp8) else 0
+    qsc = ksc = None
+    if index_scales is not None:
+        idx = MSA_NVFP4
+        qsc, ksc = (t.data_ptr() for t in index_scales)
     qk = MSA_FP8_E4M3 if qk_dtype == fp8 else 0
     table = block_table.data_ptr() if block_table is not None else None
     return Problem(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, index_dim,
                    block_size, top_k, main, q_pos0, softmax_scale, idx, qk,
-                   num_pages if block_table is not None else 0, table)
+                   num_pages if block_table is not None else 0, table, qsc, ksc)
 
 
-def problem_of(w, softmax_scale: float = 0.0) -> Problem:
-    """Problem of a :class:`~block_sparse_gqa_04_b200.workload.Workload`."""
+def problem_of(w, softmax_scale: float = 0.0, index_scales=None) -> Problem:
+    """Problem of a :class:`~block_sparse_gqa_04_b200.workload.Workload` (an
+    NVFP4 workload needs its scale tensors, whose addresses the problem holds)."""
+    if w.index_dtype == "nvfp4" and index_scales is None:
+        raise ValueError("an NVFP4 problem needs index_scales=(q_idx_scale, k_idx_scale)")
     return make_problem(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
                         w.head_dim, w.index_dim, w.block_size, w.top_k, w.torch_dtype,
                         w.q_pos0, softmax_scale, index_dtype=w.torch_index_dtype,
-                        qk_dtype=w.torch_qk_dtype)
+                        qk_dtype=w.torch_qk_dtype, index_scales=index_scales)
 
 
 def workspace_size(p: Problem, op: int = OP_FORWARD) -> int:
@@ -231,11 +241,34 @@ def _paged(block_table, kv_len, batch, num_pages, block_size):
     return {"num_pages": int(num_pages), "block_table": block_table}
 
 
+def _index_dim(q_idx: torch.Tensor) -> int:
+    """Elements per index row: NVFP4 codes (uint8) hold two per byte."""
+    return q_idx.shape[-1] * (2 if q_idx.dtype == torch.uint8 else 1)
+
+
+def _check_scales(q_idx, k_idx, index_scales):
+    """NVFP4 index tensors (uint8 codes [.., di/2]) come with their uint8 ue4m3
+    scales [.., di/16]; other dtypes with none."""
+    if q_idx.dtype != torch.uint8:
+        if index_scales is not None:
+            raise ValueError("index_scales are for NVFP4 (uint8) index tensors only")
+        return
+    if index_scales is None or len(index_scales) != 2:
+        raise ValueError("NVFP4 (uint8) q_idx/k_idx need index_scales=(q_idx_scale, k_idx_scale)")
+    if q_idx.shape[-1] % 8 != 0:
+        raise ValueError("NVFP4 index rows hold a multiple of 16 elements")
+    for name, t, sc in (("q_idx", q_idx, index_scales[0]), ("k_idx", k_idx, index_scales[1])):
+        want = tuple(t.shape[:-1]) + (t.shape[-1] // 8,)
+        if sc.dtype != torch.uint8 or tuple(sc.shape) != want:
+            raise ValueError(f"{name}_scale must be uint8 {want}, got {sc.dtype} {tuple(sc.shape)}")
+    _require_cuda(*index_scales)
+
+
 def _check_index_pair(q_idx: torch.Tensor, k_idx: torch.Tensor, paged: bool = False) -> int:
     """q_idx [B, Sq, Hkv, di] and k_idx [B, Skv, di] (paged: [pages, 128, di])
     of one dtype: the index kernels read k_idx with q_idx's element size and
     batch, so a mismatch would read past the end of k_idx.  Returns Skv (the
-    rows per page for a paged cache)."""
+    rows per page for a paged cache).  NVFP4 codes have di/2 bytes per row."""
     if q_idx.dim() != 4:
         raise ValueError(f"q_idx must be [B, Sq, Hkv, di], got {tuple(q_idx.shape)}")
     B, _, _, di = q_idx.shape
@@ -250,17 +283,23 @@ def _check_index_pair(q_idx: torch.Tensor, k_idx: torch.Tensor, paged: bool = Fa
 
 def select(q_idx: torch.Tensor, k_idx: torch.Tensor, *, q_pos0: int = 0, block_size: int = 128,
            top_k: int = 16, return_block_scores: bool = False,
-           workspace: Optional[torch.Tensor] = None, block_table=None, kv_len=None):
+           workspace: Optional[torch.Tensor] = None, block_table=None, kv_len=None,
+           index_scales=None):
     """Index branch: returns q2k [Hkv, B*Sq, top_k] int32 (and block scores).
-    With block_table and kv_len, k_idx is a paged cache [pages, 128, di]."""
+    With block_table and kv_len, k_idx is a paged cache [pages, 128, di].  NVFP4
+    index tensors: uint8 codes [.., di/2] with index_scales=(q_idx_scale,
+    k_idx_scale), uint8 [.., di/16]."""
     Skv = _check_index_pair(q_idx, k_idx, paged=block_table is not None)
+    _check_scales(q_idx, k_idx, index_scales)
     _require_cuda(q_idx, k_idx)
-    B, Sq, Hkv, di = q_idx.shape
+    B, Sq, Hkv, _ = q_idx.shape
+    di = _index_dim(q_idx)
     if block_table is not None:
         Skv = int(kv_len) if kv_len is not None else None
     pg = _paged(block_table, kv_len, B, k_idx.shape[0], block_size)
-    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, top_k, q_idx.dtype, q_pos0,
-                     index_dtype=q_idx.dtype, **pg)
+    main = torch.bfloat16 if q_idx.dtype in (torch.uint8, torch.float8_e4m3fn) else q_idx.dtype
+    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, top_k, main, q_pos0,
+                     index_dtype=q_idx.dtype, index_scales=index_scales, **pg)
     dev = q_idx.device
     q2k = torch.empty((Hkv, B * Sq, top_k), dtype=torch.int32, device=dev)
     nblk = -(-Skv // block_size)
@@ -275,21 +314,25 @@ def select(q_idx: torch.Tensor, k_idx: torch.Tensor, *, q_pos0: int = 0, block_s
 
 def select_static(q_idx: torch.Tensor, k_idx: torch.Tensor, q2k: torch.Tensor, *,
                   q_pos0: int = 0, block_size: int = 128,
-                  device_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+                  device_status: Optional[torch.Tensor] = None,
+                  index_scales=None) -> torch.Tensor:
     """Index branch through msa_select_static, which allocates nothing: the
     caller passes the output q2k [Hkv, B*Sq, top_k] int32 (and optionally a
     one-element int32 device tensor that receives the device status word).
     For callers that cannot lend the library device memory; the library's
     fixed scratch is shared, so calls must not overlap on the GPU."""
     Skv = _check_index_pair(q_idx, k_idx)
+    _check_scales(q_idx, k_idx, index_scales)
     _require_cuda(q_idx, k_idx, q2k, device_status)
-    B, Sq, Hkv, di = q_idx.shape
+    B, Sq, Hkv, _ = q_idx.shape
+    di = _index_dim(q_idx)
     if q2k.dtype != torch.int32 or tuple(q2k.shape[:2]) != (Hkv, B * Sq):
         raise ValueError("q2k must be int32 [Hkv, B*Sq, top_k]")
     if device_status is not None and device_status.dtype != torch.int32:
         raise ValueError("device_status must be an int32 tensor")
-    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, q2k.shape[2], q_idx.dtype, q_pos0,
-                     index_dtype=q_idx.dtype)
+    main = torch.bfloat16 if q_idx.dtype in (torch.uint8, torch.float8_e4m3fn) else q_idx.dtype
+    p = make_problem(B, Sq, Skv, Hkv, Hkv, 64, di, block_size, q2k.shape[2], main, q_pos0,
+                     index_dtype=q_idx.dtype, index_scales=index_scales)
     _check(load().msa_select_static(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(q2k),
                                     _ptr(device_status), _stream(q_idx.device)),
            "msa_select_static")
@@ -464,7 +507,8 @@ def _forward_host(q, k, v, q_idx, k_idx, block_table, out, dev, kw, ret_lse, ret
 def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, top_k: int = 16,
             softmax_scale: float = 0.0, return_lse: bool = False, return_q2k: bool = False,
             workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-            device=None, check_device_status: bool = False, block_table=None, kv_len=None):
+            device=None, check_device_status: bool = False, block_table=None, kv_len=None,
+            index_scales=None):
     """Index branch + main branch.  Returns out (and lse, q2k when asked).
 
     CUDA tensors are used in place.  Host tensors (ideally pinned) are copied to
@@ -474,8 +518,13 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
     the call and raises if the device recorded a problem (a bounded wait that
     gave up).  With block_table ([B, ceil(kv_len/128)] int32) and kv_len, k, v
     and k_idx are a paged KV cache: [pages, 128, Hkv, D] and [pages, 128, di].
+    NVFP4 index tensors (device tensors only): uint8 codes [.., di/2] with
+    index_scales=(q_idx_scale, k_idx_scale), uint8 [.., di/16].
     """
     _check_index_pair(q_idx, k_idx, paged=block_table is not None)
+    _check_scales(q_idx, k_idx, index_scales)
+    if not q.is_cuda and index_scales is not None:
+        raise ValueError("NVFP4 index tensors are taken on the device only")
     if not q.is_cuda:
         for t in (k, v, q_idx, k_idx):
             if t.is_cuda:
@@ -491,7 +540,8 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
         return _forward_host(q, k, v, q_idx, k_idx, block_table, out,
                              torch.device(device or "cuda"), kw, return_lse, return_q2k)
     _require_cuda(q, k, v, q_idx, k_idx)
-    B, Sq, Hq, D, Skv, Hkv, di = _dims(q, k, q_idx, v=v, k_idx=k_idx, kv_len=kv_len)
+    B, Sq, Hq, D, Skv, Hkv, _ = _dims(q, k, q_idx, v=v, k_idx=k_idx, kv_len=kv_len)
+    di = _index_dim(q_idx)
     pg = _paged(block_table, kv_len, B, k.shape[0], block_size)
     _check_qkv_dtypes(q, k, v)
     if out is not None and (out.dtype != v.dtype or tuple(out.shape) != tuple(q.shape)
@@ -499,7 +549,8 @@ def forward(q, k, v, q_idx, k_idx, *, q_pos0: int = 0, block_size: int = 128, to
         raise ValueError(f"out must be a contiguous {tuple(q.shape)} tensor of v's dtype "
                          f"{v.dtype}, got {tuple(out.shape)} {out.dtype}")
     p = make_problem(B, Sq, Skv, Hq, Hkv, D, di, block_size, top_k, v.dtype, q_pos0,
-                     softmax_scale, index_dtype=q_idx.dtype, qk_dtype=q.dtype, **pg)
+                     softmax_scale, index_dtype=q_idx.dtype, qk_dtype=q.dtype,
+                     index_scales=index_scales, **pg)
     dev = q.device
     o = out if out is not None else torch.empty(q.shape, dtype=v.dtype, device=dev)
     lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=dev) if return_lse else None

@@ -22,6 +22,10 @@ Recipe (the same for every workload):
     token of a drawn block gets ``0.5 * mean_i q_idx[b, i, g, :]`` added to its
     index key, in fp32, before k_idx is rounded to bf16 (the mean is taken over
     the sequence's stored, already rounded q_idx rows).
+  * index_dtype "nvfp4": q_idx and k_idx (needles included) are drawn the same
+    way in fp32 and then encoded to NVFP4 by quantize_nvfp4 (the needle shift
+    uses the mean of the fp32 q_idx draws); the inputs are the codes and the
+    scales, and both sides decode them.
 """
 from __future__ import annotations
 
@@ -47,7 +51,8 @@ class Workload:
     top_k: int
     dtype: str          # "f32" or "bf16"
     needles: int        # planted needle blocks per (sequence, group)
-    index_dtype: str = ""  # "" (same as dtype) or "fp8" (q_idx, k_idx in fp8 e4m3)
+    index_dtype: str = ""  # "" (same as dtype), "fp8" (q_idx, k_idx in fp8 e4m3) or
+                           # "nvfp4" (e2m1 codes, two per byte, + a ue4m3 scale per 16)
     qk_dtype: str = ""     # "" (same as dtype) or "fp8" (q, k in fp8 e4m3; v stays bf16)
 
     @property
@@ -64,6 +69,8 @@ class Workload:
 
     @property
     def torch_index_dtype(self) -> torch.dtype:
+        if self.index_dtype == "nvfp4":
+            return torch.uint8
         return torch.float8_e4m3fn if self.index_dtype == "fp8" else self.torch_dtype
 
     @property
@@ -112,6 +119,41 @@ def _draw(gen: torch.Generator, shape, scale: float, dtype: torch.dtype) -> torc
     return out
 
 
+# NVFP4 encoding of drawn inputs: the sixteen e2m1 magnitudes' grid and the
+# 127 finite unsigned e4m3 scale values (codes 0x00 .. 0x7e), ascending.
+_E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def _ue4m3_table() -> list:
+    vals = []
+    for code in range(127):
+        e, m = code >> 3, code & 7
+        vals.append(m * 2.0 ** -9 if e == 0 else 2.0 ** (e - 7) * (1 + m / 8))
+    return vals
+
+
+def quantize_nvfp4(x: torch.Tensor):
+    """Encodes fp32 values [..., d] (d a multiple of 16) as NVFP4: per group of
+    16 the smallest ue4m3 scale s with max|x| / s <= 6, then each x / s to the
+    nearest e2m1 value (halfway cases to the smaller magnitude), sign kept.
+    Returns (codes uint8 [..., d/2], element 2i in the low nibble; scales
+    uint8 [..., d/16])."""
+    d = x.shape[-1]
+    g = x.float().reshape(*x.shape[:-1], d // 16, 16)
+    table = torch.tensor(_ue4m3_table(), dtype=torch.float32, device=x.device)
+    target = (g.abs().amax(-1) / 6.0).contiguous()
+    sc = torch.searchsorted(table, target).clamp(max=126)
+    sval = table[sc].unsqueeze(-1)
+    q = torch.where(sval > 0, g / torch.where(sval > 0, sval, torch.ones_like(sval)),
+                    torch.zeros_like(g))
+    mids = torch.tensor([(a + b) / 2 for a, b in zip(_E2M1_GRID, _E2M1_GRID[1:])],
+                        dtype=torch.float32, device=x.device)
+    idx = torch.searchsorted(mids, q.abs().contiguous())
+    code = (idx | torch.where(q < 0, 8, 0)).to(torch.uint8).reshape(*x.shape[:-1], d)
+    packed = code[..., 0::2] | (code[..., 1::2] << 4)
+    return packed.contiguous(), sc.to(torch.uint8).contiguous()
+
+
 def needle_upper(w: Workload) -> int:
     first = w.q_pos0 // w.block_size
     return first if first > 0 else (w.q_pos0 + w.q_len - 1) // w.block_size
@@ -124,10 +166,12 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu") -> Dict[str, torch.Ten
     s_main = 1.0 if w.dtype == "f32" else 1.0 / math.sqrt(w.head_dim)
     s_idx = 1.0 if w.dtype == "f32" else 1.0 / math.sqrt(w.index_dim)
     B, Sq, Skv = w.batch, w.q_len, w.kv_len
+    nvfp4 = w.index_dtype == "nvfp4"
     q = _draw(gen, (B * Sq, w.num_q_heads, w.head_dim), s_main, w.torch_qk_dtype)
     k = _draw(gen, (B * Skv, w.num_kv_heads, w.head_dim), s_main, w.torch_qk_dtype)
     v = _draw(gen, (B * Skv, w.num_kv_heads, w.head_dim), s_main, dt)
-    q_idx = _draw(gen, (B * Sq, w.num_kv_heads, w.index_dim), s_idx, w.torch_index_dtype)
+    q_idx = _draw(gen, (B * Sq, w.num_kv_heads, w.index_dim), s_idx,
+                  torch.float32 if nvfp4 else w.torch_index_dtype)
     # k_idx stays fp32 until the needles are in, then is rounded once.
     k_idx32 = _draw(gen, (B * Skv, w.index_dim), s_idx, torch.float32)
     needle_ids = torch.full((B, w.num_kv_heads, max(w.needles, 0)), -1, dtype=torch.int64,
@@ -147,15 +191,23 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu") -> Dict[str, torch.Ten
                     lo = c * w.block_size
                     hi = min(lo + w.block_size, Skv)
                     kv[b, lo:hi] += shift
-    k_idx = k_idx32.to(w.torch_index_dtype)
-    return {
+    out = {
         "q": q.view(B, Sq, w.num_q_heads, w.head_dim),
         "k": k.view(B, Skv, w.num_kv_heads, w.head_dim),
         "v": v.view(B, Skv, w.num_kv_heads, w.head_dim),
-        "q_idx": q_idx.view(B, Sq, w.num_kv_heads, w.index_dim),
-        "k_idx": k_idx.view(B, Skv, w.index_dim),
         "needles": needle_ids,
     }
+    if nvfp4:
+        qc, qs = quantize_nvfp4(q_idx)
+        kc, ks = quantize_nvfp4(k_idx32)
+        di = w.index_dim
+        out.update(q_idx=qc.view(B, Sq, w.num_kv_heads, di // 2),
+                   q_idx_scale=qs.view(B, Sq, w.num_kv_heads, di // 16),
+                   k_idx=kc.view(B, Skv, di // 2), k_idx_scale=ks.view(B, Skv, di // 16))
+        return out
+    out.update(q_idx=q_idx.view(B, Sq, w.num_kv_heads, w.index_dim),
+               k_idx=k_idx32.to(w.torch_index_dtype).view(B, Skv, w.index_dim))
+    return out
 
 
 def sample_rows(w: Workload, n: int, seed: int = 0) -> list:

@@ -70,8 +70,12 @@ typedef enum {
 /* MSA_FP8_E4M3 is an index_dtype or qk_dtype only: fp8 e4m3 index queries and
  * keys, or main-branch queries and keys, of a bf16 problem ("MiniMax új
  * eljárása ..." (aiforradalom.online), section "Elérhetőség": the MSA inference
- * kernels come in BF16, FP8, NVFP4 and FP4). */
-typedef enum { MSA_BF16 = 0, MSA_F32 = 1, MSA_FP8_E4M3 = 2 } msa_dtype_t;
+ * kernels come in BF16, FP8, NVFP4 and FP4).  MSA_NVFP4 is an index_dtype only:
+ * NVFP4 index queries and keys of a bf16 problem, e2m1 codes two per byte
+ * (element 2i in the low nibble) with one unsigned e4m3 scale byte per 16
+ * consecutive elements of index_dim (q_idx_scale, k_idx_scale); a value is
+ * e2m1(code) x scale, and scale bytes 0x7f and above are invalid. */
+typedef enum { MSA_BF16 = 0, MSA_F32 = 1, MSA_FP8_E4M3 = 2, MSA_NVFP4 = 3 } msa_dtype_t;
 
 typedef enum {
   MSA_OP_SELECT = 0,
@@ -100,7 +104,9 @@ typedef struct {
   int64_t q_pos0;         /* absolute position of query row 0 of every sequence */
   float softmax_scale;    /* main-branch logit scale; 0 selects 1/sqrt(head_dim) */
   int32_t index_dtype;    /* 0: q_idx and k_idx have `dtype`; MSA_FP8_E4M3: they are
-                             fp8 e4m3 (bf16 problems); other values are invalid  */
+                             fp8 e4m3; MSA_NVFP4: they are NVFP4 codes
+                             [.., index_dim/2] uint8 with the scales below (both
+                             bf16 problems only); other values are invalid       */
   int32_t qk_dtype;       /* 0: q and k have `dtype`; MSA_FP8_E4M3: q and k are fp8
                              e4m3 and the main-branch scores q . k are formed from
                              them (bf16 problems; v, out and the partial states stay
@@ -117,6 +123,12 @@ typedef struct {
   const int32_t* block_table; /* device, [batch, ceil(kv_len/128)] int32 page ids in
                              [0, num_pages) (num_pages > 0), else ignored; an id
                              outside that range sets status bit 4 and reads page 0 */
+  const uint8_t* q_idx_scale; /* device, index_dtype MSA_NVFP4 only (else ignored):
+                             ue4m3 scales of q_idx, [batch, q_len, num_kv_heads,
+                             index_dim/16]                                        */
+  const uint8_t* k_idx_scale; /* device, MSA_NVFP4 only: scales of k_idx, [batch,
+                             kv_len, index_dim/16] (paged: [num_pages, 128,
+                             index_dim/16]); both must be non-NULL for MSA_NVFP4  */
 } msa_problem_t;
 
 /* Bytes of workspace that `op` needs for problem `p` (0 if p is invalid).

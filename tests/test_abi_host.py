@@ -348,3 +348,44 @@ def test_varlen_binding_checks_shapes_before_any_launch():
     x = workload.make_varlen_inputs([3, 2], [10, 4], 8, 2, 64, 32)
     with pytest.raises(ValueError):
         msa.forward_varlen(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], x["cu_q"], x["cu_k"])
+
+
+def test_nvfp4_problems_on_the_host(lib):
+    # NVFP4 index tensors need both scale pointers and a bf16 problem; the decode
+    # rows stream the codes, prefill shapes decode a bf16 copy (two more launches
+    # and the copies' room in the workspace)
+    sc = torch.zeros(16, dtype=torch.uint8)
+    dec = msa.make_problem(6, 1, 3000, 64, 4, 128, 128, top_k=16, q_pos0=2999,
+                           index_dtype=torch.uint8, index_scales=(sc, sc))
+    assert msa.kernel_path(dec) == "index:nvfp4-keys attn:tc"
+    bf = msa.make_problem(6, 1, 3000, 64, 4, 128, 128, top_k=16, q_pos0=2999)
+    assert msa.launch_count(dec) == msa.launch_count(bf)  # one index kernel either way
+    pre = msa.make_problem(1, 700, 2200, 64, 4, 128, 128, top_k=8, q_pos0=1500,
+                           index_dtype=torch.uint8, index_scales=(sc, sc))
+    pre_bf = msa.make_problem(1, 700, 2200, 64, 4, 128, 128, top_k=8, q_pos0=1500)
+    assert msa.kernel_path(pre) == msa.kernel_path(pre_bf) == "index:tc attn:tc"
+    assert msa.launch_count(pre) == msa.launch_count(pre_bf) + 2
+    copies = 700 * 4 * 128 * 2 + 2200 * 128 * 2
+    assert msa.workspace_size(pre) >= msa.workspace_size(pre_bf) + copies
+    # invalid: a missing scale pointer, an fp32 problem
+    bad = msa.make_problem(1, 700, 2200, 64, 4, 128, 128, top_k=8, q_pos0=1500,
+                           index_dtype=torch.uint8, index_scales=(sc, sc))
+    bad.k_idx_scale = None
+    assert msa.workspace_size(bad) == 0
+    f32 = msa.make_problem(1, 64, 64, 8, 2, 64, 32, top_k=4, dtype=torch.float32,
+                           index_dtype=torch.uint8, index_scales=(sc, sc))
+    assert msa.workspace_size(f32) == 0
+    # the training-side loss does not take NVFP4 index tensors
+    assert lib.msa_index_kl(ctypes.byref(pre), *([ctypes.c_void_p(1 << 20)] * 8),
+                            ctypes.c_void_p(1 << 20), 1 << 30, None) == 2
+
+
+def test_nvfp4_binding_checks_scales():
+    codes_q = torch.zeros((1, 4, 2, 64), dtype=torch.uint8)
+    codes_k = torch.zeros((1, 300, 64), dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        msa.select(codes_q, codes_k, top_k=4)  # no scales
+    with pytest.raises(ValueError):
+        msa.select(codes_q, codes_k, top_k=4,
+                   index_scales=(torch.zeros((1, 4, 2, 4), dtype=torch.uint8),
+                                 torch.zeros((1, 300, 8), dtype=torch.uint8)))
