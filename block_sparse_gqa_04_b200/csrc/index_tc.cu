@@ -18,17 +18,27 @@
 //     by the groups' MMAs, so shared memory only feeds B;
 //   * two 128-column fp32 accumulators alternate, so the epilogue of one unit
 //     overlaps the MMAs of the next.
-// Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
+// Warp roles: warp 0 issues TMA, warp 1 owns TMEM, warps 1 and 10 issue the
+// MMAs of the units of accumulator slot 0 and slot 1 (alternate units), warps
 // 2-9 load index queries into TMEM and run the epilogue (one query row per
 // thread: masked max over the row's 128 columns, one fp32 store per unit).
 // The epilogue is two warpgroups, one per accumulator, so that two units drain
-// at once while the tensor cores fill the next.
+// at once while the tensor cores fill the next.  Two issuing threads keep the
+// MMA pipe fed: it queues one instruction, and the barrier tests, commits and
+// loop work one thread does between its units would otherwise leave it idle
+// (one thread: ~950 SM cycles per 512-cycle unit; two: 7 % faster for the GEMM
+// and 4 % with the streamed selection at 128K).  A thread's commits track only
+// its own MMAs, so the k_idx stage and the query region are released by both
+// (their barriers count two arrivals).
 //
 // Streaming selection (FUSE): instead of writing the block maxima, each
-// epilogue thread keeps, for each group its warpgroup drains, the top (k-1)
+// epilogue thread keeps, for each group its warpgroup drains, the largest
 // keys (orderable score, lower id on ties) of the earlier blocks c < floor(t/Bk)
-// of its query row, as a min-heap in shared memory with its root in registers
-// ("MiniMax lancerer MSA" (snilld.dk), section "Teknisk forklaring hvorfor
+// of its query row, in a descending array of kMaxKeep entries in shared memory
+// with its last entry in a register.  A new key enters with a branch-free
+// insertion (entry i becomes max(a[i], min(a[i-1], key))), the same
+// instructions on every lane, so a warp pays one pass however many of its rows
+// take the key ("MiniMax lancerer MSA" (snilld.dk), section "Teknisk forklaring hvorfor
 // kompleksiteten skifter": the top-k over raw block scores is where the gain
 // can be lost, so the block scores never make an HBM round trip).  A query
 // tile's blocks may be split between the contiguous shares of neighbouring
@@ -47,7 +57,7 @@ namespace msa {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 320;               // TMA, MMA, two epilogue warpgroups
+constexpr int kThreads = 352;               // TMA, MMA, two epilogue warpgroups, 2nd MMA
 constexpr int kMaxGroups = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 256;           // accumulators follow the A region
@@ -183,15 +193,15 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&bars->full[s], 1);
-      tc::mbar_init(&bars->empty[s], 1);
+      tc::mbar_init(&bars->empty[s], 2);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->acc_full[s], 1);
       tc::mbar_init(&bars->acc_empty[s], 4);
     }
     tc::mbar_init(&bars->a_full, 8);
-    tc::mbar_init(&bars->a_empty, 1);
-    tc::mbar_init(&bars->mma_done, 1);
+    tc::mbar_init(&bars->a_empty, 2);
+    tc::mbar_init(&bars->mma_done, 2);
     bars->abort = 0;
     tc::fence_mbar_init();
   }
@@ -229,13 +239,14 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       // every copy issued has landed before the CTA can leave
       if (!armed.drain(bars->full)) failed = true;
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 1 || warp == 10) {
+    // ---------------- MMA issuers: warp 1 the units of slot 0, warp 10 of slot 1 ----------------
+    const int me = warp == 1 ? 0 : 1;
     if (lane == 0 && L0 < L1) {
       Walk w;
       w.start(P, L0, per_seq);
-      int stage = 0, slot = 0;
-      uint32_t phase = 0, acc_phase = 0, a_phase = 0;
+      int stage = 0;
+      uint32_t phase = 0, a_phase = 0, n = 0;
       bool seg_start = true;
       for (long long L = L0; L < L1 && !failed; ++L) {
         if (seg_start) {
@@ -246,8 +257,10 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
         if (!tc::mbar_spin(&bars->full[stage], phase, abort)) { failed = true; break; }
         tc::tc_fence_after();
         const uint32_t sbase = tc::smem_addr(stages + stage * X::kStageBytes);
-        for (int g = 0; g < P.Hkv; ++g) {
-          if (!tc::mbar_spin(&bars->acc_empty[slot], acc_phase ^ 1, abort)) {
+        for (int g = 0; g < P.Hkv; ++g, ++n) {
+          const int slot = int(n & 1);
+          if (slot != me) continue;
+          if (!tc::mbar_spin(&bars->acc_empty[slot], ((n >> 1) & 1) ^ 1, abort)) {
             failed = true;
             break;
           }
@@ -264,8 +277,6 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
               tc::mma_ts(d, tmem + g * X::kGroupCols + kk * 8, bd, X::kIdesc, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&bars->acc_full[slot]);
-          slot ^= 1;
-          if (slot == 0) acc_phase ^= 1;
         }
         if (failed) break;
         tc::mma_commit(&bars->empty[stage]);
@@ -276,7 +287,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
       // every MMA issued has completed before TMEM is freed
       if (!tc::mma_drain(&bars->mma_done)) failed = true;
     }
-  } else {
+  } else if (warp <= 9) {
     // ---------------- index-query loader + epilogue (two warpgroups) ----------------
     const int ewg = (warp - 2) >> 2;        // accumulator slot this warpgroup drains
     const int quarter = warp & 3;           // TMEM lanes this warp may touch
@@ -284,10 +295,14 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
     const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
     const int et = threadIdx.x - 64;        // epilogue thread: the keep lists' column
     const int nkeep = P.K - 1;
-    // per group of this warpgroup (g = ewg + 2j): number of kept keys, the
-    // smallest of them (0 while fewer than nkeep are kept)
-    int cnt0 = 0, cnt1 = 0;
-    uint64_t mkey0 = 0, mkey1 = 0;
+    // per group of this warpgroup (g = ewg + 2j): the smallest of the kMaxKeep
+    // kept keys (0, below every key, while fewer are kept).  The arrays start
+    // empty: all zero.
+    uint64_t low0 = 0, low1 = 0;
+    if (FUSE) {
+#pragma unroll
+      for (int e = 0; e < 2 * kMaxKeep; ++e) keep[size_t(e) * kEpiThreads + et] = 0;
+    }
     if (L0 < L1) {
       Walk w;
       w.start(P, L0, per_seq);
@@ -368,67 +383,49 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, Problem P,
                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
           if (!FUSE) {
             if (valid) bmax[((long long)g * P.T + r) * P.nblk + w.c] = m;
-          } else if (valid && earlier && nkeep > 0) {
-            // an earlier block of this row (c < floor(t/Bk)): keep its key if
-            // it is among the nkeep largest so far
+          } else if (nkeep > 0) {
+            // an earlier block of this row (c < floor(t/Bk)) enters the kept
+            // keys if it beats the smallest; the insertion runs on every lane
+            // of the warp once any lane needs it (0 leaves the array as it is)
             const int j = g >> 1;
-            uint64_t* kl = keep + size_t(j) * kMaxKeep * kEpiThreads + et;
-            const uint64_t key = block_key(m, w.c);
-            // the kept keys form a binary min-heap (root = smallest kept key,
-            // also held in mkey): filling sifts a key up, replacing the root
-            // sifts the new key down, at most log2(16) levels either way
-            auto offer = [&](int& cnt, uint64_t& mkey) {
-              int pos;
-              if (cnt < nkeep) {
-                pos = cnt++;
-                while (pos > 0) {
-                  const int up = (pos - 1) >> 1;
-                  const uint64_t pk = kl[up * kEpiThreads];
-                  if (pk <= key) break;
-                  kl[pos * kEpiThreads] = pk;
-                  pos = up;
-                }
-              } else if (key > mkey) {
-                pos = 0;
-                for (;;) {
-                  const int l = 2 * pos + 1;
-                  if (l >= nkeep) break;
-                  uint64_t ck = kl[l * kEpiThreads];
-                  int c2 = l;
-                  if (l + 1 < nkeep) {
-                    const uint64_t rk = kl[(l + 1) * kEpiThreads];
-                    if (rk < ck) { ck = rk; c2 = l + 1; }
-                  }
-                  if (ck >= key) break;
-                  kl[pos * kEpiThreads] = ck;
-                  pos = c2;
-                }
-              } else {
-                return;
+            const uint64_t key = (valid && earlier) ? block_key(m, w.c) : 0;
+            if (__any_sync(MSA_FULL_MASK, key > (j ? low1 : low0))) {
+              uint64_t* kl = keep + size_t(j) * kMaxKeep * kEpiThreads + et;
+              uint64_t a[kMaxKeep];
+#pragma unroll
+              for (int e = 0; e < kMaxKeep; ++e) a[e] = kl[size_t(e) * kEpiThreads];
+              uint64_t prev = a[0];
+              a[0] = a[0] > key ? a[0] : key;
+#pragma unroll
+              for (int e = 1; e < kMaxKeep; ++e) {
+                const uint64_t up = prev < key ? prev : key;  // min(old a[e-1], key)
+                prev = a[e];
+                a[e] = a[e] > up ? a[e] : up;
               }
-              kl[pos * kEpiThreads] = key;
-              mkey = cnt < nkeep ? 0 : kl[0];
-            };
-            if (j == 0) offer(cnt0, mkey0);
-            else offer(cnt1, mkey1);
+#pragma unroll
+              for (int e = 0; e < kMaxKeep; ++e) kl[size_t(e) * kEpiThreads] = a[e];
+              if (j) low1 = a[kMaxKeep - 1];
+              else low0 = a[kMaxKeep - 1];
+            }
           }
         }
         if (FUSE && nkeep > 0 && (w.c + 1 == w.nc || L + 1 == L1)) {
-          // end of this CTA's share of the query tile: its partial lists go to
-          // the CTA's slot among the tile's shares (unused entries are 0, below
-          // every key)
-          if (valid) {
-            const long long T0 = (long long)w.b * per_seq + pairs_before_at(P, w.u, per_seq);
-            const int slot = int(blockIdx.x) - cta_of_pair(T0, per_seq * P.B, gridDim.x);
-            for (int j = 0; 2 * j + ewg < P.Hkv; ++j) {
-              const int g = 2 * j + ewg;
-              const int cnt = j ? cnt1 : cnt0;
-              const uint64_t* kl = keep + size_t(j) * kMaxKeep * kEpiThreads + et;
-              uint64_t* dst = cand + ((size_t(g) * nslot + slot) * nkeep) * P.T + r;
-              for (int e = 0; e < nkeep; ++e) dst[size_t(e) * P.T] = e < cnt ? kl[e * kEpiThreads] : 0;
-            }
+          // end of this CTA's share of the query tile: its partial lists (the
+          // nkeep largest kept keys; 0, below every key, where fewer were
+          // kept) go to the CTA's slot among the tile's shares, and the arrays
+          // start empty again
+          const long long T0 = (long long)w.b * per_seq + pairs_before_at(P, w.u, per_seq);
+          const int slot = int(blockIdx.x) - cta_of_pair(T0, per_seq * P.B, gridDim.x);
+          for (int j = 0; 2 * j + ewg < P.Hkv; ++j) {
+            const int g = 2 * j + ewg;
+            uint64_t* kl = keep + size_t(j) * kMaxKeep * kEpiThreads + et;
+            uint64_t* dst = cand + ((size_t(g) * nslot + slot) * nkeep) * P.T + r;
+            for (int e = 0; e < nkeep; ++e)
+              if (valid) dst[size_t(e) * P.T] = kl[size_t(e) * kEpiThreads];
+#pragma unroll
+            for (int e = 0; e < kMaxKeep; ++e) kl[size_t(e) * kEpiThreads] = 0;
           }
-          cnt0 = cnt1 = 0;
+          low0 = low1 = 0;
         }
         seg_start = w.next(P);
       }
@@ -539,7 +536,7 @@ int sm_count() {
 }  // namespace
 
 bool index_tc_supported(const Problem& P) {
-  return !P.f32 && !P.idx4 && P.DI == 128 && P.Bk == 128 && P.Hkv <= kMaxGroups && P.Sq > 8 &&
+  return !P.f32 && P.DI == 128 && P.Bk == 128 && P.Hkv <= kMaxGroups && P.Sq > 8 &&
          P.kv_rows < (1LL << 31);
 }
 
