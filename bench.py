@@ -320,8 +320,8 @@ def run_e2e(msa, w, xh, out_h, steps, warmup):
 NCU_TRAFFIC = {
     # stage: (workload, source file, git blob id, bytes per launch)
     "attn": ("prefill_128k", "block_sparse_gqa_04_b200/csrc/attn_tc.cu",
-             "95f0d7f1c440128b0586d8654bf0d3d8bdd585d3",
-             round((394030080 + 2957622016) * 8327168 / 724992)),
+             "d88ea0f99b5bd71195a3ac24e70e86333f30b3a0",
+             round((407079424 + 2957662464) * 8327168 / 724992)),
 }
 
 

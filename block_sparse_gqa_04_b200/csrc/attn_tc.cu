@@ -30,6 +30,14 @@
 // issued as soon as its previous P V has completed, so it overlaps the
 // previous tile's epilogue.  Each softmax thread holds its whole S row (and
 // later its O row) in registers, so a tile costs one TMEM round trip each.
+// Two threads issue the MMAs, one per TMEM buffer (warp 1 the even tiles, warp
+// 10 the odd ones), each in a straight line: wait for the tile's descriptor,
+// K/V, Q and its buffer's previous P V, issue S, wait for P, issue P V.  (One
+// thread polling every barrier of both buffers noticed a ready P up to ~900
+// cycles late; two straight-line threads cut the attention by ~4.5 %.)  A
+// thread's commits track only its own MMAs, so a K/V buffer is released by the
+// last tile of each parity in the list's run (the producer stands in for the
+// missing parity of a one-tile run): its empty barrier counts two arrivals.
 //
 // With fp8 (e4m3) q and k (aiforradalom.online "Elérhetőség": the inference
 // kernels come in BF16 and FP8 among others) the score product S = Q K^T runs as
@@ -49,7 +57,7 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 320;                 // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
+constexpr int kThreads = 352;                 // warp 0 TMA, warps 1, 10 MMA, warps 2-9 softmax
 constexpr int kRows = 128;
 constexpr int kTileBytes = kRows * 128 * 2;   // 32 KB: 128 rows x 128 dims of bf16
 constexpr int kHalf = kTileBytes / 2;         // one 64-dim half of a bf16 tile
@@ -82,7 +90,8 @@ constexpr int kDesc = 4;  // tile descriptors in flight
 
 // What the producer warp tells the MMA warp and the softmax warps about a tile.
 struct TileDesc {
-  int c, e0, n, flags;     // flags: 1 new list, 2 last tile of its list here, kv stage << 2
+  int c, e0, n, flags;     // flags: 1 new list, 2 last tile of its list here, 4 kv stage,
+                          // 8 last tile of its parity in the list, 16 kv load parity
   int rows[kQPerTile];     // query rows of the gathered queries
 };
 
@@ -92,7 +101,7 @@ struct Bars {
   uint64_t s_full[2], p_full[2], o_full[2], buf_empty[2];
   uint64_t d_full[kDesc], d_empty[kDesc];
   TileDesc desc[kDesc];
-  uint64_t mma_done;       // the MMA thread's final commit (drain before TMEM is freed)
+  uint64_t mma_done;       // the MMA threads' final commits (drain before TMEM is freed)
   uint32_t tmem_base;
   int abort;
 };
@@ -207,7 +216,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->kv_full[s], 1);
-      tc::mbar_init(&bars->kv_empty[s], 1);
+      tc::mbar_init(&bars->kv_empty[s], 2);  // both MMA issuers (or one + the producer)
       tc::mbar_init(&bars->s_full[s], 1);
       tc::mbar_init(&bars->p_full[s], 4);
       tc::mbar_init(&bars->o_full[s], 1);
@@ -215,9 +224,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     }
     for (int d = 0; d < kDesc; ++d) {
       tc::mbar_init(&bars->d_full[d], 1);
-      tc::mbar_init(&bars->d_empty[d], 5);  // the MMA thread and the four softmax warps
+      tc::mbar_init(&bars->d_empty[d], 5);  // the tile's MMA thread and its four softmax warps
     }
-    tc::mbar_init(&bars->mma_done, 1);
+    tc::mbar_init(&bars->mma_done, 2);
     bars->abort = 0;
     tc::fence_mbar_init();
   }
@@ -246,6 +255,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     const uint64_t q_policy = tc::policy_evict_last();
     int kv_stage = 0, q_stage = 0;
     uint32_t kv_phase = 0, q_phase = 0;
+    int cur_kvs = 0;
+    uint32_t cur_kvpar = 0;
     int prev_lid = -1;
     tc::ArmedRing q_armed, kv_armed;  // lane 0: copies issued into each ring
     auto fetch = [&](int j, TileRec& r) -> bool {
@@ -265,6 +276,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       const int j = jb + lane;
       const long long nt = tile_of(j + 1);
       const int last = cur_ok && !(nt < total && nt < cur.tend);
+      // tile j + 1 is the last of the run: j is the last of its parity too
+      int next_last = __shfl_down_sync(MSA_FULL_MASK, last, 1);
+      {
+        const int tend0 = __shfl_sync(MSA_FULL_MASK, nxt.tend, 0);
+        const int ok0 = __shfl_sync(MSA_FULL_MASK, nxt_ok ? 1 : 0, 0);
+        if (lane == 31) {
+          const long long nnt = tile_of(j + 2);
+          next_last = ok0 && !(nnt < total && nnt < tend0);
+        }
+      }
+      const int release = cur_ok && (last || (next_last && nt < total && nt < cur.tend));
       int lid_prev = __shfl_up_sync(MSA_FULL_MASK, cur.lid, 1);
       if (lane == 0) lid_prev = prev_lid;
       const int new_list = cur_ok && cur.lid != lid_prev;
@@ -279,6 +301,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const int tn = __shfl_sync(MSA_FULL_MASK, cur.n, jj);
         const int tnew = __shfl_sync(MSA_FULL_MASK, new_list, jj);
         const int tlast = __shfl_sync(MSA_FULL_MASK, last, jj);
+        const int trel = __shfl_sync(MSA_FULL_MASK, release, jj);
         int trow[kQPerTile];
 #pragma unroll
         for (int e = 0; e < kQPerTile; ++e) trow[e] = __shfl_sync(MSA_FULL_MASK, cur.rows[e], jj);
@@ -296,6 +319,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
               if (!QK8) tc::tma_load_3d(dst + kHalf, &tmap_k, fb, 64, tg, key0);
               tc::tma_load_3d(dst + C::kKBytes, &tmap_v, fb, 0, tg, key0);
               tc::tma_load_3d(dst + C::kKBytes + kHalf, &tmap_v, fb, 64, tg, key0);
+              cur_kvs = kv_stage;
+              cur_kvpar = kv_phase;
+              // a one-tile run has one issuer: the producer stands in for the other
+              if (tlast) tc::mbar_arrive(&bars->kv_empty[kv_stage]);
             }
           }
           good = good && tc::mbar_wait(&bars->q_empty[q_stage], q_phase ^ 1, abort);
@@ -330,7 +357,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             D.c = tc_;
             D.e0 = te0;
             D.n = tn;
-            D.flags = (tnew ? 1 : 0) | (tlast ? 2 : 0) | ((tnew ? kv_stage : (kv_stage ^ 1)) << 2);
+            D.flags = (tnew ? 1 : 0) | (tlast ? 2 : 0) | (cur_kvs << 2) | (trel ? 8 : 0) |
+                      int(cur_kvpar << 4);
 #pragma unroll
             for (int e = 0; e < kQPerTile; ++e) D.rows[e] = trow[e];
             tc::mbar_arrive(&bars->d_full[d]);
@@ -350,97 +378,57 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     // too: the copies complete whether or not anyone consumes them)
     if (lane == 0 && !(q_armed.drain(bars->q_full) && kv_armed.drain(bars->kv_full))) failed = true;
     if (lane != 0) failed = false;  // lane 0 speaks for the warp
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    // Event loop: issue S = Q K^T of the next tile as soon as its descriptor,
-    // K/V, Q and TMEM buffer are ready, and O = P V of the oldest tile as soon
-    // as its P is in TMEM, whichever comes first.  At most two tiles are in
-    // flight (one per TMEM buffer).  The barriers are tested without blocking
-    // (a blocking test of one would hide the other becoming ready).
+  } else if (warp == 1 || warp == 10) {
+    // ---------------- MMA issuers: warp 1 the tiles of TMEM buffer 0, warp 10 of buffer 1 ----------------
+    const int me = warp == 1 ? 0 : 1;
     if (lane == 0) {
-      uint32_t kv_phase[2] = {0, 0};
-      int ns = 0, np = 0;
-      uint32_t idle = 0;
-      uint32_t sgot = 0;  // barriers of tile ns already seen complete (each is polled until then)
-      while (tile_of(np) < total) {
-        bool progress = false;
-        // O = P V first (it is on its warpgroup's path).  Its P implies that the
-        // O columns are drained: the same four warps read the buffer's previous O
-        // before they wrote this P.
-        if (np < ns && tc::mbar_poll(&bars->p_full[np & 1], (np >> 1) & 1)) {
-          tc::tc_fence_after();
-          const int buf = np & 1, d = np % kDesc;
-          const int flags = bars->desc[d].flags;
-          const int kvs = flags >> 2;
-          const uint32_t va = tc::smem_addr(kvbuf + kvs * C::kKVBytes + C::kKBytes);
-          const uint32_t o = tmem + buf * 256 + 128;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            tc::mma_ts(o, tmem + buf * 256 + kk * 8, tc::sdesc_sw128(va + kk * 2048, kHalf, 1024),
-                       kIdescO, kk > 0 ? 1u : 0u);
-          }
-          tc::mma_commit(&bars->o_full[buf]);
-          if (flags & 2) tc::mma_commit(&bars->kv_empty[kvs]);
-          tc::mbar_arrive(&bars->d_empty[d]);
-          ++np;
-          progress = true;
-        }
-        if (ns < np + 2 && tile_of(ns) < total) {
-          const int d = ns % kDesc, buf = ns & 1, qs = ns % kQStages;
-          if (!(sgot & 1) && tc::mbar_poll(&bars->d_full[d], (ns / kDesc) & 1)) sgot |= 1;
-          if (sgot & 1) {
-            const int flags = bars->desc[d].flags;
-            const int kvs = flags >> 2;
-            // S overwrites only the S|P columns of its buffer, which are free
-            // once the P V product of the buffer's previous tile has completed
-            if (!(sgot & 2) && (!(flags & 1) || tc::mbar_poll(&bars->kv_full[kvs], kv_phase[kvs])))
-              sgot |= 2;
-            if (!(sgot & 4) && tc::mbar_poll(&bars->q_full[qs], (ns / kQStages) & 1)) sgot |= 4;
-            if (!(sgot & 8) && tc::mbar_poll(&bars->o_full[buf], ((ns >> 1) & 1) ^ 1)) sgot |= 8;
-            if (sgot == 15) {
-              tc::tc_fence_after();
-              const uint32_t qa = tc::smem_addr(qbuf + qs * C::kQStageBytes);
-              const uint32_t ka = tc::smem_addr(kvbuf + kvs * C::kKVBytes);
-              const uint32_t dt = tmem + buf * 256;
-              if (QK8) {
-                // fp8: 128-byte rows of 128 dims, K = 32 per MMA
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  tc::mma_ss_f8(dt, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
-                                tc::sdesc_sw128(ka + kk * 32, 16, 1024), C::kIdescS,
-                                kk > 0 ? 1u : 0u);
-              } else {
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                  const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                  // Q: 8-row groups 2 KB apart, the 64-dim halves 1 KB apart inside
-                  const uint32_t qoff = (kk >> 2) * 1024 + (kk & 3) * 32;
-                  tc::mma_ss(dt, tc::sdesc_sw128(qa + qoff, 16, 2048),
-                             tc::sdesc_sw128(ka + off, 16, 1024), C::kIdescS, kk > 0 ? 1u : 0u);
-                }
-              }
-              tc::mma_commit(&bars->s_full[buf]);
-              if (QK8) tc::mma_commit(&bars->q_empty[qs]);  // the Q stage is read
-              if (flags & 1) kv_phase[kvs] ^= 1;
-              sgot = 0;
-              ++ns;
-              progress = true;
-            }
-          }
-        }
-        // the idle loop polls without sleeping: a sleep delays the issue of the
-        // next MMA group by up to its length while the pipe runs dry
-        if (progress) {
-          idle = 0;
-        } else if (++idle > tc::kWaitLimit || (idle > 64 && *abort)) {
+      for (int ns = me; tile_of(ns) < total && !failed; ns += 2) {
+        const int d = ns % kDesc, buf = me, qs = ns % kQStages;
+        if (!tc::mbar_spin(&bars->d_full[d], (ns / kDesc) & 1, abort)) { failed = true; break; }
+        const int flags = bars->desc[d].flags;
+        const int kvs = (flags >> 2) & 1;
+        if (!tc::mbar_spin(&bars->kv_full[kvs], (flags >> 4) & 1, abort) ||
+            !tc::mbar_spin(&bars->q_full[qs], (ns / kQStages) & 1, abort) ||
+            !tc::mbar_spin(&bars->o_full[buf], ((ns >> 1) & 1) ^ 1, abort)) {
           failed = true;
           break;
         }
+        tc::tc_fence_after();
+        const uint32_t qa = tc::smem_addr(qbuf + qs * C::kQStageBytes);
+        const uint32_t ka = tc::smem_addr(kvbuf + kvs * C::kKVBytes);
+        const uint32_t dt = tmem + buf * 256;
+        if (QK8) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc::mma_ss_f8(dt, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
+                          tc::sdesc_sw128(ka + kk * 32, 16, 1024), C::kIdescS, kk > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+            const uint32_t qoff = (kk >> 2) * 1024 + (kk & 3) * 32;
+            tc::mma_ss(dt, tc::sdesc_sw128(qa + qoff, 16, 2048),
+                       tc::sdesc_sw128(ka + off, 16, 1024), C::kIdescS, kk > 0 ? 1u : 0u);
+          }
+        }
+        tc::mma_commit(&bars->s_full[buf]);
+        if (QK8) tc::mma_commit(&bars->q_empty[qs]);  // the Q stage is read
+        if (!tc::mbar_spin(&bars->p_full[buf], (ns >> 1) & 1, abort)) { failed = true; break; }
+        tc::tc_fence_after();
+        const uint32_t va = ka + C::kKBytes;
+        const uint32_t o = tmem + buf * 256 + 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_ts(o, tmem + buf * 256 + kk * 8, tc::sdesc_sw128(va + kk * 2048, kHalf, 1024),
+                     kIdescO, kk > 0 ? 1u : 0u);
+        tc::mma_commit(&bars->o_full[buf]);
+        if (flags & 8) tc::mma_commit(&bars->kv_empty[kvs]);
+        tc::mbar_arrive(&bars->d_empty[d]);
       }
       // every MMA issued has completed before TMEM is freed
       if (!tc::mma_drain(&bars->mma_done)) failed = true;
     }
-  } else {
+  } else if (warp <= 9) {
     // ---------------- softmax + epilogue (two warpgroups) ----------------
     const int wg = (warp - 2) >> 2;          // tiles j with j % 2 == wg, TMEM buffer wg
     const int quarter = warp & 3;
