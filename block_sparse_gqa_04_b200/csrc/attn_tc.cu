@@ -177,16 +177,13 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint32_t to_bf16x2(uint64_t x) {
   return pack_bf16(__uint_as_float(uint32_t(x)), __uint_as_float(uint32_t(x >> 32)));
 }
-// 2^x for both bf16 halves
-__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
+// 2^x in fp32 on the exp2 unit (flushes subnormal results to zero)
+__device__ __forceinline__ float ex2_f32(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// the two bf16 halves widened to fp32 (exact)
-__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t p) {
-  return (uint64_t(p & 0xffff0000u) << 32) | uint64_t(p << 16);
-}
+
 
 template <bool QK8>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -466,10 +463,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       m = fmaxf(fmaxf(m, max32(v[1], -INFINITY)), fmaxf(max32(v[2], -INFINITY),
                                                        max32(v[3], -INFINITY)));
       const float ms = m * sl2;
-      // P = 2^(S*scale*log2e - max), written over S, and its sum, two columns
-      // at a time: the scaled logits (packed fp32x2 FMA) are rounded to bf16
-      // and exponentiated with the bf16x2 exp2, which gives P in the bf16 the
-      // P V product takes at half the exp2-unit cost
+      // P = 2^(S*scale*log2e - max), written over S as bf16, and its sum in
+      // fp32, two columns at a time: the scaled logits come from packed fp32x2
+      // FMAs, the exponentials from the fp32 exp2 (the exp2 unit takes the same
+      // time per value in fp32 as in bf16x2, and this loop is bound by issue
+      // slots: summing fp32 values saves widening the bf16 ones, -3 % for the
+      // kernel), and each pair is rounded once to bf16x2 for the P V product
       const uint64_t sl2x2 = f2(sl2, sl2), nmsx2 = f2(-ms, -ms);
       uint64_t lsum[2] = {0, 0};
 #pragma unroll
@@ -478,9 +477,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
           const uint64_t z = fma2((uint64_t(v[q4][x + 1]) << 32) | v[q4][x], sl2x2, nmsx2);
-          const uint32_t pp = ex2_bf16x2(to_bf16x2(z));
-          lsum[(x >> 1) & 1] = add2(lsum[(x >> 1) & 1], bf16x2_to_f2(pp));
-          pw[x >> 1] = pp;
+          const float pa = ex2_f32(__uint_as_float(uint32_t(z)));
+          const float pb = ex2_f32(__uint_as_float(uint32_t(z >> 32)));
+          lsum[(x >> 1) & 1] = add2(lsum[(x >> 1) & 1], f2(pa, pb));
+          pw[x >> 1] = pack_bf16(pa, pb);
         }
         tmem_st16(sbase + q4 * 16, pw);  // P columns 16*q4.. (S is all in registers)
       }
