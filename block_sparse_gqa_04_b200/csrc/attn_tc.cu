@@ -21,9 +21,10 @@
 //     the local block, and write P (bf16) back over S in TMEM;
 //   * O = P V runs with P from TMEM and V as an MN-major shared-memory operand;
 //   * the softmax warps normalise O by the row sum, stage the bf16 rows in the
-//     tile's own Q buffer (free once S is done) and store them with TMA (each
-//     warp its own 32 rows, which are contiguous in the entry-ordered partial
-//     states); the base-2 log-normaliser goes with them.
+//     tile's own Q buffer (free once S is done) and copy them out with
+//     coalesced 16-byte stores (each warp its own 32 rows, which are contiguous
+//     in the entry-ordered partial states), leaving the TMA unit to the Q
+//     gathers; the base-2 log-normaliser goes with them.
 // Two softmax warpgroups take alternate tiles, each with its own TMEM buffer
 // pair (S|P, O) of 256 columns, so two tiles are in their softmax while the
 // tensor cores run the MMAs of their neighbours; a buffer's next S = Q K^T is
@@ -190,9 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_v,
-               const __grid_constant__ CUtensorMap tmap_o32,
-               const __grid_constant__ CUtensorMap tmap_o16, Problem P, Lists L,
-               float* __restrict__ part_lse, int* __restrict__ status) {
+               Problem P, Lists L,
+               float* __restrict__ part_lse, int* __restrict__ status,
+               uint8_t* __restrict__ part_o) {
   using C = Cfg<QK8>;
   constexpr int kQStages = C::kQStages;
   extern __shared__ uint8_t smem_raw[];
@@ -231,8 +232,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     tc::tma_prefetch(&tmap_q);
     tc::tma_prefetch(&tmap_k);
     tc::tma_prefetch(&tmap_v);
-    tc::tma_prefetch(&tmap_o32);
-    tc::tma_prefetch(&tmap_o16);
   }
   if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
   tc::tc_fence_before();
@@ -495,16 +494,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       // Stage the normalised bf16 O row in this tile's Q buffer (bf16 q/k: S is
       // done with it) or in the warpgroup's staging area (fp8 q/k).  Each warp
       // owns 32 consecutive rows (two gathered queries, contiguous in the
-      // entry-ordered partial states) and stores them itself with TMA.  The
-      // staging uses the 128-byte swizzle (16-byte chunk k of a row goes to
-      // chunk k ^ (row % 8)), which the TMA store undoes.
+      // entry-ordered partial states) and stores them itself.  The staging
+      // uses the 128-byte swizzle (16-byte chunk k of a row goes to chunk
+      // k ^ (row % 8)), so that the row-per-lane writes and the chunk-per-lane
+      // reads both spread over the banks.
       uint8_t* wst = QK8 ? obuf + wg * C::kOStageBytes + quarter * 8192
                          : qbuf + qs * C::kQStageBytes + quarter * 8192;
-      if (QK8) {
-        // this warp's previous store from the area must have read it
-        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        __syncwarp();
-      }
       const float inv = 1.f / l;
       const uint64_t invx2 = f2(inv, inv);
       uint32_t o[4][32];
@@ -530,26 +525,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&bars->buf_empty[wg]);
       if (valid) part_lse[(long long)(e0 + el) * kGroup + hh] = ms + __log2f(l);
-      tc::fence_async_smem();
-      __syncwarp();
+      // the warp's rows from the staging area to the partial states with
+      // coalesced 16-byte stores (two 256-byte rows per instruction), streaming
+      // past L2 (the combine reads them once); the load/store units carry them
+      // so that the TMA unit is left to the Q gathers
       const int nrows = min(32, n * kGroup - quarter * 32);  // 0, 16 or 32
+      uint8_t* gdst = part_o + (size_t(e0) * kGroup + quarter * 32) * 256;
+      for (int it = 0; it < nrows / 2; ++it) {
+        const int r = 2 * it + (lane >> 4), k = lane & 15;
+        const uint4 u = *reinterpret_cast<const uint4*>(wst + (k >> 3) * 4096 + r * 128 +
+                                                        (((k & 7) ^ (r & 7)) << 4));
+        __stcs(reinterpret_cast<uint4*>(gdst + r * 256 + k * 16), u);
+      }
+      __syncwarp();
       if (lane == 0) {
-        if (nrows > 0) {
-          const CUtensorMap* map = nrows == 32 ? &tmap_o32 : &tmap_o16;
-          const int grow = e0 * kGroup + quarter * 32;
-          // partial states are read once, by the combine: first out of L2
-          const uint64_t o_policy = tc::policy_evict_first();
-#pragma unroll
-          for (int h = 0; h < 2; ++h) tc::tma_store_2d_hint(map, wst + h * 4096, 64 * h, grow, o_policy);
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-          if (!QK8) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        }
-        // bf16: the Q buffer may be refilled once the store has read it
+        // bf16: the staging area is the tile's Q buffer, free again
         if (!QK8) tc::mbar_arrive(&bars->q_empty[qs]);
         tc::mbar_arrive(&bars->d_empty[d]);
       }
     }
-    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   if (failed) {
     bars->abort = 1;
@@ -599,7 +593,7 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
                            cudaStream_t s) {
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap mq, mk, mv, mo32, mo16;
+  CUtensorMap mq, mk, mv;
   const CUtensorMapDataType qk_type =
       P.qk8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const cuuint64_t qk_row = P.qk8 ? 128 : 256;  // bytes of one 128-dim row of q or k
@@ -641,27 +635,13 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  {
-    // partial states: [entries * 16 rows, 128 dims] bf16, stored 16 or 32 rows at a time
-    cuuint64_t dims[2] = {128, cuuint64_t(P.T) * P.Hq * P.K};
-    cuuint64_t strides[1] = {128 * 2};
-    cuuint32_t estr[2] = {1, 1};
-    cuuint32_t box32[2] = {64, 32}, box16[2] = {64, 16};
-    if (enc(&mo32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, part.o, dims, strides, box32, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-    if (enc(&mo16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, part.o, dims, strides, box16, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
   auto kern = P.qk8 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
   const size_t smem = P.qk8 ? smem_bytes<true>() : smem_bytes<false>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<sm_count(), kThreads, smem, s>>>(mq, mk, mv, mo32, mo16, P, L, part.lse2, status);
+  kern<<<sm_count(), kThreads, smem, s>>>(mq, mk, mv, P, L, part.lse2, status,
+                                           static_cast<uint8_t*>(part.o));
   return cudaGetLastError();
 }
 

@@ -162,11 +162,6 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
 
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map,
                                                  uint64_t* bar, int c0, int c1,
@@ -186,16 +181,6 @@ __device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* m
       " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
       "r"(smem_addr(bar)), "l"(policy)
-      : "memory");
-}
-
-// Tiled TMA store of a 2D box from shared memory (bulk-group completion).
-__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, const void* src,
-                                                  int c0, int c1, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint"
-      " [%0, {%1, %2}], [%3], %4;" ::"l"(reinterpret_cast<uint64_t>(map)),
-      "r"(c0), "r"(c1), "r"(smem_addr(src)), "l"(policy)
       : "memory");
 }
 
