@@ -20,33 +20,33 @@
 //   * the softmax warps read their row, apply the scale and the causal cut of
 //     the local block, and write P (bf16) back over S in TMEM;
 //   * O = P V runs with P from TMEM and V as an MN-major shared-memory operand;
-//   * the softmax warps normalise O by the row sum, stage the bf16 rows in the
-//     tile's own Q buffer (free once S is done) and copy them out with
-//     coalesced 16-byte stores (each warp its own 32 rows, which are contiguous
-//     in the entry-ordered partial states), leaving the TMA unit to the Q
-//     gathers; the base-2 log-normaliser goes with them.
+//   * the epilogue warps normalise O by the row sum, stage the bf16 rows in a
+//     shared-memory area and store them with TMA (each warp its own 32 rows,
+//     which are contiguous in the entry-ordered partial states); the softmax
+//     warps write the base-2 log-normaliser.
 // Two softmax warpgroups take alternate tiles, each with its own TMEM buffer
 // pair (S|P, O) of 256 columns, so two tiles are in their softmax while the
-// tensor cores run the MMAs of their neighbours; a buffer's next S = Q K^T is
-// issued as soon as its previous P V has completed, so it overlaps the
-// previous tile's epilogue.  Each softmax thread holds its whole S row (and
-// later its O row) in registers, so a tile costs one TMEM round trip each.
+// tensor cores run the MMAs of their neighbours.  A fourth warpgroup does the
+// epilogue of every tile, so a softmax warpgroup goes from one tile's P
+// straight to its next S, which is issued as soon as the previous P V has
+// completed.  The warpgroups trade registers (setmaxnreg) so that a softmax
+// thread holds its whole S row.  A Q stage is released as soon as its S
+// product has completed.
 // Two threads issue the MMAs, one per TMEM buffer (warp 1 the even tiles, warp
-// 10 the odd ones), each in a straight line: wait for the tile's descriptor,
-// K/V, Q and its buffer's previous P V, issue S, wait for P, issue P V.  (One
-// thread polling every barrier of both buffers noticed a ready P up to ~900
-// cycles late; two straight-line threads cut the attention by ~4.5 %.)  A
-// thread's commits track only its own MMAs, so a K/V buffer is released by the
-// last tile of each parity in the list's run (the producer stands in for the
-// missing parity of a one-tile run): its empty barrier counts two arrivals.
+// 2 the odd ones), each in a straight line: wait for the tile's descriptor,
+// K/V, Q and its buffer's previous P V, issue S, wait for P and for the
+// epilogue to have read the buffer's previous O, issue P V.  (One thread
+// polling every barrier of both buffers noticed a ready P up to ~900 cycles
+// late.)  A thread's commits track only its own MMAs, so a K/V buffer is
+// released by the last tile of each parity in the list's run (the producer
+// stands in for the missing parity of a one-tile run): its empty barrier counts
+// two arrivals.
 //
 // With fp8 (e4m3) q and k (aiforradalom.online "Elérhetőség": the inference
 // kernels come in BF16 and FP8 among others) the score product S = Q K^T runs as
 // kind::f8f6f4 MMAs on 128-byte rows (K = 32 per instruction) and P V stays
 // bf16.  A query's Q rows are then 2 KB (one 2D box of 16 rows), a Q stage 16 KB,
-// so four stages fit, and each stage is released as soon as its S product has
-// completed; the output rows are staged in a separate 32 KB area per softmax
-// warpgroup instead of the tile's Q stage.
+// and four stages fit.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -58,7 +58,8 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 352;                 // warp 0 TMA, warps 1, 10 MMA, warps 2-9 softmax
+// warp 0 TMA, warps 1-2 MMA, warp 3 idle, warps 4-11 softmax, warps 12-15 epilogue
+constexpr int kThreads = 512;
 constexpr int kRows = 128;
 constexpr int kTileBytes = kRows * 128 * 2;   // 32 KB: 128 rows x 128 dims of bf16
 constexpr int kHalf = kTileBytes / 2;         // one 64-dim half of a bf16 tile
@@ -73,10 +74,9 @@ template <bool QK8>
 struct Cfg {
   static constexpr int kQBox = QK8 ? 2048 : 4096;          // one query's 16 head rows
   static constexpr int kQStageBytes = kQPerTile * kQBox;   // 16 or 32 KB
-  static constexpr int kQStages = QK8 ? 4 : 3;
+  static constexpr int kQStages = QK8 ? 4 : 2;
   static constexpr int kKBytes = QK8 ? 16384 : kTileBytes; // 128 keys x 128 dims
   static constexpr int kKVBytes = kKBytes + kTileBytes;    // K then V
-  static constexpr int kOStageBytes = QK8 ? kTileBytes : 0;  // per warpgroup (else the Q stage)
   static constexpr uint32_t kIdescS =
       QK8 ? tc::idesc_e4m3_f32(128, 128) : tc::idesc_bf16_f32(128, 128, 0, 0);
 };
@@ -87,7 +87,7 @@ struct Cfg {
 // inside the same narrow window of the tile order, i.e. on the same query
 // chunk of the same group, whose Q rows then stay resident in L2.
 constexpr int kChunk = 8;
-constexpr int kDesc = 4;  // tile descriptors in flight
+constexpr int kDesc = 6;  // tile descriptors in flight
 
 // What the producer warp tells the MMA warp and the softmax warps about a tile.
 struct TileDesc {
@@ -99,9 +99,10 @@ struct TileDesc {
 struct Bars {
   uint64_t kv_full[2], kv_empty[2];
   uint64_t q_full[kMaxQStages], q_empty[kMaxQStages];
-  uint64_t s_full[2], p_full[2], o_full[2], buf_empty[2];
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2], l_full[2], l_empty[2];
   uint64_t d_full[kDesc], d_empty[kDesc];
   TileDesc desc[kDesc];
+  float lsum[2][kRows];    // row sums of P, softmax -> epilogue, per TMEM buffer
   uint64_t mma_done;       // the MMA threads' final commits (drain before TMEM is freed)
   uint32_t tmem_base;
   int abort;
@@ -110,8 +111,7 @@ struct Bars {
 template <bool QK8>
 constexpr size_t smem_bytes() {
   using C = Cfg<QK8>;
-  return 1024 + C::kQStages * C::kQStageBytes + 2 * C::kKVBytes + 2 * C::kOStageBytes +
-         sizeof(Bars) + 64;
+  return 1024 + C::kQStages * C::kQStageBytes + 2 * C::kKVBytes + kTileBytes + sizeof(Bars) + 64;
 }
 static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448,
               "shared memory of one CTA");
@@ -145,14 +145,27 @@ __device__ __forceinline__ float max32(const uint32_t (&v)[32], float m) {
   return fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
+}
+
+// Register split between the warpgroups (setmaxnreg acts on a whole
+// warpgroup): the CTA is launched with 512 x 128 registers; the producer/MMA
+// warpgroup gives 32 of each thread's back, the epilogue 64, and each softmax
+// warpgroup takes 48 more (96 + 64 + 2 x 176 = 512 = 4 x 128), so that a
+// softmax thread holds its whole S row.  No role spills at these counts.
+constexpr int kRegsCtl = 96, kRegsEpi = 64, kRegsSoftmax = 176;
+static_assert(kRegsCtl + kRegsEpi + 2 * kRegsSoftmax <= 4 * 128, "register split");
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Two-wide fp32 helpers (sm_100 packed FMA / add / mul on a 64-bit pair).
@@ -191,38 +204,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_v,
-               Problem P, Lists L,
-               float* __restrict__ part_lse, int* __restrict__ status,
-               uint8_t* __restrict__ part_o) {
+               const __grid_constant__ CUtensorMap tmap_o32,
+               const __grid_constant__ CUtensorMap tmap_o16, Problem P, Lists L,
+               float* __restrict__ part_lse, int* __restrict__ status) {
   using C = Cfg<QK8>;
   constexpr int kQStages = C::kQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qbuf = smem;                                  // [stages]: Q (bf16: then output staging)
+  uint8_t* qbuf = smem;                                  // [stages]: Q
   uint8_t* kvbuf = qbuf + kQStages * C::kQStageBytes;    // [2][K | V 32 KB]
-  uint8_t* obuf = kvbuf + 2 * C::kKVBytes;               // fp8 q/k: [2][32 KB] output staging
-  Bars* bars = reinterpret_cast<Bars*>(obuf + 2 * C::kOStageBytes);
+  uint8_t* obuf = kvbuf + 2 * C::kKVBytes;               // output staging, 32 KB
+  Bars* bars = reinterpret_cast<Bars*>(obuf + kTileBytes);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
       tc::mbar_init(&bars->q_full[s], 1);
-      // bf16: the four warps that stored the tile from it; fp8: the S MMAs' commit
-      tc::mbar_init(&bars->q_empty[s], QK8 ? 1 : 4);
+      tc::mbar_init(&bars->q_empty[s], 1);  // the S MMAs' commit
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->kv_full[s], 1);
       tc::mbar_init(&bars->kv_empty[s], 2);  // both MMA issuers (or one + the producer)
       tc::mbar_init(&bars->s_full[s], 1);
-      tc::mbar_init(&bars->p_full[s], 4);
+      tc::mbar_init(&bars->p_full[s], 4);    // the buffer's softmax warps
       tc::mbar_init(&bars->o_full[s], 1);
-      tc::mbar_init(&bars->buf_empty[s], 4);
+      tc::mbar_init(&bars->o_empty[s], 4);   // the epilogue warps have read O
+      tc::mbar_init(&bars->l_full[s], 4);    // the softmax warps wrote the row sums
+      tc::mbar_init(&bars->l_empty[s], 4);   // the epilogue warps read them
     }
     for (int d = 0; d < kDesc; ++d) {
       tc::mbar_init(&bars->d_full[d], 1);
-      tc::mbar_init(&bars->d_empty[d], 5);  // the tile's MMA thread and its four softmax warps
+      // the tile's MMA thread, its four softmax warps and the four epilogue warps
+      tc::mbar_init(&bars->d_empty[d], 9);
     }
     tc::mbar_init(&bars->mma_done, 2);
     bars->abort = 0;
@@ -232,6 +247,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     tc::tma_prefetch(&tmap_q);
     tc::tma_prefetch(&tmap_k);
     tc::tma_prefetch(&tmap_v);
+    tc::tma_prefetch(&tmap_o32);
+    tc::tma_prefetch(&tmap_o16);
   }
   if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
   tc::tc_fence_before();
@@ -240,8 +257,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
   const uint32_t tmem = bars->tmem_base;
   const int total = __ldg(L.tile_off + P.nlists);
   bool failed = false;
+  static_assert(kThreads == 512, "four warpgroups");
 
-  if (warp == 0) {
+  if (warp < 4) {
+   regs_dec<kRegsCtl>();
+   if (warp == 0) {
     // ---------------- producer: tile descriptors + TMA ----------------
     // Lane l holds the record of tile jb + l of this CTA (prefetched one batch
     // ahead); lane 0 waits for buffer space and issues the copies tile by tile.
@@ -374,9 +394,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     // too: the copies complete whether or not anyone consumes them)
     if (lane == 0 && !(q_armed.drain(bars->q_full) && kv_armed.drain(bars->kv_full))) failed = true;
     if (lane != 0) failed = false;  // lane 0 speaks for the warp
-  } else if (warp == 1 || warp == 10) {
-    // ---------------- MMA issuers: warp 1 the tiles of TMEM buffer 0, warp 10 of buffer 1 ----------------
-    const int me = warp == 1 ? 0 : 1;
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers: warp 1 the tiles of TMEM buffer 0, warp 2 of buffer 1 ----------------
+    const int me = warp - 1;
     if (lane == 0) {
       for (int ns = me; tile_of(ns) < total && !failed; ns += 2) {
         const int d = ns % kDesc, buf = me, qs = ns % kQStages;
@@ -408,8 +428,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
           }
         }
         tc::mma_commit(&bars->s_full[buf]);
-        if (QK8) tc::mma_commit(&bars->q_empty[qs]);  // the Q stage is read
-        if (!tc::mbar_spin(&bars->p_full[buf], (ns >> 1) & 1, abort)) { failed = true; break; }
+        tc::mma_commit(&bars->q_empty[qs]);  // the Q stage is read
+        // P is in TMEM, and the epilogue has read this buffer's previous O
+        if (!tc::mbar_spin(&bars->p_full[buf], (ns >> 1) & 1, abort) ||
+            !tc::mbar_spin(&bars->o_empty[buf], ((ns >> 1) & 1) ^ 1, abort)) {
+          failed = true;
+          break;
+        }
         tc::tc_fence_after();
         const uint32_t va = ka + C::kKBytes;
         const uint32_t o = tmem + buf * 256 + 128;
@@ -424,17 +449,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       // every MMA issued has completed before TMEM is freed
       if (!tc::mma_drain(&bars->mma_done)) failed = true;
     }
-  } else if (warp <= 9) {
-    // ---------------- softmax + epilogue (two warpgroups) ----------------
-    const int wg = (warp - 2) >> 2;          // tiles j with j % 2 == wg, TMEM buffer wg
+   }
+  } else if (warp < 12) {
+    // ---------------- softmax (two warpgroups) ----------------
+    regs_inc<kRegsSoftmax>();
+    const int wg = (warp - 4) >> 2;          // tiles j with j % 2 == wg, TMEM buffer wg
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
-    const uint32_t sbase = tmem + lane_addr + wg * 256;  // S|P at +0, O at +128
+    const uint32_t sbase = tmem + (uint32_t(quarter * 32) << 16) + wg * 256;  // S|P
     const float sl2 = P.scale * 1.4426950408889634f;
     const int el = row / kGroup, hh = row % kGroup;
     for (int j = wg; tile_of(j) < total; j += 2) {
-      const int d = j % kDesc, qs = j % kQStages;
+      const int d = j % kDesc;
       const uint32_t par = (j >> 1) & 1;
       if (!warp_wait(&bars->d_full[d], (j / kDesc) & 1, abort)) { failed = true; break; }
       const TileDesc& D = bars->desc[d];
@@ -466,22 +492,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       // fp32, two columns at a time: the scaled logits come from packed fp32x2
       // FMAs, the exponentials from the fp32 exp2 (the exp2 unit takes the same
       // time per value in fp32 as in bf16x2, and this loop is bound by issue
-      // slots: summing fp32 values saves widening the bf16 ones, -3 % for the
-      // kernel), and each pair is rounded once to bf16x2 for the P V product
+      // slots: summing fp32 values saves widening the bf16 ones), and each pair
+      // is rounded once to bf16x2 for the P V product
       const uint64_t sl2x2 = f2(sl2, sl2), nmsx2 = f2(-ms, -ms);
       uint64_t lsum[2] = {0, 0};
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t pw[16];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const uint64_t z = fma2((uint64_t(v[q4][x + 1]) << 32) | v[q4][x], sl2x2, nmsx2);
-          const float pa = ex2_f32(__uint_as_float(uint32_t(z)));
-          const float pb = ex2_f32(__uint_as_float(uint32_t(z >> 32)));
-          lsum[(x >> 1) & 1] = add2(lsum[(x >> 1) & 1], f2(pa, pb));
-          pw[x >> 1] = pack_bf16(pa, pb);
+        for (int x8 = 0; x8 < 2; ++x8) {
+          uint32_t pw[8];
+#pragma unroll
+          for (int x = 0; x < 16; x += 2) {
+            const uint32_t* s2 = v[q4] + x8 * 16 + x;
+            const uint64_t z = fma2((uint64_t(s2[1]) << 32) | s2[0], sl2x2, nmsx2);
+            const float pa = ex2_f32(__uint_as_float(uint32_t(z)));
+            const float pb = ex2_f32(__uint_as_float(uint32_t(z >> 32)));
+            lsum[(x >> 1) & 1] = add2(lsum[(x >> 1) & 1], f2(pa, pb));
+            pw[x >> 1] = pack_bf16(pa, pb);
+          }
+          tmem_st8(sbase + q4 * 16 + x8 * 8, pw);  // P columns 16*q4 + 8*x8 ..
         }
-        tmem_st16(sbase + q4 * 16, pw);  // P columns 16*q4.. (S is all in registers)
       }
       const uint64_t lsx = add2(lsum[0], lsum[1]);
       const float l = __uint_as_float(uint32_t(lsx)) + __uint_as_float(uint32_t(lsx >> 32));
@@ -489,61 +519,93 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&bars->p_full[wg]);
-      if (!warp_wait(&bars->o_full[wg], par, abort)) { failed = true; break; }
+      // the row sum to the epilogue (its slot is free once the epilogue has
+      // read the buffer's previous one)
+      if (!warp_wait(&bars->l_empty[wg], par ^ 1, abort)) { failed = true; break; }
+      bars->lsum[wg][row] = l;
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(&bars->l_full[wg]);
+        tc::mbar_arrive(&bars->d_empty[d]);
+      }
+      if (valid) part_lse[(long long)(e0 + el) * kGroup + hh] = ms + __log2f(l);
+    }
+  } else {
+    // ---------------- epilogue: every tile in order ----------------
+    regs_dec<kRegsEpi>();
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+    // Each warp owns 32 consecutive rows (two gathered queries, contiguous in
+    // the entry-ordered partial states) and stores them itself with TMA.  The
+    // staging uses the 128-byte swizzle (16-byte chunk k of a row goes to chunk
+    // k ^ (row % 8)), which the TMA store undoes.
+    uint8_t* wst = obuf + quarter * 8192;
+    // partial states are read once, by the combine: first out of L2
+    const uint64_t o_policy = tc::policy_evict_first();
+    for (int j = 0; tile_of(j) < total; ++j) {
+      const int b = j & 1, d = j % kDesc;
+      const uint32_t par = (j >> 1) & 1;
+      if (!warp_wait(&bars->d_full[d], (j / kDesc) & 1, abort) ||
+          !warp_wait(&bars->l_full[b], par, abort)) {
+        failed = true;
+        break;
+      }
+      const int e0 = bars->desc[d].e0, n = bars->desc[d].n;
+      const float inv = 1.f / bars->lsum[b][row];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->l_empty[b]);
+      if (!warp_wait(&bars->o_full[b], par, abort)) { failed = true; break; }
       tc::tc_fence_after();
-      // Stage the normalised bf16 O row in this tile's Q buffer (bf16 q/k: S is
-      // done with it) or in the warpgroup's staging area (fp8 q/k).  Each warp
-      // owns 32 consecutive rows (two gathered queries, contiguous in the
-      // entry-ordered partial states) and stores them itself.  The staging
-      // uses the 128-byte swizzle (16-byte chunk k of a row goes to chunk
-      // k ^ (row % 8)), so that the row-per-lane writes and the chunk-per-lane
-      // reads both spread over the banks.
-      uint8_t* wst = QK8 ? obuf + wg * C::kOStageBytes + quarter * 8192
-                         : qbuf + qs * C::kQStageBytes + quarter * 8192;
-      const float inv = 1.f / l;
+      // the warp's previous stores have read the staging area
+      if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      __syncwarp();
       const uint64_t invx2 = f2(inv, inv);
-      uint32_t o[4][32];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tc::tmem_ld32(sbase + 128 + q4 * 32, o[q4]);
-      tc::tmem_ld_wait();
-#pragma unroll
+      const uint32_t obase = tmem + lane_addr + b * 256 + 128;
+      // O in four 32-column pieces (the buffer's next P V needs O only after
+      // that buffer's next S and softmax, so the round trips cost nothing)
+#pragma unroll 1
       for (int q4 = 0; q4 < 4; ++q4) {
-        uint8_t* half = wst + (q4 >> 1) * 4096 + lane * 128;
+        uint32_t o[32];
+        tc::tmem_ld32(obase + q4 * 32, o);
+        tc::tmem_ld_wait();
+        if (q4 == 3) {
+          // all of O has been read: the buffer's next P V may overwrite it
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&bars->o_empty[b]);
+        }
+        // columns 32*q4 ..: 64-dim half q4 / 2, 16-byte chunks 4*(q4 % 2) ..
+        uint8_t* hp = wst + (q4 >> 1) * 4096 + lane * 128;
 #pragma unroll
         for (int k8 = 0; k8 < 4; ++k8) {
-          const uint32_t* w8 = o[q4] + 8 * k8;
+          const uint32_t* w8 = o + 8 * k8;
           uint4 u;
           u.x = to_bf16x2(mul2((uint64_t(w8[1]) << 32) | w8[0], invx2));
           u.y = to_bf16x2(mul2((uint64_t(w8[3]) << 32) | w8[2], invx2));
           u.z = to_bf16x2(mul2((uint64_t(w8[5]) << 32) | w8[4], invx2));
           u.w = to_bf16x2(mul2((uint64_t(w8[7]) << 32) | w8[6], invx2));
           const int chunk = (q4 & 1) * 4 + k8;
-          *reinterpret_cast<uint4*>(half + ((chunk ^ (lane & 7)) << 4)) = u;
+          *reinterpret_cast<uint4*>(hp + ((chunk ^ (lane & 7)) << 4)) = u;
         }
       }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&bars->buf_empty[wg]);
-      if (valid) part_lse[(long long)(e0 + el) * kGroup + hh] = ms + __log2f(l);
-      // the warp's rows from the staging area to the partial states with
-      // coalesced 16-byte stores (two 256-byte rows per instruction), streaming
-      // past L2 (the combine reads them once); the load/store units carry them
-      // so that the TMA unit is left to the Q gathers
-      const int nrows = min(32, n * kGroup - quarter * 32);  // 0, 16 or 32
-      uint8_t* gdst = part_o + (size_t(e0) * kGroup + quarter * 32) * 256;
-      for (int it = 0; it < nrows / 2; ++it) {
-        const int r = 2 * it + (lane >> 4), k = lane & 15;
-        const uint4 u = *reinterpret_cast<const uint4*>(wst + (k >> 3) * 4096 + r * 128 +
-                                                        (((k & 7) ^ (r & 7)) << 4));
-        __stcs(reinterpret_cast<uint4*>(gdst + r * 256 + k * 16), u);
-      }
+      tc::fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        // bf16: the staging area is the tile's Q buffer, free again
-        if (!QK8) tc::mbar_arrive(&bars->q_empty[qs]);
+        const int nrows = min(32, n * kGroup - quarter * 32);  // 0, 16 or 32
+        if (nrows > 0) {
+          const CUtensorMap* map = nrows == 32 ? &tmap_o32 : &tmap_o16;
+          const int grow = e0 * kGroup + quarter * 32;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tc::tma_store_2d_hint(map, wst + h * 4096, 64 * h, grow, o_policy);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
         tc::mbar_arrive(&bars->d_empty[d]);
       }
     }
+    // every store has completed before the CTA exits
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   if (failed) {
     bars->abort = 1;
@@ -593,7 +655,7 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
                            cudaStream_t s) {
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo32, mo16;
   const CUtensorMapDataType qk_type =
       P.qk8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const cuuint64_t qk_row = P.qk8 ? 128 : 256;  // bytes of one 128-dim row of q or k
@@ -635,13 +697,27 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  {
+    // partial states: [entries * 16 rows, 128 dims] bf16, stored 16 or 32 rows at a time
+    cuuint64_t dims[2] = {128, cuuint64_t(P.T) * P.Hq * P.K};
+    cuuint64_t strides[1] = {128 * 2};
+    cuuint32_t estr[2] = {1, 1};
+    cuuint32_t box32[2] = {64, 32}, box16[2] = {64, 16};
+    if (enc(&mo32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, part.o, dims, strides, box32, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    if (enc(&mo16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, part.o, dims, strides, box16, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   auto kern = P.qk8 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
   const size_t smem = P.qk8 ? smem_bytes<true>() : smem_bytes<false>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<sm_count(), kThreads, smem, s>>>(mq, mk, mv, P, L, part.lse2, status,
-                                           static_cast<uint8_t*>(part.o));
+  kern<<<sm_count(), kThreads, smem, s>>>(mq, mk, mv, mo32, mo16, P, L, part.lse2, status);
   return cudaGetLastError();
 }
 
