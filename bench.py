@@ -320,8 +320,8 @@ def run_e2e(msa, w, xh, out_h, steps, warmup):
 NCU_TRAFFIC = {
     # stage: (workload, source file, git blob id, bytes per launch)
     "attn": ("prefill_128k", "block_sparse_gqa_04_b200/csrc/attn_tc.cu",
-             "67621afd957179f3b476385ed053fc9aad15f4aa",
-             round((393061632 + 2958702592) * 8327168 / 724992)),
+             "14b66a335fad31600ee1ed6bbb190907efbfc464",
+             round((415465472 + 2956862976) * 8327168 / 724992)),
 }
 
 
