@@ -717,6 +717,19 @@ cudaError_t launch_attn_tc(const Problem& P, const void* q, const void* k, const
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
+  // The warpgroups' setmaxnreg split draws on the registers the CTA is
+  // launched with; a build that gave the kernel fewer than the split adds up
+  // to would leave the softmax warpgroups waiting for registers forever, so
+  // such a build is refused here.
+  static int regs[2] = {0, 0};  // per instantiation, looked up once
+  int& nregs = regs[P.qk8 ? 1 : 0];
+  if (nregs == 0) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    nregs = fa.numRegs;
+  }
+  if (nregs * 4 < kRegsCtl + kRegsEpi + 2 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
   kern<<<sm_count(), kThreads, smem, s>>>(mq, mk, mv, mo32, mo16, P, L, part.lse2, status);
   return cudaGetLastError();
 }

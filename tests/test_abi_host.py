@@ -389,3 +389,25 @@ def test_nvfp4_binding_checks_scales():
         msa.select(codes_q, codes_k, top_k=4,
                    index_scales=(torch.zeros((1, 4, 2, 4), dtype=torch.uint8),
                                  torch.zeros((1, 300, 8), dtype=torch.uint8)))
+
+
+def test_attention_register_split_fits_the_launch(lib):
+    # attn_tc_kernel moves registers between its four warpgroups with
+    # setmaxnreg (96 + 64 + 2 x 176 per thread of a warpgroup), drawing on the
+    # 512 x 128 registers the CTA is launched with: ptxas must give the kernel
+    # exactly 128 registers per thread and spill nothing (the launcher also
+    # refuses a build with fewer).
+    from block_sparse_gqa_04_b200 import build
+    log = open(os.path.join(build.BUILD, "attn_tc.ptxas.txt")).read()
+    src = open(os.path.join(build.CSRC, "attn_tc.cu")).read()
+    m = re.search(r"kRegsCtl = (\d+), kRegsEpi = (\d+), kRegsSoftmax = (\d+);", src)
+    ctl, epi, sm = map(int, m.groups())
+    assert re.search(r"constexpr int kThreads = 512;", src)
+    blocks = re.findall(r"Function properties for \S*attn_tc_kernel\S*\n\s*(\d+) bytes stack frame, "
+                        r"(\d+) bytes spill stores, (\d+) bytes spill loads\n"
+                        r"ptxas info\s*: Used (\d+) registers", log)
+    assert len(blocks) == 2, "both instantiations (bf16 and fp8 q/k)"
+    for stack, st, ld, regs in blocks:
+        assert int(regs) == 128
+        assert int(st) == 0 and int(ld) == 0
+        assert int(regs) * 4 >= ctl + epi + 2 * sm
