@@ -89,7 +89,8 @@ struct Cfg {
 constexpr int kChunk = 8;
 constexpr int kDesc = 6;  // tile descriptors in flight
 
-// What the producer warp tells the MMA warp and the softmax warps about a tile.
+// What the producer warp tells the MMA threads, the softmax and the epilogue
+// warps about a tile.
 struct TileDesc {
   int c, e0, n, flags;     // flags: 1 new list, 2 last tile of its list here, 4 kv stage,
                           // 8 last tile of its parity in the list, 16 kv load parity
@@ -99,6 +100,8 @@ struct TileDesc {
 struct Bars {
   uint64_t kv_full[2], kv_empty[2];
   uint64_t q_full[kMaxQStages], q_empty[kMaxQStages];
+  // per TMEM buffer: S computed, P written, O computed, O read by the
+  // epilogue, row sums written, row sums read
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2], l_full[2], l_empty[2];
   uint64_t d_full[kDesc], d_empty[kDesc];
   TileDesc desc[kDesc];
